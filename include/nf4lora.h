@@ -1,0 +1,199 @@
+/*
+ * nf4lora.h -- C ABI of the NF4-LoRA linear layer library (libnf4lora.so),
+ * hand-written CUDA for NVIDIA B200 (sm_100a).
+ *
+ * The layer is the frozen-base linear of QLoRA:
+ *
+ *     Y  = X . W_hat^T + s . (X . A^T) . B^T,        s = alpha / r
+ *     dX = dY . W_hat  + s . (dY . B) . A
+ *     dA = s . (dY . B)^T . X
+ *     dB = s . dY^T . (X . A^T)
+ *
+ * where W_hat is the bfloat16 dequantisation of a 4-bit NormalFloat (NF4)
+ * encoding of the frozen weight W.  No gradient of W is ever formed.
+ *
+ * Sources: "第 04 篇：QLoRA 原理" (jupiter-lab.pages.dev), cited below as
+ * [QP] with its section numbers; the compassingai.com QLoRA concept page,
+ * cited as [CA] with its headings.
+ *
+ * Conventions common to every entry point
+ * ---------------------------------------
+ * Layout:     row-major.  W and W_hat are [d_out, d_in]; A is [r, d_in];
+ *             B is [d_out, r]; X is [M, d_in]; Y and dY are [M, d_out]
+ *             ([CA] "與原始 LoRA 的技術關係": B in R^{d x r}, A in R^{r x k}).
+ * bfloat16:   passed as uint16_t bit patterns.
+ * Pointers:   every array argument is a DEVICE pointer unless stated, at
+ *             least 16-byte aligned.  The caller owns all memory; the library
+ *             never allocates, frees or synchronises.
+ * Streams:    `stream` is a cudaStream_t (NULL = legacy default stream).  All
+ *             work is enqueued on it; NF4_OK means "enqueued".
+ * Errors:     arguments are checked on the host before anything is enqueued;
+ *             a failed check returns a negative nf4_status and enqueues
+ *             nothing.  A failed launch returns NF4_ERR_CUDA.  The text of
+ *             the last error of the calling thread is available from
+ *             nf4lora_last_error_string().  Kernels bound every wait they
+ *             perform; one that gives up records NF4_ERR_TIMEOUT in a device
+ *             status word that nf4lora_device_status() returns.
+ * Devices:    one device per call (the current one); the kernels are built
+ *             for sm_100a only.
+ */
+#ifndef NF4LORA_H
+#define NF4LORA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    NF4_OK = 0,
+    NF4_ERR_INVALID_ARG = -1,       /* NULL pointer, negative size, bad r or s  */
+    NF4_ERR_UNSUPPORTED_SHAPE = -2, /* d_in % 64 != 0, d_out % 8 != 0, ...     */
+    NF4_ERR_MISALIGNED = -3,        /* a pointer not 16-byte aligned           */
+    NF4_ERR_WORKSPACE = -4,         /* workspace NULL or smaller than required */
+    NF4_ERR_CUDA = -5,              /* a CUDA runtime call or launch failed    */
+    NF4_ERR_TIMEOUT = -6,           /* a kernel gave up a bounded wait         */
+    NF4_ERR_DEVICE = -7             /* current device is not sm_100            */
+} nf4_status;
+
+/* Block sizes of the encoding: 64 weights share one first-level absmax scale
+ * ([QP] §3.4, §5.1); 256 first-level scales share one second-level fp32 scale
+ * ([QP] §5.2). */
+#define NF4_BLOCK_SIZE 64
+#define NF4_DQ_BLOCK_SIZE 256
+
+/*
+ * An NF4 + double-quantised weight ([QP] §2.1 "store the 4-bit indices, the
+ * block scales or their second-level state, and the codebook"; §5.2).
+ * All pointers are device pointers owned by the caller.
+ *   codes       [d_out * d_in / 2] bytes.  Two 4-bit level indices per byte,
+ *               row-major element order, the even element in the high nibble.
+ *               Index j means the j-th NF4 level in ascending order (the table
+ *               of [QP] §4.3: -1, -0.6961928, ..., 0, ..., 0.7229568, 1).
+ *   qscale      [n_b] int8, n_b = d_out * d_in / 64.  Symmetric 8-bit code of
+ *               (absmax_b - mean) / scale2_g, in [-127, 127].
+ *   scale2      [n_g] fp32, n_g = ceil(n_b / 256).  Per group of 256 blocks,
+ *               max |absmax_b - mean|.
+ *   scale_mean  [1] fp32, the mean of all first-level absmax scales.
+ * Restored block scale: s_b = fp32(qscale_b * fp32(scale2_g / 127)) + mean;
+ * weight: w_hat = bf16_rne(fp32(level[code] * s_b))  ([QP] §6.1).
+ */
+typedef struct {
+    int64_t d_out;
+    int64_t d_in;
+    uint8_t* codes;
+    int8_t* qscale;
+    float* scale2;
+    float* scale_mean;
+} nf4_tensor;
+
+/* ---------------------------------------------------------------- sizing */
+
+/* Bytes of one encoded [d_out, d_in] weight when laid out by
+ * nf4_tensor_from_buffer (each part padded to 256 bytes).  The unpadded
+ * storage is n/2 + n_b + 4 n_g + 4 bytes, about 4.127 bits per weight
+ * ([QP] §5.3, §8.1).  Returns 0 for invalid shapes.  Host only. */
+size_t nf4_packed_bytes(int64_t d_out, int64_t d_in);
+
+/* Fill `t` with pointers into one caller-owned device buffer `base` of
+ * `bytes` >= nf4_packed_bytes(d_out, d_in) bytes (256-byte aligned).  Host
+ * only; touches no device memory.  Returns NF4_OK or an error status. */
+int nf4_tensor_from_buffer(nf4_tensor* t, void* base, size_t bytes, int64_t d_out,
+                           int64_t d_in);
+
+/* Workspace (device bytes, 256-byte aligned) that each call needs. */
+size_t nf4_quantize_workspace_bytes(int64_t d_out, int64_t d_in);
+size_t qlora_fwd_workspace_bytes(int64_t M, int64_t d_out, int64_t d_in, int r);
+size_t qlora_bwd_workspace_bytes(int64_t M, int64_t d_out, int64_t d_in, int r);
+
+/* ---------------------------------------------------------------- encode */
+
+/*
+ * nf4_quantize -- encode the fp32 weight W [d_out, d_in] (device) into `out`
+ * (whose pointers and d_out/d_in the caller set, e.g. by
+ * nf4_tensor_from_buffer).
+ *   1. per block of 64 consecutive weights, absmax a_b = max |w|
+ *      ([QP] §3.4, §4.4; [CA] "NF4 量化機制詳解" steps 1-2);
+ *   2. per weight, x = w / a_b (IEEE fp32 division) and the code = number of
+ *      the 15 fp32 midpoints (level_j + level_{j+1}) / 2 strictly below x, i.e.
+ *      the nearest level with ties to the lower one; an all-zero block codes
+ *      every weight as the exact 0 (index 7) ([QP] §3.2, §4.3; [CA] step 3);
+ *   3. pack two codes per byte ([QP] §2.1);
+ *   4. mean = fp32(sum / n_b), the sum of all a_b in fp64 by a fixed pairwise
+ *      tree (adjacent pairs, level by level) ([QP] §5.2);
+ *   5. per group of 256 blocks, scale2 = max |a_b - mean| and
+ *      qscale_b = rint((a_b - mean) / scale2 * 127) ([QP] §5.2, §3.3).
+ * Requirements: d_out >= 1, d_in >= 64, d_in % 64 == 0; W 16-byte aligned;
+ * ws >= nf4_quantize_workspace_bytes(d_out, d_in).  Results are bit-identical
+ * to the stated arithmetic on every run.  Non-finite W is undefined.
+ */
+int nf4_quantize(const float* W, int64_t d_out, int64_t d_in, const nf4_tensor* out,
+                 void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * nf4_dequantize -- W_hat [d_out, d_in] bfloat16 (device) from `w`, with the
+ * bit-exact definition above ([QP] §6.1 double dequantisation, §6.2 BF16
+ * compute dtype).  Materialises the whole weight; the layer calls below never
+ * do.
+ */
+int nf4_dequantize(const nf4_tensor* w, uint16_t* W_hat, void* stream);
+
+/* ---------------------------------------------------------------- layer */
+
+/*
+ * qlora_linear_fwd -- Y [M, d_out] = X . W_hat^T + (s X A^T) . B^T
+ * ([QP] §2.2-§2.3, §6.1-§6.3; [CA] compute graph).
+ *   A [r, d_in], B [d_out, r], X [M, d_in]: bfloat16, device.
+ *   scaling: s (alpha / r, alpha / sqrt(r), ...).
+ *   T_saved: NULL, or [M, r] bfloat16 (device) that receives bf16(s X A^T)
+ *            for reuse by qlora_linear_bwd.
+ * The weight is decoded tile by tile in on-chip memory and never written to
+ * device memory; products accumulate in fp32; Y is rounded to bfloat16.
+ * Requirements: M >= 1, 1 <= r <= 256, r % 8 == 0, d_in % 64 == 0,
+ * d_out % 8 == 0, ws >= qlora_fwd_workspace_bytes(M, d_out, d_in, r).
+ */
+int qlora_linear_fwd(const nf4_tensor* w, const uint16_t* A, const uint16_t* B, int r,
+                     float scaling, const uint16_t* X, int64_t M, uint16_t* Y,
+                     uint16_t* T_saved, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * qlora_linear_bwd -- gradients of the forward above ([QP] §2.4: the frozen
+ * base passes the input gradient but no weight gradient is formed; §6.4:
+ * only the adapters receive gradients):
+ *   dX [M, d_in]  = dY W_hat + s (dY B) A
+ *   dA [r, d_in]  = s (dY B)^T X
+ *   dB [d_out, r] = dY^T T,    T = bf16(s X A^T)  (T_saved, or recomputed
+ *                                                  from X when T_saved is NULL)
+ * dX, dA or dB may be NULL to skip that output (X is then only needed for dA
+ * and for recomputing T).  accumulate_grads = 1 adds the new dA / dB to the
+ * values already in those buffers (gradient accumulation, [QP] §6.4) instead
+ * of overwriting them.  Requirements as for the forward, and
+ * ws >= qlora_bwd_workspace_bytes(M, d_out, d_in, r).
+ */
+int qlora_linear_bwd(const nf4_tensor* w, const uint16_t* A, const uint16_t* B, int r,
+                     float scaling, const uint16_t* X, const uint16_t* T_saved,
+                     const uint16_t* dY, int64_t M, uint16_t* dX, uint16_t* dA,
+                     uint16_t* dB, int accumulate_grads, void* ws, size_t ws_bytes,
+                     void* stream);
+
+/* ---------------------------------------------------------------- status */
+
+/* Text of the last error returned to the calling host thread ("" if none). */
+const char* nf4lora_last_error_string(void);
+
+/* Reads (and clears) the device status word of the current device after
+ * synchronising `stream`: NF4_OK, or NF4_ERR_TIMEOUT if a kernel gave up a
+ * bounded wait since the last call.  Returns NF4_ERR_CUDA if the
+ * synchronisation fails. */
+int nf4lora_device_status(void* stream);
+
+/* Library version, e.g. "nf4lora 0.1.0 sm_100a". */
+const char* nf4lora_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NF4LORA_H */

@@ -1,0 +1,236 @@
+"""Python binding of libnf4lora (the NF4-LoRA linear layer for B200, sm_100a).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of ``lib/libnf4lora.so`` behind the C ABI declared in
+``include/nf4lora.h``.  PyTorch provides device memory and the current CUDA
+stream.  Importing fails loudly if the shared library has not been built
+(``python -m nf4_base_lora_b200.build``); there is no fallback.
+
+Layer (QLoRA frozen-base linear, "第 04 篇：QLoRA 原理" §2.2-§2.4, §6.1-§6.4):
+
+    Y  = X W_hat^T + s (X A^T) B^T
+    dX = dY W_hat + s (dY B) A,   dA = s (dY B)^T X,   dB = s dY^T (X A^T)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "lib", "libnf4lora.so")
+
+NF4_OK = 0
+STATUS_NAMES = {0: "NF4_OK", -1: "NF4_ERR_INVALID_ARG", -2: "NF4_ERR_UNSUPPORTED_SHAPE",
+                -3: "NF4_ERR_MISALIGNED", -4: "NF4_ERR_WORKSPACE", -5: "NF4_ERR_CUDA",
+                -6: "NF4_ERR_TIMEOUT", -7: "NF4_ERR_DEVICE"}
+
+# Every symbol the C ABI exports (include/nf4lora.h), in declaration order.
+ABI_SYMBOLS = ("nf4_packed_bytes", "nf4_tensor_from_buffer", "nf4_quantize_workspace_bytes",
+               "qlora_fwd_workspace_bytes", "qlora_bwd_workspace_bytes", "nf4_quantize",
+               "nf4_dequantize", "qlora_linear_fwd", "qlora_linear_bwd",
+               "nf4lora_last_error_string", "nf4lora_device_status", "nf4lora_version")
+
+
+class Nf4TensorStruct(ctypes.Structure):
+    _fields_ = [("d_out", ctypes.c_int64), ("d_in", ctypes.c_int64),
+                ("codes", ctypes.c_void_p), ("qscale", ctypes.c_void_p),
+                ("scale2", ctypes.c_void_p), ("scale_mean", ctypes.c_void_p)]
+
+
+class Nf4Error(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__("%s (%d): %s" % (STATUS_NAMES.get(status, "?"), status, message))
+        self.status = status
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError("libnf4lora.so is not built (%s); run python -m nf4_base_lora_b200.build"
+                          % LIB_PATH)
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I64, SZ, I, F = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int,
+                        ctypes.c_float)
+    S = ctypes.POINTER(Nf4TensorStruct)
+    sig = {
+        "nf4_packed_bytes": (SZ, [I64, I64]),
+        "nf4_tensor_from_buffer": (I, [S, P, SZ, I64, I64]),
+        "nf4_quantize_workspace_bytes": (SZ, [I64, I64]),
+        "qlora_fwd_workspace_bytes": (SZ, [I64, I64, I64, I]),
+        "qlora_bwd_workspace_bytes": (SZ, [I64, I64, I64, I]),
+        "nf4_quantize": (I, [P, I64, I64, S, P, SZ, P]),
+        "nf4_dequantize": (I, [S, P, P]),
+        "qlora_linear_fwd": (I, [S, P, P, I, F, P, I64, P, P, P, SZ, P]),
+        "qlora_linear_bwd": (I, [S, P, P, I, F, P, P, P, I64, P, P, P, I, P, SZ, P]),
+        "nf4lora_last_error_string": (ctypes.c_char_p, []),
+        "nf4lora_device_status": (I, [P]),
+        "nf4lora_version": (ctypes.c_char_p, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+def _check(status: int) -> None:
+    if status != NF4_OK:
+        raise Nf4Error(status, lib.nf4lora_last_error_string().decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream() -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _bf16(t: torch.Tensor, name: str) -> torch.Tensor:
+    if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+        raise ValueError("%s must be a contiguous bfloat16 CUDA tensor" % name)
+    return t
+
+
+def _workspace(nbytes: int, device) -> Optional[torch.Tensor]:
+    if nbytes == 0:
+        return None
+    # torch's caching allocator returns 512-byte aligned blocks
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+# ---------------------------------------------------------------- sizing
+def nf4_packed_bytes(d_out: int, d_in: int) -> int:
+    return int(lib.nf4_packed_bytes(d_out, d_in))
+
+
+def nf4_quantize_workspace_bytes(d_out: int, d_in: int) -> int:
+    return int(lib.nf4_quantize_workspace_bytes(d_out, d_in))
+
+
+def qlora_fwd_workspace_bytes(M: int, d_out: int, d_in: int, r: int) -> int:
+    return int(lib.qlora_fwd_workspace_bytes(M, d_out, d_in, r))
+
+
+def qlora_bwd_workspace_bytes(M: int, d_out: int, d_in: int, r: int) -> int:
+    return int(lib.qlora_bwd_workspace_bytes(M, d_out, d_in, r))
+
+
+class NF4Tensor:
+    """An encoded weight: one device buffer holding the packed codes, the
+    int8 scale codes, the fp32 group scales and the fp32 mean."""
+
+    def __init__(self, d_out: int, d_in: int, device="cuda", buffer: Optional[torch.Tensor] = None):
+        nbytes = nf4_packed_bytes(d_out, d_in)
+        if nbytes == 0:
+            raise Nf4Error(-2, "unsupported weight shape [%d, %d]" % (d_out, d_in))
+        self.buffer = buffer if buffer is not None else torch.zeros(nbytes, dtype=torch.uint8, device=device)
+        self.struct = Nf4TensorStruct()
+        _check(lib.nf4_tensor_from_buffer(ctypes.byref(self.struct), _ptr(self.buffer),
+                                          self.buffer.numel(), d_out, d_in))
+        self.d_out, self.d_in = d_out, d_in
+
+    def _view(self, attr: str, dtype, count: int) -> torch.Tensor:
+        off = getattr(self.struct, attr) - self.buffer.data_ptr()
+        itemsize = torch.empty((), dtype=dtype).element_size()
+        return self.buffer[off:off + count * itemsize].view(dtype)
+
+    @property
+    def codes(self) -> torch.Tensor:
+        return self._view("codes", torch.uint8, self.d_out * self.d_in // 2)
+
+    @property
+    def qscale(self) -> torch.Tensor:
+        return self._view("qscale", torch.int8, self.d_out * self.d_in // 64)
+
+    @property
+    def scale2(self) -> torch.Tensor:
+        nb = self.d_out * self.d_in // 64
+        return self._view("scale2", torch.float32, (nb + 255) // 256)
+
+    @property
+    def scale_mean(self) -> torch.Tensor:
+        return self._view("scale_mean", torch.float32, 1)
+
+
+# ---------------------------------------------------------------- entry points
+def nf4_quantize(W: torch.Tensor, out: Optional[NF4Tensor] = None) -> NF4Tensor:
+    """Encode fp32 W [d_out, d_in] (CUDA) to NF4 + double-quantised scales."""
+    if W.dtype != torch.float32 or not W.is_cuda or not W.is_contiguous() or W.dim() != 2:
+        raise ValueError("W must be a contiguous 2-D float32 CUDA tensor")
+    d_out, d_in = W.shape
+    out = out if out is not None else NF4Tensor(d_out, d_in, W.device)
+    ws = _workspace(nf4_quantize_workspace_bytes(d_out, d_in), W.device)
+    _check(lib.nf4_quantize(_ptr(W), d_out, d_in, ctypes.byref(out.struct), _ptr(ws),
+                            0 if ws is None else ws.numel(), _stream()))
+    return out
+
+
+def nf4_dequantize(w: NF4Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Materialise W_hat [d_out, d_in] in bfloat16."""
+    out = out if out is not None else torch.empty((w.d_out, w.d_in), dtype=torch.bfloat16,
+                                                  device=w.buffer.device)
+    _check(lib.nf4_dequantize(ctypes.byref(w.struct), _ptr(out), _stream()))
+    return out
+
+
+def qlora_linear_fwd(w: NF4Tensor, A: torch.Tensor, B: torch.Tensor, scaling: float, X: torch.Tensor,
+                     save_t: bool = True, Y: Optional[torch.Tensor] = None,
+                     workspace: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Y = X W_hat^T + s (X A^T) B^T.  Returns (Y, T) with T = bf16(s X A^T)
+    (or None when save_t is False)."""
+    _bf16(A, "A"), _bf16(B, "B"), _bf16(X, "X")
+    r = A.shape[0]
+    M = X.shape[0]
+    Y = Y if Y is not None else torch.empty((M, w.d_out), dtype=torch.bfloat16, device=X.device)
+    T = torch.empty((M, r), dtype=torch.bfloat16, device=X.device) if save_t else None
+    need = qlora_fwd_workspace_bytes(M, w.d_out, w.d_in, r)
+    ws = workspace if workspace is not None else _workspace(need, X.device)
+    _check(lib.qlora_linear_fwd(ctypes.byref(w.struct), _ptr(A), _ptr(B), r, ctypes.c_float(scaling),
+                                _ptr(X), M, _ptr(Y), _ptr(T), _ptr(ws), 0 if ws is None else ws.numel(),
+                                _stream()))
+    return Y, T
+
+
+def qlora_linear_bwd(w: NF4Tensor, A: torch.Tensor, B: torch.Tensor, scaling: float,
+                     X: Optional[torch.Tensor], T: Optional[torch.Tensor], dY: torch.Tensor,
+                     need_dx: bool = True, need_da: bool = True, need_db: bool = True,
+                     dA: Optional[torch.Tensor] = None, dB: Optional[torch.Tensor] = None,
+                     accumulate: bool = False, dX: Optional[torch.Tensor] = None,
+                     workspace: Optional[torch.Tensor] = None):
+    """Returns (dX, dA, dB); an output not requested is None.  With
+    accumulate=True the gradients are added into the given dA / dB."""
+    _bf16(A, "A"), _bf16(B, "B"), _bf16(dY, "dY")
+    r = A.shape[0]
+    M = dY.shape[0]
+    dev = dY.device
+    if need_dx and dX is None:
+        dX = torch.empty((M, w.d_in), dtype=torch.bfloat16, device=dev)
+    if need_da and dA is None:
+        dA = torch.zeros((r, w.d_in), dtype=torch.bfloat16, device=dev)
+    if need_db and dB is None:
+        dB = torch.zeros((w.d_out, r), dtype=torch.bfloat16, device=dev)
+    dX = dX if need_dx else None
+    dA = dA if need_da else None
+    dB = dB if need_db else None
+    need = qlora_bwd_workspace_bytes(M, w.d_out, w.d_in, r)
+    ws = workspace if workspace is not None else _workspace(need, dev)
+    _check(lib.qlora_linear_bwd(ctypes.byref(w.struct), _ptr(A), _ptr(B), r, ctypes.c_float(scaling),
+                                _ptr(X), _ptr(T), _ptr(dY), M, _ptr(dX), _ptr(dA), _ptr(dB),
+                                1 if accumulate else 0, _ptr(ws), 0 if ws is None else ws.numel(),
+                                _stream()))
+    return dX, dA, dB
+
+
+def device_status() -> None:
+    """Raise Nf4Error(NF4_ERR_TIMEOUT) if a kernel abandoned a bounded wait."""
+    _check(lib.nf4lora_device_status(_stream()))
+
+
+def version() -> str:
+    return lib.nf4lora_version().decode()

@@ -1,0 +1,401 @@
+// Host orchestration of the NF4-LoRA linear layer on the tcgen05 engine.
+//
+// Forward   ("第 04 篇：QLoRA 原理" §6.1-§6.3):
+//   1. T = bf16(s X A^T)                       LoRA down: tcgen05, split-K
+//   2. Y = X W_hat^T + T B^T                    fused dequant-GEMM, LoRA up as
+//                                               extension k-steps of the same
+//                                               accumulator
+// Backward  (§2.4: input gradient through the frozen base; no dW):
+//   1. V = bf16(s dY B)                         tcgen05, split-K over d_out
+//   2. dX = dY W_hat + V A                      fused dequant-GEMM (MN-major
+//                                               decode of the same codes)
+//   3. dB = dY^T T,  dA = V^T X                 tcgen05, split over tokens,
+//                                               deterministic fixed-order sum
+// Few tokens (M <= 16) run the fused GEMMs "swapped": weight rows fill the
+// 128-wide MMA M and tokens the N = 16 side, split-K over all SMs, so the
+// weight stream (4.127 bits per weight) sets the pace.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+
+#include "gemm.cuh"
+#include "layer.h"
+
+namespace nf4lora {
+
+// ------------------------------------------------------------------ tensor maps
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// bf16 matrix [outer, inner] with row stride ld (elements), 128-byte swizzle,
+// box {64, box_outer}.
+static bool map_bf16(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t ld,
+                     uint32_t box_outer) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {ld * 2};
+    cuuint32_t box[2] = {64, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Packed NF4 codes viewed as bytes [d_out, d_in / 2], box {box_inner bytes, box_outer rows}.
+static bool map_codes(CUtensorMap* m, const uint8_t* codes, int64_t d_out, int64_t d_in,
+                      uint32_t box_inner, uint32_t box_outer) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(d_in / 2), static_cast<cuuint64_t>(d_out)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(d_in / 2)};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ launch
+template <int BN, int ASRC, int BSRC, int AE, int BE, int EPI>
+static cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& ae,
+                          const CUtensorMap& be, const GemmArgs& args, dim3 grid, cudaStream_t st) {
+    using C = GemmConfig<BN, ASRC, BSRC, AE, BE, EPI>;
+    auto kern = k_gemm<BN, ASRC, BSRC, AE, BE, EPI>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, C::kThreads, C::kSmemBytes, st>>>(a, b, ae, be, args);
+    return cudaGetLastError();
+}
+
+// fixed-order sum over split-K slices: out[r, c] = bf16(alpha * sum_z part[z]) (+ out)
+__global__ void k_reduce_splits(const float* __restrict__ part, int splits, int64_t slice, int rows,
+                                int cols, int64_t ldp, float alpha, uint16_t* __restrict__ out,
+                                int64_t ldo, uint16_t* __restrict__ out2, int64_t ldo2, int out2_cols,
+                                int accumulate) {
+    const int64_t total = static_cast<int64_t>(rows) * cols;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t r = i / cols, c = i % cols;
+        const float* p = part + r * ldp + c;
+        float acc = 0.0f;
+        for (int z = 0; z < splits; ++z) acc += p[z * slice];
+        const float v = acc * alpha;
+        float o = v;
+        if (accumulate) o += bf16_bits_to_float(out[r * ldo + c]);
+        __nv_bfloat16 h = __float2bfloat16_rn(o);
+        out[r * ldo + c] = *reinterpret_cast<uint16_t*>(&h);
+        if (out2 != nullptr && c < out2_cols) {
+            __nv_bfloat16 h2 = __float2bfloat16_rn(v);
+            out2[r * ldo2 + c] = *reinterpret_cast<uint16_t*>(&h2);
+        }
+    }
+}
+
+static cudaError_t reduce(const float* part, int splits, int64_t slice, int rows, int cols, int64_t ldp,
+                          float alpha, uint16_t* out, int64_t ldo, uint16_t* out2, int64_t ldo2,
+                          int out2_cols, int accumulate, int num_sms, cudaStream_t st) {
+    const int64_t total = static_cast<int64_t>(rows) * cols;
+    int64_t grid = (total + 255) / 256;
+    grid = std::min<int64_t>(grid, int64_t(num_sms) * 8);
+    if (grid < 1) grid = 1;
+    k_reduce_splits<<<static_cast<unsigned>(grid), 256, 0, st>>>(part, splits, slice, rows, cols, ldp, alpha,
+                                                                 out, ldo, out2, ldo2, out2_cols, accumulate);
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ split sizing
+struct Split {
+    int splits;
+    int k_per_split;
+};
+
+// Split k_steps over grid.z so that tiles * splits fills about `target` CTAs,
+// each split keeping at least `min_steps` k-steps; never leaves a split empty.
+static Split choose_split(int tiles, int k_steps, int target, int min_steps) {
+    int s = std::max(1, target / std::max(1, tiles));
+    s = std::min(s, std::max(1, k_steps / std::max(1, min_steps)));
+    int kps = (k_steps + s - 1) / s;
+    s = (k_steps + kps - 1) / kps;
+    return {s, kps};
+}
+
+static inline int64_t align256(int64_t b) { return (b + 255) & ~int64_t(255); }
+static inline int round64(int r) { return (r + 63) / 64 * 64; }
+static inline int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
+
+// partial-buffer sizes (floats) of each split-K GEMM, with the split it will use
+static int64_t down_part_floats(int64_t M, int64_t K, int r64, int num_sms, Split* sp) {
+    Split s = choose_split(ceil_div(M, 128), ceil_div(K, 64), num_sms, 4);
+    if (sp) *sp = s;
+    return int64_t(s.splits) * M * r64;
+}
+
+static constexpr int kSmallM = 16;
+
+// ------------------------------------------------------------------ layer ops
+struct Maps {
+    CUtensorMap a, b, ae, be;
+    Maps() { std::memset(this, 0, sizeof(*this)); }
+};
+
+template <int EPI, int ASRC, int BSRC>
+static cudaError_t launch_lora_gemm(int bn, const Maps& m, const GemmArgs& args, dim3 grid, cudaStream_t st) {
+    switch (bn) {
+        case 64: return launch<64, ASRC, BSRC, 0, 0, EPI>(m.a, m.b, m.ae, m.be, args, grid, st);
+        case 128: return launch<128, ASRC, BSRC, 0, 0, EPI>(m.a, m.b, m.ae, m.be, args, grid, st);
+        default: return launch<256, ASRC, BSRC, 0, 0, EPI>(m.a, m.b, m.ae, m.be, args, grid, st);
+    }
+}
+
+static int bn_for(int r64) { return r64 <= 64 ? 64 : (r64 <= 128 ? 128 : 256); }
+
+// T_pad[M, r64] = bf16(s X A^T) (zero columns beyond r); optional T_saved[M, r].
+static int lora_down(const LayerCtx& c, const uint16_t* A, int r, float s, const uint16_t* X, int64_t M,
+                     uint16_t* T_pad, uint16_t* T_saved, float* part) {
+    const int r64 = round64(r), bn = bn_for(r64);
+    Maps m;
+    if (!map_bf16(&m.a, X, c.d_in, M, c.d_in, 128) || !map_bf16(&m.b, A, c.d_in, r, c.d_in, bn))
+        return -1;
+    Split sp;
+    down_part_floats(M, c.d_in, r64, c.num_sms, &sp);
+    GemmArgs g{};
+    g.rows = static_cast<int>(M);
+    g.cols = r64;
+    g.k_main = ceil_div(c.d_in, 64);
+    g.k_per_split = sp.k_per_split;
+    g.part = part;
+    g.ldp = r64;
+    g.part_slice = M * r64;
+    dim3 grid(ceil_div(M, 128), 1, sp.splits);
+    if (launch_lora_gemm<EPI_F32_PART, SRC_TMA_K, SRC_TMA_K>(bn, m, g, grid, c.stream) != cudaSuccess) return -2;
+    if (reduce(part, sp.splits, M * r64, static_cast<int>(M), r64, r64, s, T_pad, r64, T_saved, r, r, 0,
+               c.num_sms, c.stream) != cudaSuccess)
+        return -2;
+    return 0;
+}
+
+int64_t fwd_workspace_bytes(int64_t M, int64_t d_out, int64_t d_in, int r, int num_sms) {
+    const int r64 = round64(r);
+    int64_t part = down_part_floats(M, d_in, r64, num_sms, nullptr);
+    if (M <= kSmallM) {
+        Split s = choose_split(ceil_div(d_out, 128), ceil_div(d_in, 64), 2 * num_sms, 4);
+        part = std::max<int64_t>(part, int64_t(s.splits) * M * d_out);
+    }
+    return align256(M * r64 * 2) + align256(part * 4);
+}
+
+int layer_fwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, float s, const uint16_t* X,
+              int64_t M, uint16_t* Y, uint16_t* T_saved, uint8_t* ws) {
+    const int r64 = round64(r);
+    uint16_t* T_pad = reinterpret_cast<uint16_t*>(ws);
+    float* part = reinterpret_cast<float*>(ws + align256(M * r64 * 2));
+    int rc = lora_down(c, A, r, s, X, M, T_pad, T_saved, part);
+    if (rc) return rc;
+    Maps m;
+    GemmArgs g{};
+    g.qscale = c.qscale;
+    g.scale2 = c.scale2;
+    g.scale_mean = c.scale_mean;
+    g.w_rows = c.d_out;
+    g.w_blocks_per_row = c.d_in / 64;
+    g.k_main = ceil_div(c.d_in, 64);
+    g.k_ext = r64 / 64;
+    g.alpha = 1.0f;
+    if (M <= kSmallM) {
+        // swapped: D[n, m] = W_hat[n, :] . X[m, :] + B[n, :] . T[m, :]
+        if (!map_codes(&m.a, c.codes, c.d_out, c.d_in, 32, 128) || !map_bf16(&m.b, X, c.d_in, M, c.d_in, 16) ||
+            !map_bf16(&m.ae, B, r, c.d_out, r, 128) || !map_bf16(&m.be, T_pad, r64, M, r64, 16))
+            return -1;
+        const int tiles = ceil_div(c.d_out, 128);
+        Split sp = choose_split(tiles, g.k_main, 2 * c.num_sms, 4);
+        g.rows = static_cast<int>(c.d_out);
+        g.cols = static_cast<int>(M);
+        g.k_per_split = sp.k_per_split;
+        g.part = part;
+        g.ldp = c.d_out;
+        g.part_slice = M * c.d_out;
+        dim3 grid(tiles, 1, sp.splits);
+        if (launch<16, SRC_DEC_K, SRC_TMA_K, 0, 0, EPI_F32_PART_T>(m.a, m.b, m.ae, m.be, g, grid, c.stream) !=
+            cudaSuccess)
+            return -2;
+        if (reduce(part, sp.splits, M * c.d_out, static_cast<int>(M), static_cast<int>(c.d_out), c.d_out, 1.0f, Y,
+                   c.d_out, nullptr, 0, 0, 0, c.num_sms, c.stream) != cudaSuccess)
+            return -2;
+        return 0;
+    }
+    if (!map_bf16(&m.a, X, c.d_in, M, c.d_in, 128) || !map_codes(&m.b, c.codes, c.d_out, c.d_in, 32, 256) ||
+        !map_bf16(&m.ae, T_pad, r64, M, r64, 128) || !map_bf16(&m.be, B, r, c.d_out, r, 256))
+        return -1;
+    g.rows = static_cast<int>(M);
+    g.cols = static_cast<int>(c.d_out);
+    g.k_per_split = g.k_main;
+    g.out = Y;
+    g.ldo = c.d_out;
+    dim3 grid(ceil_div(M, 128), ceil_div(c.d_out, 256), 1);
+    if (launch<256, SRC_TMA_K, SRC_DEC_K, 0, 0, EPI_BF16>(m.a, m.b, m.ae, m.be, g, grid, c.stream) != cudaSuccess)
+        return -2;
+    return 0;
+}
+
+int64_t bwd_workspace_bytes(int64_t M, int64_t d_out, int64_t d_in, int r, int num_sms) {
+    const int r64 = round64(r);
+    int64_t part = down_part_floats(M, d_in, r64, num_sms, nullptr);
+    // V = s dY B: split over d_out
+    Split sv = choose_split(ceil_div(M, 128), ceil_div(d_out, 64), num_sms, 4);
+    part = std::max<int64_t>(part, int64_t(sv.splits) * M * r64);
+    // dB, dA: split over tokens
+    Split sb = choose_split(ceil_div(d_out, 128), ceil_div(M, 64), num_sms, 4);
+    part = std::max<int64_t>(part, int64_t(sb.splits) * d_out * r64);
+    Split sa = choose_split(ceil_div(d_in, 128), ceil_div(M, 64), num_sms, 4);
+    part = std::max<int64_t>(part, int64_t(sa.splits) * d_in * r64);
+    if (M <= kSmallM) {
+        Split sx = choose_split(ceil_div(d_in, 128), ceil_div(d_out, 64), 2 * num_sms, 4);
+        part = std::max<int64_t>(part, int64_t(sx.splits) * M * d_in);
+    }
+    return 2 * align256(M * r64 * 2) + align256(part * 4);
+}
+
+int layer_bwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, float s, const uint16_t* X,
+              const uint16_t* T_saved, const uint16_t* dY, int64_t M, uint16_t* dX, uint16_t* dA,
+              uint16_t* dB, int accumulate, uint8_t* ws) {
+    const int r64 = round64(r), bn = bn_for(r64);
+    uint16_t* V_pad = reinterpret_cast<uint16_t*>(ws);
+    uint16_t* T_pad = reinterpret_cast<uint16_t*>(ws + align256(M * r64 * 2));
+    float* part = reinterpret_cast<float*>(ws + 2 * align256(M * r64 * 2));
+    int rc;
+
+    // ---- V = bf16(s dY B): D[m, j] = sum_n dY[m, n] B[n, j]
+    if (dX != nullptr || dA != nullptr) {
+        Maps m;
+        if (!map_bf16(&m.a, dY, c.d_out, M, c.d_out, 128) || !map_bf16(&m.b, B, r, c.d_out, r, 64)) return -1;
+        Split sp = choose_split(ceil_div(M, 128), ceil_div(c.d_out, 64), c.num_sms, 4);
+        GemmArgs g{};
+        g.rows = static_cast<int>(M);
+        g.cols = r64;
+        g.k_main = ceil_div(c.d_out, 64);
+        g.k_per_split = sp.k_per_split;
+        g.part = part;
+        g.ldp = r64;
+        g.part_slice = M * r64;
+        dim3 grid(ceil_div(M, 128), 1, sp.splits);
+        if (launch_lora_gemm<EPI_F32_PART, SRC_TMA_K, SRC_TMA_MN>(bn, m, g, grid, c.stream) != cudaSuccess) return -2;
+        if (reduce(part, sp.splits, M * r64, static_cast<int>(M), r64, r64, s, V_pad, r64, nullptr, 0, 0, 0,
+                   c.num_sms, c.stream) != cudaSuccess)
+            return -2;
+    }
+
+    // ---- dX = dY W_hat + V A
+    if (dX != nullptr) {
+        Maps m;
+        GemmArgs g{};
+        g.qscale = c.qscale;
+        g.scale2 = c.scale2;
+        g.scale_mean = c.scale_mean;
+        g.w_rows = c.d_out;
+        g.w_blocks_per_row = c.d_in / 64;
+        g.k_main = ceil_div(c.d_out, 64);
+        g.k_ext = r64 / 64;
+        g.alpha = 1.0f;
+        if (M <= kSmallM) {
+            // swapped: D[k, m] = sum_n W_hat[n, k] dY[m, n] + sum_j A[j, k] V[m, j]
+            if (!map_codes(&m.a, c.codes, c.d_out, c.d_in, 64, 64) || !map_bf16(&m.b, dY, c.d_out, M, c.d_out, 16) ||
+                !map_bf16(&m.ae, A, c.d_in, r, c.d_in, 64) || !map_bf16(&m.be, V_pad, r64, M, r64, 16))
+                return -1;
+            const int tiles = ceil_div(c.d_in, 128);
+            Split sp = choose_split(tiles, g.k_main, 2 * c.num_sms, 4);
+            g.rows = static_cast<int>(c.d_in);
+            g.cols = static_cast<int>(M);
+            g.k_per_split = sp.k_per_split;
+            g.part = part;
+            g.ldp = c.d_in;
+            g.part_slice = M * c.d_in;
+            dim3 grid(tiles, 1, sp.splits);
+            if (launch<16, SRC_DEC_MN, SRC_TMA_K, 1, 0, EPI_F32_PART_T>(m.a, m.b, m.ae, m.be, g, grid, c.stream) !=
+                cudaSuccess)
+                return -2;
+            if (reduce(part, sp.splits, M * c.d_in, static_cast<int>(M), static_cast<int>(c.d_in), c.d_in, 1.0f, dX,
+                       c.d_in, nullptr, 0, 0, 0, c.num_sms, c.stream) != cudaSuccess)
+                return -2;
+        } else {
+            if (!map_bf16(&m.a, dY, c.d_out, M, c.d_out, 128) || !map_codes(&m.b, c.codes, c.d_out, c.d_in, 128, 64) ||
+                !map_bf16(&m.ae, V_pad, r64, M, r64, 128) || !map_bf16(&m.be, A, c.d_in, r, c.d_in, 64))
+                return -1;
+            g.rows = static_cast<int>(M);
+            g.cols = static_cast<int>(c.d_in);
+            g.k_per_split = g.k_main;
+            g.out = dX;
+            g.ldo = c.d_in;
+            dim3 grid(ceil_div(M, 128), ceil_div(c.d_in, 256), 1);
+            if (launch<256, SRC_TMA_K, SRC_DEC_MN, 0, 1, EPI_BF16>(m.a, m.b, m.ae, m.be, g, grid, c.stream) !=
+                cudaSuccess)
+                return -2;
+        }
+    }
+
+    // ---- dB = dY^T T: D[n, j] = sum_m dY[m, n] T[m, j]
+    if (dB != nullptr) {
+        const uint16_t* T = T_saved;
+        int64_t ldt = r;
+        if (T == nullptr) {
+            rc = lora_down(c, A, r, s, X, M, T_pad, nullptr, part);
+            if (rc) return rc;
+            T = T_pad;
+            ldt = r64;
+        }
+        Maps m;
+        if (!map_bf16(&m.a, dY, c.d_out, M, c.d_out, 64) || !map_bf16(&m.b, T, ldt, M, ldt, 64)) return -1;
+        Split sp = choose_split(ceil_div(c.d_out, 128), ceil_div(M, 64), c.num_sms, 4);
+        GemmArgs g{};
+        g.rows = static_cast<int>(c.d_out);
+        g.cols = r64;
+        g.k_main = ceil_div(M, 64);
+        g.k_per_split = sp.k_per_split;
+        g.part = part;
+        g.ldp = r64;
+        g.part_slice = c.d_out * r64;
+        dim3 grid(ceil_div(c.d_out, 128), 1, sp.splits);
+        if (launch_lora_gemm<EPI_F32_PART, SRC_TMA_MN, SRC_TMA_MN>(bn, m, g, grid, c.stream) != cudaSuccess) return -2;
+        if (reduce(part, sp.splits, c.d_out * r64, static_cast<int>(c.d_out), r, r64, 1.0f, dB, r, nullptr, 0, 0,
+                   accumulate, c.num_sms, c.stream) != cudaSuccess)
+            return -2;
+    }
+
+    // ---- dA = V^T X: D[k, j] = sum_m X[m, k] V[m, j], stored transposed
+    if (dA != nullptr) {
+        Maps m;
+        if (!map_bf16(&m.a, X, c.d_in, M, c.d_in, 64) || !map_bf16(&m.b, V_pad, r64, M, r64, 64)) return -1;
+        Split sp = choose_split(ceil_div(c.d_in, 128), ceil_div(M, 64), c.num_sms, 4);
+        GemmArgs g{};
+        g.rows = static_cast<int>(c.d_in);
+        g.cols = r64;
+        g.k_main = ceil_div(M, 64);
+        g.k_per_split = sp.k_per_split;
+        g.part = part;
+        g.ldp = c.d_in;
+        g.part_slice = int64_t(r64) * c.d_in;
+        dim3 grid(ceil_div(c.d_in, 128), 1, sp.splits);
+        if (launch_lora_gemm<EPI_F32_PART_T, SRC_TMA_MN, SRC_TMA_MN>(bn, m, g, grid, c.stream) != cudaSuccess)
+            return -2;
+        if (reduce(part, sp.splits, int64_t(r64) * c.d_in, r, static_cast<int>(c.d_in), c.d_in, 1.0f, dA, c.d_in,
+                   nullptr, 0, 0, accumulate, c.num_sms, c.stream) != cudaSuccess)
+            return -2;
+    }
+    return 0;
+}
+
+}  // namespace nf4lora

@@ -1,0 +1,116 @@
+"""GPU parity of the fused NF4-LoRA linear layer (forward and backward)
+against the fp64 oracle, on seeded inputs at sizes that span several tiles
+and ragged tails, for both the few-token (M <= 16) and the many-token paths."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from parity import assert_close
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def nf():
+    import nf4_base_lora_b200 as nf
+    return nf
+
+
+def setup(nf, d_out, d_in, m, r, alpha=16.0, b_std=0.05, outliers=True, index=0):
+    c = workloads.linear_case(d_out, d_in, m, r, alpha, outliers=outliers, index=index, b_std=b_std)
+    qt = oracle.quantize(c.W)
+    W_hat = oracle.dequantize(qt, c.W.shape)
+    w = nf.nf4_quantize(torch.from_numpy(c.W).cuda())
+    dev = {k: getattr(c, k).cuda() for k in ("A", "B", "X", "dY")}
+    return c, W_hat, w, dev
+
+
+CASES = [
+    # (d_out, d_in, M, r)
+    (128, 64, 1, 8),
+    (256, 512, 4, 16),
+    (384, 320, 16, 64),
+    (136, 192, 3, 8),         # ragged d_out vs the 128-row tile
+    (512, 512, 16, 8),
+    (256, 256, 17, 16),       # first many-token size
+    (264, 320, 130, 64),      # ragged tokens and d_out
+    (512, 768, 300, 128),
+    (1024, 512, 256, 24),
+    (384, 1024, 200, 192),
+]
+
+
+@pytest.mark.parametrize("d_out,d_in,m,r", CASES)
+def test_forward_matches_oracle(nf, d_out, d_in, m, r):
+    c, W_hat, w, dev = setup(nf, d_out, d_in, m, r)
+    Y, T = nf.qlora_linear_fwd(w, dev["A"], dev["B"], c.scaling, dev["X"])
+    torch.cuda.synchronize()
+    nf.device_status()
+    Y_ref, T_ref = oracle.forward(W_hat, c.A, c.B, c.X, c.scaling)
+    assert_close(Y, Y_ref, "Y")
+    assert_close(T, T_ref, "T")
+
+
+@pytest.mark.parametrize("d_out,d_in,m,r", CASES)
+def test_backward_matches_oracle(nf, d_out, d_in, m, r):
+    c, W_hat, w, dev = setup(nf, d_out, d_in, m, r)
+    _, T = nf.qlora_linear_fwd(w, dev["A"], dev["B"], c.scaling, dev["X"])
+    dX, dA, dB = nf.qlora_linear_bwd(w, dev["A"], dev["B"], c.scaling, dev["X"], T, dev["dY"])
+    torch.cuda.synchronize()
+    nf.device_status()
+    dX_ref, dA_ref, dB_ref = oracle.backward(W_hat, c.A, c.B, c.X, c.dY, c.scaling)
+    assert_close(dX, dX_ref, "dX")
+    assert_close(dA, dA_ref, "dA")
+    assert_close(dB, dB_ref, "dB")
+
+
+def test_backward_recomputes_t_when_not_saved(nf):
+    c, W_hat, w, dev = setup(nf, 256, 256, 40, 16)
+    dX, dA, dB = nf.qlora_linear_bwd(w, dev["A"], dev["B"], c.scaling, dev["X"], None, dev["dY"])
+    torch.cuda.synchronize()
+    dX_ref, dA_ref, dB_ref = oracle.backward(W_hat, c.A, c.B, c.X, c.dY, c.scaling)
+    assert_close(dB, dB_ref, "dB")
+    assert_close(dA, dA_ref, "dA")
+    assert_close(dX, dX_ref, "dX")
+
+
+def test_zero_b_gives_base_product_and_zero_da(nf):
+    c, W_hat, w, dev = setup(nf, 256, 512, 64, 16)
+    B0 = torch.zeros_like(dev["B"])
+    Y, T = nf.qlora_linear_fwd(w, dev["A"], B0, c.scaling, dev["X"])
+    dX, dA, dB = nf.qlora_linear_bwd(w, dev["A"], B0, c.scaling, dev["X"], T, dev["dY"])
+    torch.cuda.synchronize()
+    W_dev = nf.nf4_dequantize(w)
+    ref = (dev["X"].float() @ W_dev.float().t())
+    assert_close(Y, ref, "Y (B = 0)")
+    assert torch.count_nonzero(dA) == 0
+    assert_close(dX, dev["dY"].float() @ W_dev.float(), "dX (B = 0)")
+
+
+def test_accumulate_and_skipped_outputs(nf):
+    c, W_hat, w, dev = setup(nf, 256, 256, 32, 8)
+    _, T = nf.qlora_linear_fwd(w, dev["A"], dev["B"], c.scaling, dev["X"])
+    dX, dA, dB = nf.qlora_linear_bwd(w, dev["A"], dev["B"], c.scaling, dev["X"], T, dev["dY"])
+    _, dA2, dB2 = nf.qlora_linear_bwd(w, dev["A"], dev["B"], c.scaling, dev["X"], T, dev["dY"],
+                                      need_dx=False, dA=dA.clone(), dB=dB.clone(), accumulate=True)
+    only_dx, none_a, none_b = nf.qlora_linear_bwd(w, dev["A"], dev["B"], c.scaling, None, None, dev["dY"],
+                                                  need_da=False, need_db=False)
+    torch.cuda.synchronize()
+    assert none_a is None and none_b is None
+    assert torch.equal(only_dx, dX)
+    assert_close(dA2, 2 * dA.float(), "dA accumulated")
+    assert_close(dB2, 2 * dB.float(), "dB accumulated")
+
+
+def test_layer_is_deterministic(nf):
+    c, W_hat, w, dev = setup(nf, 512, 512, 256, 64)
+    outs = []
+    for _ in range(3):
+        Y, T = nf.qlora_linear_fwd(w, dev["A"], dev["B"], c.scaling, dev["X"])
+        g = nf.qlora_linear_bwd(w, dev["A"], dev["B"], c.scaling, dev["X"], T, dev["dY"])
+        outs.append([Y.clone(), T.clone()] + [t.clone() for t in g])
+    for o in outs[1:]:
+        for a, b in zip(outs[0], o):
+            assert torch.equal(a, b)
