@@ -147,16 +147,20 @@ int nf4_dequantize(const nf4_tensor* w, uint16_t* W_hat, void* stream);
  * ([QP] §2.2-§2.3, §6.1-§6.3; [CA] compute graph).
  *   A [r, d_in], B [d_out, r], X [M, d_in]: bfloat16, device.
  *   scaling: s (alpha / r, alpha / sqrt(r), ...).
- *   T_saved: NULL, or [M, r] bfloat16 (device) that receives bf16(s X A^T)
- *            for reuse by qlora_linear_bwd.
+ *   T_saved: NULL, or [M, r] fp32 (device) that receives T = s X A^T (fp32
+ *            accumulation) for reuse by qlora_linear_bwd.
  * The weight is decoded tile by tile in on-chip memory and never written to
- * device memory; products accumulate in fp32; Y is rounded to bfloat16.
+ * device memory; products accumulate in fp32; Y is rounded to bfloat16.  The
+ * rank-r intermediate T enters the LoRA-up product as a pair of bfloat16
+ * arrays hi = bf16(T), lo = bf16(T - hi) (about 16 significant bits), so the
+ * adapter branch is not limited to bfloat16 precision ([QP] §6.3: the adapter
+ * dtype may be wider than the base compute dtype).
  * Requirements: M >= 1, 1 <= r <= 256, r % 8 == 0, d_in % 64 == 0,
  * d_out % 8 == 0, ws >= qlora_fwd_workspace_bytes(M, d_out, d_in, r).
  */
 int qlora_linear_fwd(const nf4_tensor* w, const uint16_t* A, const uint16_t* B, int r,
                      float scaling, const uint16_t* X, int64_t M, uint16_t* Y,
-                     uint16_t* T_saved, void* ws, size_t ws_bytes, void* stream);
+                     float* T_saved, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * qlora_linear_bwd -- gradients of the forward above ([QP] §2.4: the frozen
@@ -164,8 +168,10 @@ int qlora_linear_fwd(const nf4_tensor* w, const uint16_t* A, const uint16_t* B, 
  * only the adapters receive gradients):
  *   dX [M, d_in]  = dY W_hat + s (dY B) A
  *   dA [r, d_in]  = s (dY B)^T X
- *   dB [d_out, r] = dY^T T,    T = bf16(s X A^T)  (T_saved, or recomputed
- *                                                  from X when T_saved is NULL)
+ *   dB [d_out, r] = dY^T T,    T = s X A^T   (fp32 T_saved, or recomputed
+ *                                             from X when T_saved is NULL)
+ * The rank-r intermediates T and V = s dY B enter the tensor-core products
+ * as bfloat16 hi/lo pairs, as in the forward.
  * dX, dA or dB may be NULL to skip that output (X is then only needed for dA
  * and for recomputing T).  accumulate_grads = 1 adds the new dA / dB to the
  * values already in those buffers (gradient accumulation, [QP] §6.4) instead
@@ -173,7 +179,7 @@ int qlora_linear_fwd(const nf4_tensor* w, const uint16_t* A, const uint16_t* B, 
  * ws >= qlora_bwd_workspace_bytes(M, d_out, d_in, r).
  */
 int qlora_linear_bwd(const nf4_tensor* w, const uint16_t* A, const uint16_t* B, int r,
-                     float scaling, const uint16_t* X, const uint16_t* T_saved,
+                     float scaling, const uint16_t* X, const float* T_saved,
                      const uint16_t* dY, int64_t M, uint16_t* dX, uint16_t* dA,
                      uint16_t* dB, int accumulate_grads, void* ws, size_t ws_bytes,
                      void* stream);

@@ -182,13 +182,13 @@ def nf4_dequantize(w: NF4Tensor, out: Optional[torch.Tensor] = None) -> torch.Te
 def qlora_linear_fwd(w: NF4Tensor, A: torch.Tensor, B: torch.Tensor, scaling: float, X: torch.Tensor,
                      save_t: bool = True, Y: Optional[torch.Tensor] = None,
                      workspace: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
-    """Y = X W_hat^T + s (X A^T) B^T.  Returns (Y, T) with T = bf16(s X A^T)
-    (or None when save_t is False)."""
+    """Y = X W_hat^T + s (X A^T) B^T.  Returns (Y, T) with T = s X A^T in
+    fp32 (or None when save_t is False), for reuse by the backward."""
     _bf16(A, "A"), _bf16(B, "B"), _bf16(X, "X")
     r = A.shape[0]
     M = X.shape[0]
     Y = Y if Y is not None else torch.empty((M, w.d_out), dtype=torch.bfloat16, device=X.device)
-    T = torch.empty((M, r), dtype=torch.bfloat16, device=X.device) if save_t else None
+    T = torch.empty((M, r), dtype=torch.float32, device=X.device) if save_t else None
     need = qlora_fwd_workspace_bytes(M, w.d_out, w.d_in, r)
     ws = workspace if workspace is not None else _workspace(need, X.device)
     _check(lib.qlora_linear_fwd(ctypes.byref(w.struct), _ptr(A), _ptr(B), r, ctypes.c_float(scaling),
@@ -203,9 +203,12 @@ def qlora_linear_bwd(w: NF4Tensor, A: torch.Tensor, B: torch.Tensor, scaling: fl
                      dA: Optional[torch.Tensor] = None, dB: Optional[torch.Tensor] = None,
                      accumulate: bool = False, dX: Optional[torch.Tensor] = None,
                      workspace: Optional[torch.Tensor] = None):
-    """Returns (dX, dA, dB); an output not requested is None.  With
+    """Returns (dX, dA, dB); an output not requested is None.  T is the fp32
+    [M, r] array the forward saved (or None: recomputed from X).  With
     accumulate=True the gradients are added into the given dA / dB."""
     _bf16(A, "A"), _bf16(B, "B"), _bf16(dY, "dY")
+    if T is not None and (T.dtype != torch.float32 or not T.is_contiguous()):
+        raise ValueError("T must be the contiguous float32 array saved by the forward")
     r = A.shape[0]
     M = dY.shape[0]
     dev = dY.device

@@ -185,7 +185,7 @@ int nf4_dequantize(const nf4_tensor* w, uint16_t* W_hat, void* stream) {
 }
 
 int qlora_linear_fwd(const nf4_tensor* w, const uint16_t* A, const uint16_t* B, int r, float scaling,
-                     const uint16_t* X, int64_t M, uint16_t* Y, uint16_t* T_saved, void* ws, size_t ws_bytes,
+                     const uint16_t* X, int64_t M, uint16_t* Y, float* T_saved, void* ws, size_t ws_bytes,
                      void* stream) {
     int rc = check_layer_common(w, A, B, r, scaling, M);
     if (rc) return rc;
@@ -206,7 +206,7 @@ int qlora_linear_fwd(const nf4_tensor* w, const uint16_t* A, const uint16_t* B, 
 }
 
 int qlora_linear_bwd(const nf4_tensor* w, const uint16_t* A, const uint16_t* B, int r, float scaling,
-                     const uint16_t* X, const uint16_t* T_saved, const uint16_t* dY, int64_t M, uint16_t* dX,
+                     const uint16_t* X, const float* T_saved, const uint16_t* dY, int64_t M, uint16_t* dX,
                      uint16_t* dA, uint16_t* dB, int accumulate_grads, void* ws, size_t ws_bytes, void* stream) {
     int rc = check_layer_common(w, A, B, r, scaling, M);
     if (rc) return rc;

@@ -7,7 +7,10 @@
 // 64-wide k-steps ("split"), followed -- in split 0 only -- by the extension
 // k-steps that carry the rank-r LoRA product, so that X W_hat^T + T B^T (or
 // dY W_hat + V A) lands in ONE accumulator without a second pass over the
-// output.
+// output.  The rank-r activation (T or V) is held as a pair of bf16 arrays,
+// hi = bf16(v) and lo = bf16(v - hi), side by side; the extension runs over
+// [hi | lo] while the LoRA weight tile is re-read for the second half
+// (ext_wrap), which keeps ~16 mantissa bits of the fp32 intermediate.
 //
 // Each operand tile is either
 //   * copied by TMA from a bf16 tensor (128-byte swizzle, K-major or
@@ -46,6 +49,8 @@ struct GemmArgs {
     int k_main;         // 64-wide main k-steps in total
     int k_per_split;    // main k-steps per grid.z slice
     int k_ext;          // extension k-steps (grid.z slice 0 only)
+    int ext_wrap_a;     // extension k-step j reads A_ext at (j % ext_wrap_a) when > 0
+    int ext_wrap_b;     // ... and B_ext at (j % ext_wrap_b) when > 0
     // NF4 operand
     const int8_t* qscale;
     const float* scale2;
@@ -179,7 +184,7 @@ __global__ void __launch_bounds__(GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI>:
         s_abort = 0;
         fence_barrier_init();
     }
-    if (threadIdx.x < 16) s_lut[threadIdx.x] = kNf4Levels[threadIdx.x];
+    if (threadIdx.x < 16) s_lut[threadIdx.x] = nf4_level(threadIdx.x);
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&map_a);
         tma_prefetch_desc(&map_b);
@@ -236,19 +241,21 @@ __global__ void __launch_bounds__(GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI>:
                     }
                 } else {
                     const int j = it - n_main;
+                    const int ja = args.ext_wrap_a > 0 ? j % args.ext_wrap_a : j;
+                    const int jb = args.ext_wrap_b > 0 ? j % args.ext_wrap_b : j;
                     mbar_arrive_expect_tx(bar, C::kTxExt);
                     if constexpr (AE_MN) {
-                        tma_load_2d(a_tile(s), &map_ae, bar, r0, j * 64);
-                        tma_load_2d(a_tile(s) + 8192, &map_ae, bar, r0 + 64, j * 64);
+                        tma_load_2d(a_tile(s), &map_ae, bar, r0, ja * 64);
+                        tma_load_2d(a_tile(s) + 8192, &map_ae, bar, r0 + 64, ja * 64);
                     } else {
-                        tma_load_2d(a_tile(s), &map_ae, bar, j * 64, r0);
+                        tma_load_2d(a_tile(s), &map_ae, bar, ja * 64, r0);
                     }
                     if constexpr (BE_MN) {
 #pragma unroll
                         for (int c = 0; c < BN / 64; ++c)
-                            tma_load_2d(b_tile(s) + c * 8192, &map_be, bar, c0 + c * 64, j * 64);
+                            tma_load_2d(b_tile(s) + c * 8192, &map_be, bar, c0 + c * 64, jb * 64);
                     } else {
-                        tma_load_2d(b_tile(s), &map_be, bar, j * 64, c0);
+                        tma_load_2d(b_tile(s), &map_be, bar, jb * 64, c0);
                     }
                 }
                 ++issued;

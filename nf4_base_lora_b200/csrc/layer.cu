@@ -1,12 +1,12 @@
 // Host orchestration of the NF4-LoRA linear layer on the tcgen05 engine.
 //
 // Forward   ("第 04 篇：QLoRA 原理" §6.1-§6.3):
-//   1. T = bf16(s X A^T)                       LoRA down: tcgen05, split-K
+//   1. T = s X A^T (fp32, kept as a bf16 hi|lo pair)  LoRA down: tcgen05, split-K
 //   2. Y = X W_hat^T + T B^T                    fused dequant-GEMM, LoRA up as
 //                                               extension k-steps of the same
 //                                               accumulator
 // Backward  (§2.4: input gradient through the frozen base; no dW):
-//   1. V = bf16(s dY B)                         tcgen05, split-K over d_out
+//   1. V = s dY B (bf16 hi|lo pair)             tcgen05, split-K over d_out
 //   2. dX = dY W_hat + V A                      fused dequant-GEMM (MN-major
 //                                               decode of the same codes)
 //   3. dB = dY^T T,  dA = V^T X                 tcgen05, split over tokens,
@@ -82,40 +82,94 @@ static cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b, const CUte
     return cudaGetLastError();
 }
 
-// fixed-order sum over split-K slices: out[r, c] = bf16(alpha * sum_z part[z]) (+ out)
-__global__ void k_reduce_splits(const float* __restrict__ part, int splits, int64_t slice, int rows,
-                                int cols, int64_t ldp, float alpha, uint16_t* __restrict__ out,
-                                int64_t ldo, uint16_t* __restrict__ out2, int64_t ldo2, int out2_cols,
-                                int accumulate) {
-    const int64_t total = static_cast<int64_t>(rows) * cols;
+// Fixed-order sum over the split-K slices of an fp32 partial buffer:
+//   v[r, c] = alpha * sum_z (part[z][r, c] + part[z][r, c + fold])   (fold 0: no second term)
+// written as bf16 (optionally added to the bf16 already there), or -- in split
+// mode (lo_off > 0) -- as the pair hi = bf16(v), lo = bf16(v - hi) at columns c
+// and c + lo_off; optionally also as fp32 into out32 for c < out32_cols.
+struct ReduceArgs {
+    const float* part;
+    int splits;
+    int64_t slice;
+    int rows;
+    int cols;
+    int64_t ldp;
+    int64_t fold;
+    float alpha;
+    uint16_t* out;
+    int64_t ldo;
+    int64_t lo_off;
+    int accumulate;
+    float* out32;
+    int64_t ldo32;
+    int out32_cols;
+};
+
+__global__ void k_reduce_splits(const ReduceArgs a) {
+    const int64_t total = static_cast<int64_t>(a.rows) * a.cols;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int64_t r = i / cols, c = i % cols;
-        const float* p = part + r * ldp + c;
+        const int64_t r = i / a.cols, c = i % a.cols;
+        const float* p = a.part + r * a.ldp + c;
         float acc = 0.0f;
-        for (int z = 0; z < splits; ++z) acc += p[z * slice];
-        const float v = acc * alpha;
-        float o = v;
-        if (accumulate) o += bf16_bits_to_float(out[r * ldo + c]);
-        __nv_bfloat16 h = __float2bfloat16_rn(o);
-        out[r * ldo + c] = *reinterpret_cast<uint16_t*>(&h);
-        if (out2 != nullptr && c < out2_cols) {
-            __nv_bfloat16 h2 = __float2bfloat16_rn(v);
-            out2[r * ldo2 + c] = *reinterpret_cast<uint16_t*>(&h2);
+        for (int z = 0; z < a.splits; ++z) {
+            acc += p[z * a.slice];
+            if (a.fold) acc += p[z * a.slice + a.fold];
         }
+        const float v = acc * a.alpha;
+        uint16_t* o = a.out + r * a.ldo + c;
+        if (a.lo_off > 0) {
+            const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+            o[0] = *reinterpret_cast<const uint16_t*>(&hi);
+            o[a.lo_off] = *reinterpret_cast<const uint16_t*>(&lo);
+        } else {
+            const float w = a.accumulate ? v + bf16_bits_to_float(o[0]) : v;
+            const __nv_bfloat16 h = __float2bfloat16_rn(w);
+            o[0] = *reinterpret_cast<const uint16_t*>(&h);
+        }
+        if (a.out32 != nullptr && c < a.out32_cols) a.out32[r * a.ldo32 + c] = v;
     }
 }
 
-static cudaError_t reduce(const float* part, int splits, int64_t slice, int rows, int cols, int64_t ldp,
-                          float alpha, uint16_t* out, int64_t ldo, uint16_t* out2, int64_t ldo2,
-                          int out2_cols, int accumulate, int num_sms, cudaStream_t st) {
-    const int64_t total = static_cast<int64_t>(rows) * cols;
+static cudaError_t reduce(const ReduceArgs& a, int num_sms, cudaStream_t st) {
+    const int64_t total = static_cast<int64_t>(a.rows) * a.cols;
     int64_t grid = (total + 255) / 256;
     grid = std::min<int64_t>(grid, int64_t(num_sms) * 8);
     if (grid < 1) grid = 1;
-    k_reduce_splits<<<static_cast<unsigned>(grid), 256, 0, st>>>(part, splits, slice, rows, cols, ldp, alpha,
-                                                                 out, ldo, out2, ldo2, out2_cols, accumulate);
+    k_reduce_splits<<<static_cast<unsigned>(grid), 256, 0, st>>>(a);
     return cudaGetLastError();
+}
+
+static ReduceArgs reduce_args(const float* part, int splits, int64_t slice, int rows, int cols, int64_t ldp,
+                              float alpha, uint16_t* out, int64_t ldo) {
+    ReduceArgs a{};
+    a.part = part;
+    a.splits = splits;
+    a.slice = slice;
+    a.rows = rows;
+    a.cols = cols;
+    a.ldp = ldp;
+    a.alpha = alpha;
+    a.out = out;
+    a.ldo = ldo;
+    return a;
+}
+
+// T2 / V2 [M, 2 r64] = (hi | lo) split of an fp32 [M, r] array, zero beyond r.
+__global__ void k_split_from_f32(const float* __restrict__ src, int64_t M, int r, int r64,
+                                 uint16_t* __restrict__ dst) {
+    const int64_t total = M * r64;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t m = i / r64;
+        const int j = static_cast<int>(i % r64);
+        const float v = j < r ? src[m * r + j] : 0.0f;
+        const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+        const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+        dst[m * 2 * r64 + j] = *reinterpret_cast<const uint16_t*>(&hi);
+        dst[m * 2 * r64 + r64 + j] = *reinterpret_cast<const uint16_t*>(&lo);
+    }
 }
 
 // ------------------------------------------------------------------ split sizing
@@ -137,15 +191,24 @@ static Split choose_split(int tiles, int k_steps, int target, int min_steps) {
 static inline int64_t align256(int64_t b) { return (b + 255) & ~int64_t(255); }
 static inline int round64(int r) { return (r + 63) / 64 * 64; }
 static inline int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
-
-// partial-buffer sizes (floats) of each split-K GEMM, with the split it will use
-static int64_t down_part_floats(int64_t M, int64_t K, int r64, int num_sms, Split* sp) {
-    Split s = choose_split(ceil_div(M, 128), ceil_div(K, 64), num_sms, 4);
-    if (sp) *sp = s;
-    return int64_t(s.splits) * M * r64;
-}
+static int bn_for(int cols) { return cols <= 64 ? 64 : (cols <= 128 ? 128 : 256); }
 
 static constexpr int kSmallM = 16;
+
+// The splits each split-K GEMM uses (the workspace query and the calls share them).
+static Split split_down(int64_t M, int64_t d_in, int sms) {
+    return choose_split(ceil_div(M, 128), ceil_div(d_in, 64), sms, 4);
+}
+static Split split_v(int64_t M, int64_t d_out, int sms) {
+    return choose_split(ceil_div(M, 128), ceil_div(d_out, 64), sms, 4);
+}
+static Split split_tokens(int64_t rows, int r64, int64_t M, int sms) {
+    const int tiles = ceil_div(rows, 128) * ceil_div(2 * r64, bn_for(2 * r64));
+    return choose_split(tiles, ceil_div(M, 64), sms, 4);
+}
+static Split split_small(int64_t rows, int64_t k, int sms) {
+    return choose_split(ceil_div(rows, 128), ceil_div(k, 64), 2 * sms, 4);
+}
 
 // ------------------------------------------------------------------ layer ops
 struct Maps {
@@ -162,17 +225,13 @@ static cudaError_t launch_lora_gemm(int bn, const Maps& m, const GemmArgs& args,
     }
 }
 
-static int bn_for(int r64) { return r64 <= 64 ? 64 : (r64 <= 128 ? 128 : 256); }
-
-// T_pad[M, r64] = bf16(s X A^T) (zero columns beyond r); optional T_saved[M, r].
+// T2[M, 2 r64] = hi | lo of s X A^T (zero columns beyond r); optional fp32 T_saved[M, r].
 static int lora_down(const LayerCtx& c, const uint16_t* A, int r, float s, const uint16_t* X, int64_t M,
-                     uint16_t* T_pad, uint16_t* T_saved, float* part) {
+                     uint16_t* T2, float* T_saved, float* part) {
     const int r64 = round64(r), bn = bn_for(r64);
     Maps m;
-    if (!map_bf16(&m.a, X, c.d_in, M, c.d_in, 128) || !map_bf16(&m.b, A, c.d_in, r, c.d_in, bn))
-        return -1;
-    Split sp;
-    down_part_floats(M, c.d_in, r64, c.num_sms, &sp);
+    if (!map_bf16(&m.a, X, c.d_in, M, c.d_in, 128) || !map_bf16(&m.b, A, c.d_in, r, c.d_in, bn)) return -1;
+    const Split sp = split_down(M, c.d_in, c.num_sms);
     GemmArgs g{};
     g.rows = static_cast<int>(M);
     g.cols = r64;
@@ -181,30 +240,29 @@ static int lora_down(const LayerCtx& c, const uint16_t* A, int r, float s, const
     g.part = part;
     g.ldp = r64;
     g.part_slice = M * r64;
-    dim3 grid(ceil_div(M, 128), 1, sp.splits);
+    dim3 grid(ceil_div(M, 128), ceil_div(r64, bn), sp.splits);
     if (launch_lora_gemm<EPI_F32_PART, SRC_TMA_K, SRC_TMA_K>(bn, m, g, grid, c.stream) != cudaSuccess) return -2;
-    if (reduce(part, sp.splits, M * r64, static_cast<int>(M), r64, r64, s, T_pad, r64, T_saved, r, r, 0,
-               c.num_sms, c.stream) != cudaSuccess)
-        return -2;
-    return 0;
+    ReduceArgs ra = reduce_args(part, sp.splits, M * r64, static_cast<int>(M), r64, r64, s, T2, 2 * r64);
+    ra.lo_off = r64;
+    ra.out32 = T_saved;
+    ra.ldo32 = r;
+    ra.out32_cols = r;
+    return reduce(ra, c.num_sms, c.stream) == cudaSuccess ? 0 : -2;
 }
 
 int64_t fwd_workspace_bytes(int64_t M, int64_t d_out, int64_t d_in, int r, int num_sms) {
     const int r64 = round64(r);
-    int64_t part = down_part_floats(M, d_in, r64, num_sms, nullptr);
-    if (M <= kSmallM) {
-        Split s = choose_split(ceil_div(d_out, 128), ceil_div(d_in, 64), 2 * num_sms, 4);
-        part = std::max<int64_t>(part, int64_t(s.splits) * M * d_out);
-    }
-    return align256(M * r64 * 2) + align256(part * 4);
+    int64_t part = int64_t(split_down(M, d_in, num_sms).splits) * M * r64;
+    if (M <= kSmallM) part = std::max<int64_t>(part, int64_t(split_small(d_out, d_in, num_sms).splits) * M * d_out);
+    return align256(M * r64 * 4) + align256(part * 4);
 }
 
 int layer_fwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, float s, const uint16_t* X,
-              int64_t M, uint16_t* Y, uint16_t* T_saved, uint8_t* ws) {
-    const int r64 = round64(r);
-    uint16_t* T_pad = reinterpret_cast<uint16_t*>(ws);
-    float* part = reinterpret_cast<float*>(ws + align256(M * r64 * 2));
-    int rc = lora_down(c, A, r, s, X, M, T_pad, T_saved, part);
+              int64_t M, uint16_t* Y, float* T_saved, uint8_t* ws) {
+    const int r64 = round64(r), kx = r64 / 64;
+    uint16_t* T2 = reinterpret_cast<uint16_t*>(ws);
+    float* part = reinterpret_cast<float*>(ws + align256(M * r64 * 4));
+    int rc = lora_down(c, A, r, s, X, M, T2, T_saved, part);
     if (rc) return rc;
     Maps m;
     GemmArgs g{};
@@ -214,15 +272,16 @@ int layer_fwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, fl
     g.w_rows = c.d_out;
     g.w_blocks_per_row = c.d_in / 64;
     g.k_main = ceil_div(c.d_in, 64);
-    g.k_ext = r64 / 64;
+    g.k_ext = 2 * kx;
     g.alpha = 1.0f;
     if (M <= kSmallM) {
         // swapped: D[n, m] = W_hat[n, :] . X[m, :] + B[n, :] . T[m, :]
         if (!map_codes(&m.a, c.codes, c.d_out, c.d_in, 32, 128) || !map_bf16(&m.b, X, c.d_in, M, c.d_in, 16) ||
-            !map_bf16(&m.ae, B, r, c.d_out, r, 128) || !map_bf16(&m.be, T_pad, r64, M, r64, 16))
+            !map_bf16(&m.ae, B, r, c.d_out, r, 128) || !map_bf16(&m.be, T2, 2 * r64, M, 2 * r64, 16))
             return -1;
         const int tiles = ceil_div(c.d_out, 128);
-        Split sp = choose_split(tiles, g.k_main, 2 * c.num_sms, 4);
+        const Split sp = split_small(c.d_out, c.d_in, c.num_sms);
+        g.ext_wrap_a = kx;
         g.rows = static_cast<int>(c.d_out);
         g.cols = static_cast<int>(M);
         g.k_per_split = sp.k_per_split;
@@ -233,14 +292,14 @@ int layer_fwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, fl
         if (launch<16, SRC_DEC_K, SRC_TMA_K, 0, 0, EPI_F32_PART_T>(m.a, m.b, m.ae, m.be, g, grid, c.stream) !=
             cudaSuccess)
             return -2;
-        if (reduce(part, sp.splits, M * c.d_out, static_cast<int>(M), static_cast<int>(c.d_out), c.d_out, 1.0f, Y,
-                   c.d_out, nullptr, 0, 0, 0, c.num_sms, c.stream) != cudaSuccess)
-            return -2;
-        return 0;
+        ReduceArgs ra = reduce_args(part, sp.splits, M * c.d_out, static_cast<int>(M), static_cast<int>(c.d_out),
+                                    c.d_out, 1.0f, Y, c.d_out);
+        return reduce(ra, c.num_sms, c.stream) == cudaSuccess ? 0 : -2;
     }
     if (!map_bf16(&m.a, X, c.d_in, M, c.d_in, 128) || !map_codes(&m.b, c.codes, c.d_out, c.d_in, 32, 256) ||
-        !map_bf16(&m.ae, T_pad, r64, M, r64, 128) || !map_bf16(&m.be, B, r, c.d_out, r, 256))
+        !map_bf16(&m.ae, T2, 2 * r64, M, 2 * r64, 128) || !map_bf16(&m.be, B, r, c.d_out, r, 256))
         return -1;
+    g.ext_wrap_b = kx;
     g.rows = static_cast<int>(M);
     g.cols = static_cast<int>(c.d_out);
     g.k_per_split = g.k_main;
@@ -254,36 +313,28 @@ int layer_fwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, fl
 
 int64_t bwd_workspace_bytes(int64_t M, int64_t d_out, int64_t d_in, int r, int num_sms) {
     const int r64 = round64(r);
-    int64_t part = down_part_floats(M, d_in, r64, num_sms, nullptr);
-    // V = s dY B: split over d_out
-    Split sv = choose_split(ceil_div(M, 128), ceil_div(d_out, 64), num_sms, 4);
-    part = std::max<int64_t>(part, int64_t(sv.splits) * M * r64);
-    // dB, dA: split over tokens
-    Split sb = choose_split(ceil_div(d_out, 128), ceil_div(M, 64), num_sms, 4);
-    part = std::max<int64_t>(part, int64_t(sb.splits) * d_out * r64);
-    Split sa = choose_split(ceil_div(d_in, 128), ceil_div(M, 64), num_sms, 4);
-    part = std::max<int64_t>(part, int64_t(sa.splits) * d_in * r64);
-    if (M <= kSmallM) {
-        Split sx = choose_split(ceil_div(d_in, 128), ceil_div(d_out, 64), 2 * num_sms, 4);
-        part = std::max<int64_t>(part, int64_t(sx.splits) * M * d_in);
-    }
-    return 2 * align256(M * r64 * 2) + align256(part * 4);
+    int64_t part = int64_t(split_down(M, d_in, num_sms).splits) * M * r64;
+    part = std::max<int64_t>(part, int64_t(split_v(M, d_out, num_sms).splits) * M * r64);
+    part = std::max<int64_t>(part, int64_t(split_tokens(d_out, r64, M, num_sms).splits) * d_out * 2 * r64);
+    part = std::max<int64_t>(part, int64_t(split_tokens(d_in, r64, M, num_sms).splits) * d_in * 2 * r64);
+    if (M <= kSmallM) part = std::max<int64_t>(part, int64_t(split_small(d_in, d_out, num_sms).splits) * M * d_in);
+    return 2 * align256(M * r64 * 4) + align256(part * 4);
 }
 
 int layer_bwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, float s, const uint16_t* X,
-              const uint16_t* T_saved, const uint16_t* dY, int64_t M, uint16_t* dX, uint16_t* dA,
-              uint16_t* dB, int accumulate, uint8_t* ws) {
-    const int r64 = round64(r), bn = bn_for(r64);
-    uint16_t* V_pad = reinterpret_cast<uint16_t*>(ws);
-    uint16_t* T_pad = reinterpret_cast<uint16_t*>(ws + align256(M * r64 * 2));
-    float* part = reinterpret_cast<float*>(ws + 2 * align256(M * r64 * 2));
-    int rc;
+              const float* T_saved, const uint16_t* dY, int64_t M, uint16_t* dX, uint16_t* dA, uint16_t* dB,
+              int accumulate, uint8_t* ws) {
+    const int r64 = round64(r), kx = r64 / 64;
+    uint16_t* V2 = reinterpret_cast<uint16_t*>(ws);
+    uint16_t* T2 = reinterpret_cast<uint16_t*>(ws + align256(M * r64 * 4));
+    float* part = reinterpret_cast<float*>(ws + 2 * align256(M * r64 * 4));
 
-    // ---- V = bf16(s dY B): D[m, j] = sum_n dY[m, n] B[n, j]
+    // ---- V = s dY B, held as hi | lo: D[m, j] = sum_n dY[m, n] B[n, j]
     if (dX != nullptr || dA != nullptr) {
+        const int bn = bn_for(r64);
         Maps m;
         if (!map_bf16(&m.a, dY, c.d_out, M, c.d_out, 128) || !map_bf16(&m.b, B, r, c.d_out, r, 64)) return -1;
-        Split sp = choose_split(ceil_div(M, 128), ceil_div(c.d_out, 64), c.num_sms, 4);
+        const Split sp = split_v(M, c.d_out, c.num_sms);
         GemmArgs g{};
         g.rows = static_cast<int>(M);
         g.cols = r64;
@@ -292,11 +343,11 @@ int layer_bwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, fl
         g.part = part;
         g.ldp = r64;
         g.part_slice = M * r64;
-        dim3 grid(ceil_div(M, 128), 1, sp.splits);
+        dim3 grid(ceil_div(M, 128), ceil_div(r64, bn), sp.splits);
         if (launch_lora_gemm<EPI_F32_PART, SRC_TMA_K, SRC_TMA_MN>(bn, m, g, grid, c.stream) != cudaSuccess) return -2;
-        if (reduce(part, sp.splits, M * r64, static_cast<int>(M), r64, r64, s, V_pad, r64, nullptr, 0, 0, 0,
-                   c.num_sms, c.stream) != cudaSuccess)
-            return -2;
+        ReduceArgs ra = reduce_args(part, sp.splits, M * r64, static_cast<int>(M), r64, r64, s, V2, 2 * r64);
+        ra.lo_off = r64;
+        if (reduce(ra, c.num_sms, c.stream) != cudaSuccess) return -2;
     }
 
     // ---- dX = dY W_hat + V A
@@ -309,15 +360,16 @@ int layer_bwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, fl
         g.w_rows = c.d_out;
         g.w_blocks_per_row = c.d_in / 64;
         g.k_main = ceil_div(c.d_out, 64);
-        g.k_ext = r64 / 64;
+        g.k_ext = 2 * kx;
         g.alpha = 1.0f;
         if (M <= kSmallM) {
             // swapped: D[k, m] = sum_n W_hat[n, k] dY[m, n] + sum_j A[j, k] V[m, j]
             if (!map_codes(&m.a, c.codes, c.d_out, c.d_in, 64, 64) || !map_bf16(&m.b, dY, c.d_out, M, c.d_out, 16) ||
-                !map_bf16(&m.ae, A, c.d_in, r, c.d_in, 64) || !map_bf16(&m.be, V_pad, r64, M, r64, 16))
+                !map_bf16(&m.ae, A, c.d_in, r, c.d_in, 64) || !map_bf16(&m.be, V2, 2 * r64, M, 2 * r64, 16))
                 return -1;
             const int tiles = ceil_div(c.d_in, 128);
-            Split sp = choose_split(tiles, g.k_main, 2 * c.num_sms, 4);
+            const Split sp = split_small(c.d_in, c.d_out, c.num_sms);
+            g.ext_wrap_a = kx;
             g.rows = static_cast<int>(c.d_in);
             g.cols = static_cast<int>(M);
             g.k_per_split = sp.k_per_split;
@@ -328,13 +380,14 @@ int layer_bwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, fl
             if (launch<16, SRC_DEC_MN, SRC_TMA_K, 1, 0, EPI_F32_PART_T>(m.a, m.b, m.ae, m.be, g, grid, c.stream) !=
                 cudaSuccess)
                 return -2;
-            if (reduce(part, sp.splits, M * c.d_in, static_cast<int>(M), static_cast<int>(c.d_in), c.d_in, 1.0f, dX,
-                       c.d_in, nullptr, 0, 0, 0, c.num_sms, c.stream) != cudaSuccess)
-                return -2;
+            ReduceArgs ra = reduce_args(part, sp.splits, M * c.d_in, static_cast<int>(M), static_cast<int>(c.d_in),
+                                        c.d_in, 1.0f, dX, c.d_in);
+            if (reduce(ra, c.num_sms, c.stream) != cudaSuccess) return -2;
         } else {
             if (!map_bf16(&m.a, dY, c.d_out, M, c.d_out, 128) || !map_codes(&m.b, c.codes, c.d_out, c.d_in, 128, 64) ||
-                !map_bf16(&m.ae, V_pad, r64, M, r64, 128) || !map_bf16(&m.be, A, c.d_in, r, c.d_in, 64))
+                !map_bf16(&m.ae, V2, 2 * r64, M, 2 * r64, 128) || !map_bf16(&m.be, A, c.d_in, r, c.d_in, 64))
                 return -1;
+            g.ext_wrap_b = kx;
             g.rows = static_cast<int>(M);
             g.cols = static_cast<int>(c.d_in);
             g.k_per_split = g.k_main;
@@ -347,53 +400,57 @@ int layer_bwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, fl
         }
     }
 
-    // ---- dB = dY^T T: D[n, j] = sum_m dY[m, n] T[m, j]
+    const int bn2 = bn_for(2 * r64);  // the (hi | lo) operand is 2 r64 wide
+    // ---- dB = dY^T T: D[n, c] = sum_m dY[m, n] T2[m, c], then dB[n, j] = D[n, j] + D[n, j + r64]
     if (dB != nullptr) {
-        const uint16_t* T = T_saved;
-        int64_t ldt = r;
-        if (T == nullptr) {
-            rc = lora_down(c, A, r, s, X, M, T_pad, nullptr, part);
+        if (T_saved != nullptr) {
+            k_split_from_f32<<<static_cast<unsigned>(std::min<int64_t>((M * r64 + 255) / 256, c.num_sms * 8)), 256, 0,
+                               c.stream>>>(T_saved, M, r, r64, T2);
+            if (cudaGetLastError() != cudaSuccess) return -2;
+        } else {
+            int rc = lora_down(c, A, r, s, X, M, T2, nullptr, part);
             if (rc) return rc;
-            T = T_pad;
-            ldt = r64;
         }
         Maps m;
-        if (!map_bf16(&m.a, dY, c.d_out, M, c.d_out, 64) || !map_bf16(&m.b, T, ldt, M, ldt, 64)) return -1;
-        Split sp = choose_split(ceil_div(c.d_out, 128), ceil_div(M, 64), c.num_sms, 4);
+        if (!map_bf16(&m.a, dY, c.d_out, M, c.d_out, 64) || !map_bf16(&m.b, T2, 2 * r64, M, 2 * r64, 64)) return -1;
+        const Split sp = split_tokens(c.d_out, r64, M, c.num_sms);
         GemmArgs g{};
         g.rows = static_cast<int>(c.d_out);
-        g.cols = r64;
+        g.cols = 2 * r64;
         g.k_main = ceil_div(M, 64);
         g.k_per_split = sp.k_per_split;
         g.part = part;
-        g.ldp = r64;
-        g.part_slice = c.d_out * r64;
-        dim3 grid(ceil_div(c.d_out, 128), 1, sp.splits);
-        if (launch_lora_gemm<EPI_F32_PART, SRC_TMA_MN, SRC_TMA_MN>(bn, m, g, grid, c.stream) != cudaSuccess) return -2;
-        if (reduce(part, sp.splits, c.d_out * r64, static_cast<int>(c.d_out), r, r64, 1.0f, dB, r, nullptr, 0, 0,
-                   accumulate, c.num_sms, c.stream) != cudaSuccess)
-            return -2;
+        g.ldp = 2 * r64;
+        g.part_slice = c.d_out * 2 * r64;
+        dim3 grid(ceil_div(c.d_out, 128), ceil_div(2 * r64, bn2), sp.splits);
+        if (launch_lora_gemm<EPI_F32_PART, SRC_TMA_MN, SRC_TMA_MN>(bn2, m, g, grid, c.stream) != cudaSuccess) return -2;
+        ReduceArgs ra = reduce_args(part, sp.splits, c.d_out * 2 * r64, static_cast<int>(c.d_out), r, 2 * r64, 1.0f, dB, r);
+        ra.fold = r64;
+        ra.accumulate = accumulate;
+        if (reduce(ra, c.num_sms, c.stream) != cudaSuccess) return -2;
     }
 
-    // ---- dA = V^T X: D[k, j] = sum_m X[m, k] V[m, j], stored transposed
+    // ---- dA = V^T X: D[k, c] = sum_m X[m, k] V2[m, c], stored transposed, dA[j, k] = D[k, j] + D[k, j + r64]
     if (dA != nullptr) {
         Maps m;
-        if (!map_bf16(&m.a, X, c.d_in, M, c.d_in, 64) || !map_bf16(&m.b, V_pad, r64, M, r64, 64)) return -1;
-        Split sp = choose_split(ceil_div(c.d_in, 128), ceil_div(M, 64), c.num_sms, 4);
+        if (!map_bf16(&m.a, X, c.d_in, M, c.d_in, 64) || !map_bf16(&m.b, V2, 2 * r64, M, 2 * r64, 64)) return -1;
+        const Split sp = split_tokens(c.d_in, r64, M, c.num_sms);
         GemmArgs g{};
         g.rows = static_cast<int>(c.d_in);
-        g.cols = r64;
+        g.cols = 2 * r64;
         g.k_main = ceil_div(M, 64);
         g.k_per_split = sp.k_per_split;
         g.part = part;
         g.ldp = c.d_in;
-        g.part_slice = int64_t(r64) * c.d_in;
-        dim3 grid(ceil_div(c.d_in, 128), 1, sp.splits);
-        if (launch_lora_gemm<EPI_F32_PART_T, SRC_TMA_MN, SRC_TMA_MN>(bn, m, g, grid, c.stream) != cudaSuccess)
+        g.part_slice = int64_t(2 * r64) * c.d_in;
+        dim3 grid(ceil_div(c.d_in, 128), ceil_div(2 * r64, bn2), sp.splits);
+        if (launch_lora_gemm<EPI_F32_PART_T, SRC_TMA_MN, SRC_TMA_MN>(bn2, m, g, grid, c.stream) != cudaSuccess)
             return -2;
-        if (reduce(part, sp.splits, int64_t(r64) * c.d_in, r, static_cast<int>(c.d_in), c.d_in, 1.0f, dA, c.d_in,
-                   nullptr, 0, 0, accumulate, c.num_sms, c.stream) != cudaSuccess)
-            return -2;
+        ReduceArgs ra = reduce_args(part, sp.splits, int64_t(2 * r64) * c.d_in, r, static_cast<int>(c.d_in), c.d_in,
+                                    1.0f, dA, c.d_in);
+        ra.fold = int64_t(r64) * c.d_in;
+        ra.accumulate = accumulate;
+        if (reduce(ra, c.num_sms, c.stream) != cudaSuccess) return -2;
     }
     return 0;
 }

@@ -28,9 +28,9 @@ int64_t bwd_workspace_bytes(int64_t M, int64_t d_out, int64_t d_in, int r, int n
 // Return 0 on success, -1 if a tensor map could not be encoded, -2 if a
 // launch failed.
 int layer_fwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, float s, const uint16_t* X,
-              int64_t M, uint16_t* Y, uint16_t* T_saved, uint8_t* ws);
+              int64_t M, uint16_t* Y, float* T_saved, uint8_t* ws);
 int layer_bwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, float s, const uint16_t* X,
-              const uint16_t* T_saved, const uint16_t* dY, int64_t M, uint16_t* dX, uint16_t* dA,
+              const float* T_saved, const uint16_t* dY, int64_t M, uint16_t* dX, uint16_t* dA,
               uint16_t* dB, int accumulate, uint8_t* ws);
 
 }  // namespace nf4lora

@@ -6,13 +6,29 @@
 
 namespace nf4lora {
 
-// One copy per translation unit in the constant bank.  Kernels that index it
-// with per-thread codes copy it to shared memory first, where the 16 words
-// sit in 16 different banks, so any pattern of lookups is conflict-free.
-static __constant__ float kNf4Levels[16] = {
-    -1.0000000f, -0.6961928f, -0.5250731f, -0.3949175f, -0.2844414f, -0.1847734f,
-    -0.0910500f, 0.0000000f,  0.0795803f,  0.1609302f,  0.2461123f,  0.3379152f,
-    0.4407098f,  0.5626170f,  0.7229568f,  1.0000000f};
+// Level j as an immediate (no constant-bank table).  Kernels that index the
+// levels with per-thread codes copy them to shared memory first, where the 16
+// words sit in 16 different banks, so any pattern of lookups is conflict-free.
+__device__ __forceinline__ float nf4_level(int j) {
+    switch (j) {
+        case 0: return -1.0000000f;
+        case 1: return -0.6961928f;
+        case 2: return -0.5250731f;
+        case 3: return -0.3949175f;
+        case 4: return -0.2844414f;
+        case 5: return -0.1847734f;
+        case 6: return -0.0910500f;
+        case 7: return 0.0000000f;
+        case 8: return 0.0795803f;
+        case 9: return 0.1609302f;
+        case 10: return 0.2461123f;
+        case 11: return 0.3379152f;
+        case 12: return 0.4407098f;
+        case 13: return 0.5626170f;
+        case 14: return 0.7229568f;
+        default: return 1.0000000f;
+    }
+}
 
 // Restored first-level scale of block b: s_b = q_b * (a2_g / 127) + mean,
 // each step an IEEE fp32 operation rounded once ("第 04 篇：QLoRA 原理" §6.1).

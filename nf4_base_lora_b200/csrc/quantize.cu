@@ -39,7 +39,7 @@ __global__ void __launch_bounds__(256) k_nf4_encode(const float* __restrict__ W,
     __shared__ double s_sum[kTileBlocks];
     const int tid = threadIdx.x;
     if (tid < 15) {
-        s_mid[tid] = __fmul_rn(__fadd_rn(kNf4Levels[tid], kNf4Levels[tid + 1]), 0.5f);
+        s_mid[tid] = __fmul_rn(__fadd_rn(nf4_level(tid), nf4_level(tid + 1)), 0.5f);
     } else if (tid == 15) {
         s_mid[15] = __int_as_float(0x7f800000);
     }
@@ -181,7 +181,7 @@ __global__ void __launch_bounds__(256) k_nf4_dequantize(const uint8_t* __restric
                                                        const float* __restrict__ mean_ptr,
                                                        int64_t n, uint16_t* __restrict__ out) {
     __shared__ float s_lut[16];
-    if (threadIdx.x < 16) s_lut[threadIdx.x] = kNf4Levels[threadIdx.x];
+    if (threadIdx.x < 16) s_lut[threadIdx.x] = nf4_level(threadIdx.x);
     __syncthreads();
     const float mu = *mean_ptr;
     const int64_t n_units = n / 16;
