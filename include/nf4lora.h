@@ -195,6 +195,25 @@ const char* nf4lora_last_error_string(void);
  * synchronisation fails. */
 int nf4lora_device_status(void* stream);
 
+/* ---------------------------------------------------------------- tracing */
+
+/* Start timing the library's own kernel launches (host-side tracing): each
+ * launch from now on is bracketed by two CUDA events recorded on its stream;
+ * inside a stream capture the records become graph nodes that every replay
+ * refreshes.  The first max_launches launches get a record, later ones are
+ * only counted.  Creates 2 * max_launches events (no device memory).
+ * Returns NF4_OK, NF4_ERR_INVALID_ARG or NF4_ERR_CUDA. */
+int nf4lora_trace_start(int max_launches);
+
+/* Stop bracketing launches; the records stay readable. */
+int nf4lora_trace_stop(void);
+
+/* Launches counted since nf4lora_trace_start (recorded or not). */
+int nf4lora_trace_count(void);
+
+/* Kernel name and device time in ms of record i; waits for its stop event. */
+int nf4lora_trace_get(int i, char* name, size_t name_len, float* ms);
+
 /* Library version, e.g. "nf4lora 0.1.0 sm_100a". */
 const char* nf4lora_version(void);
 

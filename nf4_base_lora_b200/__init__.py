@@ -31,7 +31,8 @@ STATUS_NAMES = {0: "NF4_OK", -1: "NF4_ERR_INVALID_ARG", -2: "NF4_ERR_UNSUPPORTED
 ABI_SYMBOLS = ("nf4_packed_bytes", "nf4_tensor_from_buffer", "nf4_quantize_workspace_bytes",
                "qlora_fwd_workspace_bytes", "qlora_bwd_workspace_bytes", "nf4_quantize",
                "nf4_dequantize", "qlora_linear_fwd", "qlora_linear_bwd",
-               "nf4lora_last_error_string", "nf4lora_device_status", "nf4lora_version")
+               "nf4lora_last_error_string", "nf4lora_device_status", "nf4lora_trace_start",
+               "nf4lora_trace_stop", "nf4lora_trace_count", "nf4lora_trace_get", "nf4lora_version")
 
 
 class Nf4TensorStruct(ctypes.Structure):
@@ -66,6 +67,10 @@ def _load() -> ctypes.CDLL:
         "qlora_linear_bwd": (I, [S, P, P, I, F, P, P, P, I64, P, P, P, I, P, SZ, P]),
         "nf4lora_last_error_string": (ctypes.c_char_p, []),
         "nf4lora_device_status": (I, [P]),
+        "nf4lora_trace_start": (I, [I]),
+        "nf4lora_trace_stop": (I, []),
+        "nf4lora_trace_count": (I, []),
+        "nf4lora_trace_get": (I, [I, ctypes.c_char_p, SZ, ctypes.POINTER(ctypes.c_float)]),
         "nf4lora_version": (ctypes.c_char_p, []),
     }
     for name, (res, args) in sig.items():
@@ -233,6 +238,32 @@ def qlora_linear_bwd(w: NF4Tensor, A: torch.Tensor, B: torch.Tensor, scaling: fl
 def device_status() -> None:
     """Raise Nf4Error(NF4_ERR_TIMEOUT) if a kernel abandoned a bounded wait."""
     _check(lib.nf4lora_device_status(_stream()))
+
+
+def trace_start(max_launches: int = 4096) -> None:
+    """Time every kernel the library launches from now on (see trace_records)."""
+    _check(lib.nf4lora_trace_start(max_launches))
+
+
+def trace_stop() -> None:
+    _check(lib.nf4lora_trace_stop())
+
+
+def trace_count() -> int:
+    return int(lib.nf4lora_trace_count())
+
+
+def trace_records(limit: Optional[int] = None):
+    """[(kernel name, device ms), ...] of the recorded launches."""
+    out = []
+    n = trace_count() if limit is None else limit
+    for i in range(n):
+        name = ctypes.create_string_buffer(64)
+        ms = ctypes.c_float(0.0)
+        if lib.nf4lora_trace_get(i, name, 64, ctypes.byref(ms)) != NF4_OK:
+            break
+        out.append((name.value.decode(), float(ms.value)))
+    return out
 
 
 def version() -> str:

@@ -201,7 +201,7 @@ int qlora_linear_fwd(const nf4_tensor* w, const uint16_t* A, const uint16_t* B, 
                static_cast<cudaStream_t>(stream)};
     rc = layer_fwd(c, A, B, r, scaling, X, M, Y, T_saved, static_cast<uint8_t*>(ws));
     if (rc == -1) return fail(NF4_ERR_CUDA, "qlora_linear_fwd: tensor map encoding failed");
-    if (rc) return fail(NF4_ERR_CUDA, "qlora_linear_fwd launch: %s", cudaGetErrorString(cudaGetLastError()));
+    if (rc) return fail(NF4_ERR_CUDA, "qlora_linear_fwd launch: %s", cudaGetErrorString(layer_last_cuda_error()));
     return ok();
 }
 
@@ -228,7 +228,7 @@ int qlora_linear_bwd(const nf4_tensor* w, const uint16_t* A, const uint16_t* B, 
     rc = layer_bwd(c, A, B, r, scaling, X, T_saved, dY, M, dX, dA, dB, accumulate_grads,
                    static_cast<uint8_t*>(ws));
     if (rc == -1) return fail(NF4_ERR_CUDA, "qlora_linear_bwd: tensor map encoding failed");
-    if (rc) return fail(NF4_ERR_CUDA, "qlora_linear_bwd launch: %s", cudaGetErrorString(cudaGetLastError()));
+    if (rc) return fail(NF4_ERR_CUDA, "qlora_linear_bwd launch: %s", cudaGetErrorString(layer_last_cuda_error()));
     return ok();
 }
 

@@ -24,8 +24,21 @@
 
 #include "gemm.cuh"
 #include "layer.h"
+#include "trace.h"
 
 namespace nf4lora {
+
+// The CUDA error behind the last failed launch of this thread (for messages).
+static thread_local cudaError_t t_launch_error = cudaSuccess;
+static cudaError_t note(cudaError_t e) {
+    if (e != cudaSuccess) t_launch_error = e;
+    return e;
+}
+cudaError_t layer_last_cuda_error() {
+    const cudaError_t e = t_launch_error;
+    t_launch_error = cudaSuccess;
+    return e;
+}
 
 // ------------------------------------------------------------------ tensor maps
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -72,14 +85,28 @@ static bool map_codes(CUtensorMap* m, const uint8_t* codes, int64_t d_out, int64
 
 // ------------------------------------------------------------------ launch
 template <int BN, int ASRC, int BSRC, int AE, int BE, int EPI>
-static cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& ae,
+static cudaError_t launch(const char* name, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& ae,
                           const CUtensorMap& be, const GemmArgs& args, dim3 grid, cudaStream_t st) {
     using C = GemmConfig<BN, ASRC, BSRC, AE, BE, EPI>;
     auto kern = k_gemm<BN, ASRC, BSRC, AE, BE, EPI>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    kern<<<grid, C::kThreads, C::kSmemBytes, st>>>(a, b, ae, be, args);
-    return cudaGetLastError();
+    // the shared-memory opt-in is per device; set it once (also keeps it out of
+    // stream captures)
+    static bool configured[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return note(e);
+    if (dev < 0 || dev >= 64 || !configured[dev]) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+        if (e != cudaSuccess) return note(e);
+        if (dev >= 0 && dev < 64) configured[dev] = true;
+    }
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(C::kThreads);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = st;
+    TraceScope trace(name, st);
+    return note(cudaLaunchKernelEx(&cfg, kern, a, b, ae, be, args));
 }
 
 // Fixed-order sum over the split-K slices of an fp32 partial buffer:
@@ -137,8 +164,12 @@ static cudaError_t reduce(const ReduceArgs& a, int num_sms, cudaStream_t st) {
     int64_t grid = (total + 255) / 256;
     grid = std::min<int64_t>(grid, int64_t(num_sms) * 8);
     if (grid < 1) grid = 1;
-    k_reduce_splits<<<static_cast<unsigned>(grid), 256, 0, st>>>(a);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(256);
+    cfg.stream = st;
+    TraceScope trace("reduce_splits", st);
+    return note(cudaLaunchKernelEx(&cfg, k_reduce_splits, a));
 }
 
 static ReduceArgs reduce_args(const float* part, int splits, int64_t slice, int rows, int cols, int64_t ldp,
@@ -217,11 +248,12 @@ struct Maps {
 };
 
 template <int EPI, int ASRC, int BSRC>
-static cudaError_t launch_lora_gemm(int bn, const Maps& m, const GemmArgs& args, dim3 grid, cudaStream_t st) {
+static cudaError_t launch_lora_gemm(const char* name, int bn, const Maps& m, const GemmArgs& args, dim3 grid,
+                                    cudaStream_t st) {
     switch (bn) {
-        case 64: return launch<64, ASRC, BSRC, 0, 0, EPI>(m.a, m.b, m.ae, m.be, args, grid, st);
-        case 128: return launch<128, ASRC, BSRC, 0, 0, EPI>(m.a, m.b, m.ae, m.be, args, grid, st);
-        default: return launch<256, ASRC, BSRC, 0, 0, EPI>(m.a, m.b, m.ae, m.be, args, grid, st);
+        case 64: return launch<64, ASRC, BSRC, 0, 0, EPI>(name, m.a, m.b, m.ae, m.be, args, grid, st);
+        case 128: return launch<128, ASRC, BSRC, 0, 0, EPI>(name, m.a, m.b, m.ae, m.be, args, grid, st);
+        default: return launch<256, ASRC, BSRC, 0, 0, EPI>(name, m.a, m.b, m.ae, m.be, args, grid, st);
     }
 }
 
@@ -241,7 +273,7 @@ static int lora_down(const LayerCtx& c, const uint16_t* A, int r, float s, const
     g.ldp = r64;
     g.part_slice = M * r64;
     dim3 grid(ceil_div(M, 128), ceil_div(r64, bn), sp.splits);
-    if (launch_lora_gemm<EPI_F32_PART, SRC_TMA_K, SRC_TMA_K>(bn, m, g, grid, c.stream) != cudaSuccess) return -2;
+    if (launch_lora_gemm<EPI_F32_PART, SRC_TMA_K, SRC_TMA_K>("lora_down", bn, m, g, grid, c.stream) != cudaSuccess) return -2;
     ReduceArgs ra = reduce_args(part, sp.splits, M * r64, static_cast<int>(M), r64, r64, s, T2, 2 * r64);
     ra.lo_off = r64;
     ra.out32 = T_saved;
@@ -289,7 +321,7 @@ int layer_fwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, fl
         g.ldp = c.d_out;
         g.part_slice = M * c.d_out;
         dim3 grid(tiles, 1, sp.splits);
-        if (launch<16, SRC_DEC_K, SRC_TMA_K, 0, 0, EPI_F32_PART_T>(m.a, m.b, m.ae, m.be, g, grid, c.stream) !=
+        if (launch<16, SRC_DEC_K, SRC_TMA_K, 0, 0, EPI_F32_PART_T>("nf4_gemm_fwd_few", m.a, m.b, m.ae, m.be, g, grid, c.stream) !=
             cudaSuccess)
             return -2;
         ReduceArgs ra = reduce_args(part, sp.splits, M * c.d_out, static_cast<int>(M), static_cast<int>(c.d_out),
@@ -306,7 +338,7 @@ int layer_fwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, fl
     g.out = Y;
     g.ldo = c.d_out;
     dim3 grid(ceil_div(M, 128), ceil_div(c.d_out, 256), 1);
-    if (launch<256, SRC_TMA_K, SRC_DEC_K, 0, 0, EPI_BF16>(m.a, m.b, m.ae, m.be, g, grid, c.stream) != cudaSuccess)
+    if (launch<256, SRC_TMA_K, SRC_DEC_K, 0, 0, EPI_BF16>("nf4_gemm_fwd", m.a, m.b, m.ae, m.be, g, grid, c.stream) != cudaSuccess)
         return -2;
     return 0;
 }
@@ -344,7 +376,7 @@ int layer_bwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, fl
         g.ldp = r64;
         g.part_slice = M * r64;
         dim3 grid(ceil_div(M, 128), ceil_div(r64, bn), sp.splits);
-        if (launch_lora_gemm<EPI_F32_PART, SRC_TMA_K, SRC_TMA_MN>(bn, m, g, grid, c.stream) != cudaSuccess) return -2;
+        if (launch_lora_gemm<EPI_F32_PART, SRC_TMA_K, SRC_TMA_MN>("lora_v", bn, m, g, grid, c.stream) != cudaSuccess) return -2;
         ReduceArgs ra = reduce_args(part, sp.splits, M * r64, static_cast<int>(M), r64, r64, s, V2, 2 * r64);
         ra.lo_off = r64;
         if (reduce(ra, c.num_sms, c.stream) != cudaSuccess) return -2;
@@ -377,7 +409,7 @@ int layer_bwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, fl
             g.ldp = c.d_in;
             g.part_slice = M * c.d_in;
             dim3 grid(tiles, 1, sp.splits);
-            if (launch<16, SRC_DEC_MN, SRC_TMA_K, 1, 0, EPI_F32_PART_T>(m.a, m.b, m.ae, m.be, g, grid, c.stream) !=
+            if (launch<16, SRC_DEC_MN, SRC_TMA_K, 1, 0, EPI_F32_PART_T>("nf4_gemm_dx_few", m.a, m.b, m.ae, m.be, g, grid, c.stream) !=
                 cudaSuccess)
                 return -2;
             ReduceArgs ra = reduce_args(part, sp.splits, M * c.d_in, static_cast<int>(M), static_cast<int>(c.d_in),
@@ -394,7 +426,7 @@ int layer_bwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, fl
             g.out = dX;
             g.ldo = c.d_in;
             dim3 grid(ceil_div(M, 128), ceil_div(c.d_in, 256), 1);
-            if (launch<256, SRC_TMA_K, SRC_DEC_MN, 0, 1, EPI_BF16>(m.a, m.b, m.ae, m.be, g, grid, c.stream) !=
+            if (launch<256, SRC_TMA_K, SRC_DEC_MN, 0, 1, EPI_BF16>("nf4_gemm_dx", m.a, m.b, m.ae, m.be, g, grid, c.stream) !=
                 cudaSuccess)
                 return -2;
         }
@@ -404,9 +436,12 @@ int layer_bwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, fl
     // ---- dB = dY^T T: D[n, c] = sum_m dY[m, n] T2[m, c], then dB[n, j] = D[n, j] + D[n, j + r64]
     if (dB != nullptr) {
         if (T_saved != nullptr) {
-            k_split_from_f32<<<static_cast<unsigned>(std::min<int64_t>((M * r64 + 255) / 256, c.num_sms * 8)), 256, 0,
-                               c.stream>>>(T_saved, M, r, r64, T2);
-            if (cudaGetLastError() != cudaSuccess) return -2;
+            TraceScope trace("split_t", c.stream);
+            cudaLaunchConfig_t cfg{};
+            cfg.gridDim = dim3(static_cast<unsigned>(std::min<int64_t>((M * r64 + 255) / 256, c.num_sms * 8)));
+            cfg.blockDim = dim3(256);
+            cfg.stream = c.stream;
+            if (note(cudaLaunchKernelEx(&cfg, k_split_from_f32, T_saved, M, r, r64, T2)) != cudaSuccess) return -2;
         } else {
             int rc = lora_down(c, A, r, s, X, M, T2, nullptr, part);
             if (rc) return rc;
@@ -423,7 +458,7 @@ int layer_bwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, fl
         g.ldp = 2 * r64;
         g.part_slice = c.d_out * 2 * r64;
         dim3 grid(ceil_div(c.d_out, 128), ceil_div(2 * r64, bn2), sp.splits);
-        if (launch_lora_gemm<EPI_F32_PART, SRC_TMA_MN, SRC_TMA_MN>(bn2, m, g, grid, c.stream) != cudaSuccess) return -2;
+        if (launch_lora_gemm<EPI_F32_PART, SRC_TMA_MN, SRC_TMA_MN>("lora_db", bn2, m, g, grid, c.stream) != cudaSuccess) return -2;
         ReduceArgs ra = reduce_args(part, sp.splits, c.d_out * 2 * r64, static_cast<int>(c.d_out), r, 2 * r64, 1.0f, dB, r);
         ra.fold = r64;
         ra.accumulate = accumulate;
@@ -444,7 +479,7 @@ int layer_bwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, fl
         g.ldp = c.d_in;
         g.part_slice = int64_t(2 * r64) * c.d_in;
         dim3 grid(ceil_div(c.d_in, 128), ceil_div(2 * r64, bn2), sp.splits);
-        if (launch_lora_gemm<EPI_F32_PART_T, SRC_TMA_MN, SRC_TMA_MN>(bn2, m, g, grid, c.stream) != cudaSuccess)
+        if (launch_lora_gemm<EPI_F32_PART_T, SRC_TMA_MN, SRC_TMA_MN>("lora_da", bn2, m, g, grid, c.stream) != cudaSuccess)
             return -2;
         ReduceArgs ra = reduce_args(part, sp.splits, int64_t(2 * r64) * c.d_in, r, static_cast<int>(c.d_in), c.d_in,
                                     1.0f, dA, c.d_in);

@@ -25,6 +25,9 @@ struct LayerCtx {
 int64_t fwd_workspace_bytes(int64_t M, int64_t d_out, int64_t d_in, int r, int num_sms);
 int64_t bwd_workspace_bytes(int64_t M, int64_t d_out, int64_t d_in, int r, int num_sms);
 
+// The CUDA error of the last failed launch of the calling thread (then reset).
+cudaError_t layer_last_cuda_error();
+
 // Return 0 on success, -1 if a tensor map could not be encoded, -2 if a
 // launch failed.
 int layer_fwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, float s, const uint16_t* X,

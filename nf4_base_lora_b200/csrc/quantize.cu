@@ -13,6 +13,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "nf4_levels.cuh"
+#include "trace.h"
 
 namespace nf4lora {
 
@@ -208,19 +209,41 @@ __global__ void __launch_bounds__(256) k_nf4_dequantize(const uint8_t* __restric
 
 }  // namespace
 
+static cudaLaunchConfig_t config(int64_t grid, int block, cudaStream_t stream) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(block);
+    cfg.stream = stream;
+    return cfg;
+}
+
 cudaError_t launch_nf4_quantize(const float* W, int64_t n, uint8_t* codes, int8_t* qscale,
                                 float* scale2, float* scale_mean, float* ws_absmax,
                                 double* ws_tile_sums, int num_sms, cudaStream_t stream) {
     const int64_t n_blocks = n / 64;
     const int64_t n_tiles = (n_blocks + kTileBlocks - 1) / kTileBlocks;
     const int64_t grid1 = n_tiles < int64_t(num_sms) * 8 ? n_tiles : int64_t(num_sms) * 8;
-    k_nf4_encode<<<static_cast<unsigned>(grid1), 256, 0, stream>>>(W, n_blocks, codes, ws_absmax,
-                                                                   ws_tile_sums);
-    k_dq_mean<<<1, 1024, 0, stream>>>(ws_tile_sums, n_tiles, n_blocks, scale_mean);
-    const int64_t grid3 = (n_tiles + 7) / 8;
-    k_dq_quantize<<<static_cast<unsigned>(grid3), 256, 0, stream>>>(ws_absmax, n_blocks, scale_mean,
-                                                                    qscale, scale2);
-    return cudaGetLastError();
+    cudaError_t e;
+    {
+        TraceScope trace("nf4_encode", stream);
+        cudaLaunchConfig_t cfg = config(grid1, 256, stream);
+        e = cudaLaunchKernelEx(&cfg, k_nf4_encode, W, n_blocks, codes, ws_absmax, ws_tile_sums);
+        if (e != cudaSuccess) return e;
+    }
+    {
+        TraceScope trace("dq_mean", stream);
+        cudaLaunchConfig_t cfg = config(1, 1024, stream);
+        e = cudaLaunchKernelEx(&cfg, k_dq_mean, static_cast<const double*>(ws_tile_sums), n_tiles, n_blocks,
+                               scale_mean);
+        if (e != cudaSuccess) return e;
+    }
+    {
+        TraceScope trace("dq_quantize", stream);
+        cudaLaunchConfig_t cfg = config((n_tiles + 7) / 8, 256, stream);
+        e = cudaLaunchKernelEx(&cfg, k_dq_quantize, static_cast<const float*>(ws_absmax), n_blocks,
+                               static_cast<const float*>(scale_mean), qscale, scale2);
+    }
+    return e;
 }
 
 cudaError_t launch_nf4_dequantize(const uint8_t* codes, const int8_t* qscale, const float* scale2,
@@ -229,9 +252,9 @@ cudaError_t launch_nf4_dequantize(const uint8_t* codes, const int8_t* qscale, co
     const int64_t units = n / 16;
     int64_t grid = (units + 255) / 256;
     if (grid > int64_t(num_sms) * 16) grid = int64_t(num_sms) * 16;
-    k_nf4_dequantize<<<static_cast<unsigned>(grid), 256, 0, stream>>>(codes, qscale, scale2,
-                                                                      scale_mean, n, out);
-    return cudaGetLastError();
+    TraceScope trace("nf4_dequantize", stream);
+    cudaLaunchConfig_t cfg = config(grid, 256, stream);
+    return cudaLaunchKernelEx(&cfg, k_nf4_dequantize, codes, qscale, scale2, scale_mean, n, out);
 }
 
 }  // namespace nf4lora
