@@ -133,6 +133,30 @@ int nf4_quantize(const float* W, int64_t d_out, int64_t d_in, const nf4_tensor* 
                  void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * nf4_quantize_noalloc -- nf4_quantize without a workspace argument.  It
+ * exists for callers that are not allowed to allocate device memory: for
+ * example a plugin whose host framework owns every byte of device memory
+ * and hands out only the tensors it manages, or code that runs where a
+ * cudaMalloc would break a stream capture or a fixed memory budget.  The
+ * pages describe no such entry point; it is an interface convenience only.
+ *
+ * The scratch the encoder needs (the fp32 absmax of every block and the fp64
+ * tree partial sums) lives in a fixed array inside the library, sized for
+ * at most 4,194,304 blocks of 64 weights (d_out * d_in <= 268,435,456); that
+ * array (16 MiB + 128 KiB) stays resident on every GPU that loads the library
+ * until the process exits.  Larger weights return NF4_ERR_UNSUPPORTED_SHAPE.
+ * The call allocates nothing; the caller still passes W and `out`.
+ * The first call on a device looks up the array's device address with that
+ * device current; make that first call before any stream capture on the
+ * device.  Every call shares the one array, so calls whose kernels overlap
+ * on the GPU (different streams without ordering) race on it; calls on one
+ * stream, or otherwise ordered, are safe.  Results are bit-identical to
+ * nf4_quantize.  Returns NF4_OK or an error status (no message is recorded).
+ */
+int nf4_quantize_noalloc(const float* W, int64_t d_out, int64_t d_in, const nf4_tensor* out,
+                         void* stream);
+
+/*
  * nf4_dequantize -- W_hat [d_out, d_in] bfloat16 (device) from `w`, with the
  * bit-exact definition above ([QP] §6.1 double dequantisation, §6.2 BF16
  * compute dtype).  Materialises the whole weight; the layer calls below never

@@ -30,7 +30,7 @@ STATUS_NAMES = {0: "NF4_OK", -1: "NF4_ERR_INVALID_ARG", -2: "NF4_ERR_UNSUPPORTED
 # Every symbol the C ABI exports (include/nf4lora.h), in declaration order.
 ABI_SYMBOLS = ("nf4_packed_bytes", "nf4_tensor_from_buffer", "nf4_quantize_workspace_bytes",
                "qlora_fwd_workspace_bytes", "qlora_bwd_workspace_bytes", "nf4_quantize",
-               "nf4_dequantize", "qlora_linear_fwd", "qlora_linear_bwd",
+               "nf4_quantize_noalloc", "nf4_dequantize", "qlora_linear_fwd", "qlora_linear_bwd",
                "nf4lora_last_error_string", "nf4lora_device_status", "nf4lora_trace_start",
                "nf4lora_trace_stop", "nf4lora_trace_count", "nf4lora_trace_get", "nf4lora_version")
 
@@ -62,6 +62,7 @@ def _load() -> ctypes.CDLL:
         "qlora_fwd_workspace_bytes": (SZ, [I64, I64, I64, I]),
         "qlora_bwd_workspace_bytes": (SZ, [I64, I64, I64, I]),
         "nf4_quantize": (I, [P, I64, I64, S, P, SZ, P]),
+        "nf4_quantize_noalloc": (I, [P, I64, I64, S, P]),
         "nf4_dequantize": (I, [S, P, P]),
         "qlora_linear_fwd": (I, [S, P, P, I, F, P, I64, P, P, P, SZ, P]),
         "qlora_linear_bwd": (I, [S, P, P, I, F, P, P, P, I64, P, P, P, I, P, SZ, P]),
@@ -173,6 +174,19 @@ def nf4_quantize(W: torch.Tensor, out: Optional[NF4Tensor] = None) -> NF4Tensor:
     ws = _workspace(nf4_quantize_workspace_bytes(d_out, d_in), W.device)
     _check(lib.nf4_quantize(_ptr(W), d_out, d_in, ctypes.byref(out.struct), _ptr(ws),
                             0 if ws is None else ws.numel(), _stream()))
+    return out
+
+
+def nf4_quantize_noalloc(W: torch.Tensor, out: NF4Tensor) -> NF4Tensor:
+    """nf4_quantize for callers that cannot allocate device memory: the
+    library's built-in scratch replaces the workspace (at most 268,435,456
+    weights; calls that overlap on the GPU share that scratch and race)."""
+    if W.dtype != torch.float32 or not W.is_cuda or not W.is_contiguous() or W.dim() != 2:
+        raise ValueError("W must be a contiguous 2-D float32 CUDA tensor")
+    d_out, d_in = W.shape
+    status = lib.nf4_quantize_noalloc(_ptr(W), d_out, d_in, ctypes.byref(out.struct), _stream())
+    if status != NF4_OK:
+        raise Nf4Error(status, "nf4_quantize_noalloc failed")
     return out
 
 

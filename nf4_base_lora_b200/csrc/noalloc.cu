@@ -1,0 +1,82 @@
+// nf4_quantize_noalloc: the encoder with its scratch in a fixed device array
+// compiled into the library, for callers that cannot allocate device memory.
+//
+// Scratch of the encoder: the fp32 first-level absmax of every 64-block and
+// one fp64 partial sum per 256 blocks.  Here it lives in g_quant_scratch, a
+// file-scope __device__ array sized for kNoallocMaxBlocks blocks, which every
+// GPU that loads the library keeps until the process exits.  Host code must
+// not pass the symbol itself to a kernel (on the host it names a stand-in, not
+// device memory): the device address is fetched with cudaGetSymbolAddress
+// once per device, with that device current, on the first call made on it.
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "../../include/nf4lora.h"
+#include "kernels.h"
+
+namespace nf4lora {
+
+namespace {
+
+constexpr int64_t kNoallocMaxBlocks = int64_t(1) << 22;                 // 268,435,456 weights
+constexpr int64_t kNoallocMaxTiles = kNoallocMaxBlocks / 256;
+constexpr int64_t kAbsmaxBytes = kNoallocMaxBlocks * 4;                  // 16 MiB
+constexpr int64_t kScratchBytes = kAbsmaxBytes + kNoallocMaxTiles * 8;   // + 128 KiB
+
+static __device__ __align__(256) unsigned char g_quant_scratch[kScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of g_quant_scratch on the current device (set-up on first use).
+cudaError_t scratch_address(int dev, void** out) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_scratch_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_quant_scratch);
+        if (e != cudaSuccess) return e;
+        g_scratch_ptr[dev] = p;
+    }
+    *out = g_scratch_ptr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+
+}  // namespace nf4lora
+
+extern "C" int nf4_quantize_noalloc(const float* W, int64_t d_out, int64_t d_in, const nf4_tensor* out,
+                                    void* stream) {
+    using namespace nf4lora;
+    // Same checks as nf4_quantize, minus the workspace, plus the size limit.
+    if (W == nullptr || out == nullptr) return NF4_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(W) & 15u) != 0) return NF4_ERR_MISALIGNED;
+    const size_t packed = nf4_packed_bytes(d_out, d_in);
+    if (packed == 0) return NF4_ERR_UNSUPPORTED_SHAPE;
+    if (out->d_out != d_out || out->d_in != d_in || !out->codes || !out->qscale || !out->scale2 ||
+        !out->scale_mean)
+        return NF4_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(out->codes) & 15u) || (reinterpret_cast<uintptr_t>(out->qscale) & 15u) ||
+        (reinterpret_cast<uintptr_t>(out->scale2) & 15u) || (reinterpret_cast<uintptr_t>(out->scale_mean) & 3u))
+        return NF4_ERR_MISALIGNED;
+    const int64_t n = d_out * d_in, n_blocks = n / 64;
+    if (n_blocks > kNoallocMaxBlocks) return NF4_ERR_UNSUPPORTED_SHAPE;  // beyond the fixed scratch
+    int dev = 0, major = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return NF4_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return NF4_ERR_CUDA;
+    if (major != 10) return NF4_ERR_DEVICE;
+    void* scratch = nullptr;
+    if (scratch_address(dev, &scratch) != cudaSuccess) return NF4_ERR_CUDA;
+    unsigned char* base = static_cast<unsigned char*>(scratch);
+    // Every scratch word the kernels read is written earlier in the same call,
+    // so nothing needs clearing between calls.
+    const cudaError_t e = launch_nf4_quantize(W, n, out->codes, out->qscale, out->scale2, out->scale_mean,
+                                              reinterpret_cast<float*>(base),
+                                              reinterpret_cast<double*>(base + kAbsmaxBytes), sms,
+                                              static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? NF4_OK : NF4_ERR_CUDA;
+}
