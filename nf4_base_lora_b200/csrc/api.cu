@@ -7,7 +7,7 @@
 #include <cstdio>
 #include <string>
 
-#include "../../include/nf4lora.h"
+#include "nf4lora.h"
 #include "common.cuh"
 #include "kernels.h"
 #include "layer.h"

@@ -214,3 +214,46 @@ __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
 }
 
 }  // namespace nf4lora
+
+namespace nf4lora {
+
+// ------------------------------------------------------------------ clusters
+// Thread-block clusters: CTAs of one cluster run together on one GPC and can
+// read each other's shared memory (distributed shared memory).
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// All threads of all CTAs of the cluster: release this CTA's shared-memory
+// writes, then wait for every other CTA to arrive.
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t cluster_map(uint32_t smem_addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr), "r"(rank));
+    return r;
+}
+
+// Remote shared-memory loads.  Volatile, so they stay after the (volatile)
+// cluster barrier; no memory clobber, so a run of them is issued back to back
+// before the first use of their results.
+__device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+        : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+        : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+    return v;
+}
+
+}  // namespace nf4lora

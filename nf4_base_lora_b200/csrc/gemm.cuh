@@ -28,9 +28,18 @@
 //
 // Warp roles: warp 0 = TMA producer (one lane), warp 1 = TMEM allocator and
 // MMA issuer (one lane), warps 2.. = decoders, then epilogue (TMEM -> regs ->
-// global).  Stages are ring-buffered with mbarriers: full (TMA bytes landed),
-// dec (decoded tile written), empty (MMAs that read the stage completed).
-// Every wait is bounded (see common.cuh).
+// global).  With two decode teams, team t decodes the k-steps t, t + 2, ...  Two rings of shared-memory stages, each with mbarriers:
+//   load ring   (deep, small slots): the TMA-copied operand and the packed
+//               codes; full = bytes landed, empty = MMAs that read it done;
+//   decode ring (shallow, one decoded bf16 tile per slot): dfull = decode
+//               warps wrote it, dempty = MMAs that read it done.
+// The deep load ring keeps many HBM requests in flight while only a few
+// decoded tiles occupy shared memory.  Every wait is bounded (common.cuh).
+//
+// Split-K over few tokens: the splits of one tile form a thread-block cluster
+// along grid.z; each CTA writes its fp32 partial tile to the workspace, one
+// cluster barrier makes them visible, and CTA rank 0 adds them in split order
+// -- no atomics or counters, the same sum on every run.
 #pragma once
 
 #include <cstdint>
@@ -41,7 +50,7 @@
 namespace nf4lora {
 
 enum OpSrc : int { SRC_TMA_K = 0, SRC_TMA_MN = 1, SRC_DEC_K = 2, SRC_DEC_MN = 3 };
-enum EpiKind : int { EPI_BF16 = 0, EPI_F32_PART = 1, EPI_F32_PART_T = 2 };
+enum EpiKind : int { EPI_BF16 = 0, EPI_F32_PART = 1, EPI_F32_PART_T = 2, EPI_CLUSTER_BF16_T = 3 };
 
 struct GemmArgs {
     int rows;           // valid rows of D over the whole problem
@@ -59,11 +68,15 @@ struct GemmArgs {
     int64_t w_blocks_per_row; // d_in / 64
     // epilogue
     float alpha;
-    uint16_t* out;      // EPI_BF16: out[row * ldo + col]
+    uint16_t* out;      // EPI_BF16: out[row * ldo + col]; EPI_CLUSTER_BF16_T: out[col * ldo + row]
     int64_t ldo;
-    float* part;        // EPI_F32_PART: part[z * part_slice + row * ldp + col]
+    float* part;        // EPI_F32_PART: part[z * part_slice + row * ldp + col];
+                        // EPI_CLUSTER_BF16_T: [tile][split][128][BN] fp32 slots
     int64_t ldp;        // EPI_F32_PART_T: part[z * part_slice + col * ldp + row]
     int64_t part_slice;
+    // 1: the kernel runs as a programmatic dependent of the previous kernel on
+    // the stream, which produces the extension operand.
+    int pdl;
 };
 
 template <int SRC>
@@ -72,7 +85,7 @@ struct OpTraits {
     static constexpr bool kMN = (SRC == SRC_TMA_MN || SRC == SRC_DEC_MN);
 };
 
-template <int BN, int ASRC, int BSRC, int AE_MN, int BE_MN, int EPI>
+template <int BN, int ASRC, int BSRC, int AE_MN, int BE_MN, int EPI, int LSTAGES = 0, int DSTAGES = 0, int TEAMS = 1>
 struct GemmConfig {
     static constexpr int kBM = 128;
     static constexpr int kBK = 64;
@@ -80,23 +93,40 @@ struct GemmConfig {
     static constexpr bool kDecB = OpTraits<BSRC>::kDecoded;
     static_assert(!(kDecA && kDecB), "at most one decoded operand");
     static constexpr bool kHasDec = kDecA || kDecB;
+    static constexpr int kTeams = kHasDec ? TEAMS : 1;
     static constexpr int kABytes = kBM * kBK * 2;             // 16 KB
     static constexpr int kBBytes = BN * kBK * 2;
     static constexpr int kDecMN = kDecA ? kBM : (kDecB ? BN : 0);  // decoded tile's M/N width
-    static constexpr int kCBytes = kDecMN * 32;               // packed codes per stage
-    static constexpr int kStageBytes = kABytes + kBBytes + kCBytes;
-    static constexpr int kStagesRaw = (225 * 1024) / kStageBytes;
-    static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
-    static_assert(kStages >= 2, "tile too large");
-    static constexpr int kDecThreads = kDecMN;                // one (row, block) unit each
-    static constexpr int kDecWarps = kDecThreads / 32;
+    static constexpr int kCBytes = kDecMN * 32;               // packed codes per k-step
+    // load slot: [A tile or A codes | B tile or B codes]; decode slot: the decoded tile
+    static constexpr int kLoadA = kDecA ? kCBytes : kABytes;
+    static constexpr int kLoadB = kDecB ? kCBytes : kBBytes;
+    static constexpr int kLoadSlot = kLoadA + kLoadB;
+    static constexpr int kDecSlot = kDecA ? kABytes : (kDecB ? kBBytes : 0);
+    static constexpr int kDS = kHasDec ? (DSTAGES > 0 ? DSTAGES : 3 * kTeams) : 1;
+    static_assert(kDS % kTeams == 0, "each team must own whole decode slots");
+    static constexpr int kBudget = 225 * 1024 - (kHasDec ? kDS * kDecSlot : 0);
+    static constexpr int kLSRaw = kBudget / kLoadSlot;
+    static constexpr int kLSCap = kHasDec ? 2 * kDS : 8;
+    static constexpr int kLSAuto = kLSRaw < kLSCap ? kLSRaw : kLSCap;
+    static constexpr int kLS = LSTAGES > 0 ? LSTAGES : (kLSAuto > 8 ? 8 : kLSAuto);
+    static_assert(kLS >= 2, "tile too large");
+    // The producer runs at most kLS k-steps ahead of the MMAs.  Its first
+    // parity wait on a decode slot (extension k-steps) is unambiguous only if
+    // it cannot be two phases ahead of that slot, i.e. kLS <= 2 * kDS.
+    static_assert(!kHasDec || kLS <= 2 * kDS, "load ring too deep for the decode ring");
+    static_assert(kLoadA % 1024 == 0 && kLoadSlot % 1024 == 0 && kDecSlot % 1024 == 0, "swizzle alignment");
+    static constexpr int kTeamThreads = kDecMN;               // one (row, block) unit each
+    static constexpr int kTeamWarps = kTeamThreads / 32;
+    static constexpr int kDecWarps = kTeamWarps * kTeams;
     static constexpr int kWorkWarps = kDecWarps > 4 ? kDecWarps : 4;
     static constexpr int kThreads = 64 + 32 * kWorkWarps;
     static constexpr int kTmemCols = BN < 32 ? 32 : BN;
-    static constexpr int kSmemBytes = kStages * kStageBytes + 1024;
-    // transaction bytes of one stage
-    static constexpr int kTxMain = (kDecA ? kCBytes : kABytes) + (kDecB ? kCBytes : kBBytes);
-    static constexpr int kTxExt = kABytes + kBBytes;
+    static constexpr int kSmemBytes = kLS * kLoadSlot + (kHasDec ? kDS * kDecSlot : 0) + 1024;
+    // CTAs per SM the configuration is built for (registers are capped to fit)
+    static constexpr int kMinBlocks = kSmemBytes <= 110 * 1024 ? 2 : 1;
+    static constexpr int kTxMain = kLoadA + kLoadB;            // bytes TMA lands per main k-step
+    static constexpr int kTxExt = kABytes + kBBytes;           // per extension k-step
     static constexpr uint32_t kIdescMain =
         make_idesc_bf16(kBM, BN, OpTraits<ASRC>::kMN ? 1 : 0, OpTraits<BSRC>::kMN ? 1 : 0);
     static constexpr uint32_t kIdescExt = make_idesc_bf16(kBM, BN, AE_MN, BE_MN);
@@ -134,6 +164,17 @@ __device__ __forceinline__ void zero_row(uint8_t* dst_row) {
     for (int j = 0; j < 8; ++j) *reinterpret_cast<uint4*>(dst_row + (j << 4)) = make_uint4(0, 0, 0, 0);
 }
 
+// Programmatic dependent launch: block until the preceding kernel on the
+// stream has completed and its writes are visible (returns at once when the
+// kernel was not launched as a dependent).
+__device__ __forceinline__ void grid_dependency_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void named_barrier_sync(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
 // Bounded wait that ignores the abort flag: used only to drain copies that
 // are still in flight when a CTA gives up.
 __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
@@ -143,15 +184,18 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
     }
 }
 
-template <int BN, int ASRC, int BSRC, int AE_MN, int BE_MN, int EPI>
-__global__ void __launch_bounds__(GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI>::kThreads, 1)
+template <int BN, int ASRC, int BSRC, int AE_MN, int BE_MN, int EPI, int LSTAGES = 0, int DSTAGES = 0, int TEAMS = 1>
+__global__ void __launch_bounds__(GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI, LSTAGES, DSTAGES, TEAMS>::kThreads,
+                                  GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI, LSTAGES, DSTAGES, TEAMS>::kMinBlocks)
     k_gemm(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
            const __grid_constant__ CUtensorMap map_ae, const __grid_constant__ CUtensorMap map_be,
            const GemmArgs args) {
-    using C = GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI>;
-    constexpr int S = C::kStages;
+    using C = GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI, LSTAGES, DSTAGES, TEAMS>;
+    constexpr int LS = C::kLS;
+    constexpr int DS = C::kDS;
+    constexpr int kEpiThreads = C::kWorkWarps * 32;
     extern __shared__ uint8_t smem_raw[];
-    __shared__ uint64_t bar_full[S], bar_dec[S], bar_empty[S], bar_accum;
+    __shared__ uint64_t bar_full[LS], bar_empty[LS], bar_dfull[DS], bar_dempty[DS], bar_accum;
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
     __shared__ float s_lut[16];
@@ -160,124 +204,159 @@ __global__ void __launch_bounds__(GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI>:
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base_u32 = (raw + 1023u) & ~1023u;
     uint8_t* base = smem_raw + (base_u32 - raw);
-    auto a_tile = [&](int s) { return base + s * C::kABytes; };
-    auto b_tile = [&](int s) { return base + S * C::kABytes + s * C::kBBytes; };
-    auto c_tile = [&](int s) { return base + S * (C::kABytes + C::kBBytes) + s * C::kCBytes; };
+    auto load_slot = [&](int it) { return base + (it % LS) * C::kLoadSlot; };
+    auto dec_slot = [&](int it) { return base + LS * C::kLoadSlot + (it % DS) * C::kDecSlot; };
+    // operand tiles and codes of iteration `it`
+    auto a_buf = [&](int it) { return C::kDecA ? dec_slot(it) : load_slot(it); };
+    auto b_buf = [&](int it) { return C::kDecB ? dec_slot(it) : load_slot(it) + C::kLoadA; };
+    auto codes_buf = [&](int it) { return load_slot(it) + (C::kDecA ? 0 : C::kLoadA); };
 
     const int r0 = blockIdx.x * C::kBM;
     const int c0 = blockIdx.y * BN;
     const int z = blockIdx.z;
-    const int kb_begin = z * args.k_per_split;
-    int kb_end = kb_begin + args.k_per_split;
-    if (kb_end > args.k_main) kb_end = args.k_main;
+    int kb_begin, kb_end;
+    if constexpr (EPI == EPI_CLUSTER_BF16_T) {
+        // spread main + extension k-steps evenly over the splits, split 0
+        // (which also runs the extension) taking correspondingly fewer main ones
+        const int splits = static_cast<int>(gridDim.z);
+        const int total = args.k_main + args.k_ext;
+        const int per = total / splits, extra = total % splits;
+        auto start = [&](int zz) {  // first iteration index (main + ext numbering) of split zz
+            return zz * per + (zz < extra ? zz : extra);
+        };
+        const int it0 = start(z), it1 = start(z + 1);
+        // split 0 owns iterations [0, it1): its k_ext extension steps come first in
+        // this numbering, so its main range is [0, it1 - k_ext)
+        kb_begin = z == 0 ? 0 : it0 - args.k_ext;
+        kb_end = it1 - args.k_ext;
+        if (kb_end > args.k_main) kb_end = args.k_main;
+        if (kb_begin < 0) kb_begin = 0;
+    } else {
+        kb_begin = z * args.k_per_split;
+        kb_end = kb_begin + args.k_per_split;
+        if (kb_end > args.k_main) kb_end = args.k_main;
+    }
     const int n_main = kb_end > kb_begin ? kb_end - kb_begin : 0;
     const int n_ext = (z == 0) ? args.k_ext : 0;
     const int n_iter = n_main + n_ext;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < S; ++s) {
-            mbar_init(&bar_full[s], 1);
-            mbar_init(&bar_dec[s], C::kDecWarps > 0 ? C::kDecWarps : 1);
-            mbar_init(&bar_empty[s], 1);
+        for (int i = 0; i < LS; ++i) {
+            mbar_init(&bar_full[i], 1);
+            mbar_init(&bar_empty[i], 1);
+        }
+        for (int i = 0; i < DS; ++i) {
+            mbar_init(&bar_dfull[i], C::kTeamWarps > 0 ? C::kTeamWarps : 1);
+            mbar_init(&bar_dempty[i], 1);
         }
         mbar_init(&bar_accum, 1);
         s_abort = 0;
         fence_barrier_init();
     }
     if (threadIdx.x < 16) s_lut[threadIdx.x] = nf4_level(threadIdx.x);
-    if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&map_a);
-        tma_prefetch_desc(&map_b);
-        if (n_ext > 0) {
-            tma_prefetch_desc(&map_ae);
-            tma_prefetch_desc(&map_be);
-        }
+    // thread 0 initialised the barriers and is the producer: it goes straight
+    // on to issue copies while the other threads wait for the barriers here
+    // (non-aligned barrier forms: lane 0 of warp 0 arrives while its other
+    // lanes wait)
+    if (threadIdx.x == 0) {
+        asm volatile("barrier.arrive 3, %0;" ::"r"(C::kThreads) : "memory");
+    } else {
+        asm volatile("barrier.sync 3, %0;" ::"r"(C::kThreads) : "memory");
     }
-    if (warp == 1) {
-        tmem_alloc(&s_tmem, C::kTmemCols);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem_d = s_tmem;
     volatile int* abort_flag = &s_abort;
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
+        // (starts while warp 1 is still allocating tensor memory)
         if (lane == 0) {
+            tma_prefetch_desc(&map_a);
+            tma_prefetch_desc(&map_b);
+            if (n_ext > 0) {
+                tma_prefetch_desc(&map_ae);
+                tma_prefetch_desc(&map_be);
+            }
             int issued = 0;
             for (int it = 0; it < n_iter; ++it) {
-                const int s = it % S;
-                const uint32_t ph = (it / S) & 1u;
-                if (it >= S && !mbar_wait(&bar_empty[s], ph ^ 1u, abort_flag)) break;
+                if (it >= LS && !mbar_wait(&bar_empty[it % LS], ((it / LS) & 1u) ^ 1u, abort_flag)) break;
                 if (*abort_flag) break;
-                uint64_t* bar = &bar_full[s];
+                uint64_t* bar = &bar_full[it % LS];
                 if (it < n_main) {
                     const int kb = kb_begin + it;
                     mbar_arrive_expect_tx(bar, C::kTxMain);
                     // operand A
                     if constexpr (ASRC == SRC_TMA_K) {
-                        tma_load_2d(a_tile(s), &map_a, bar, kb * 64, r0);
+                        tma_load_2d(a_buf(it), &map_a, bar, kb * 64, r0);
                     } else if constexpr (ASRC == SRC_TMA_MN) {
-                        tma_load_2d(a_tile(s), &map_a, bar, r0, kb * 64);
-                        tma_load_2d(a_tile(s) + 8192, &map_a, bar, r0 + 64, kb * 64);
+                        tma_load_2d(a_buf(it), &map_a, bar, r0, kb * 64);
+                        tma_load_2d(a_buf(it) + 8192, &map_a, bar, r0 + 64, kb * 64);
                     } else if constexpr (ASRC == SRC_DEC_K) {
-                        tma_load_2d(c_tile(s), &map_a, bar, kb * 32, r0);
+                        tma_load_2d(codes_buf(it), &map_a, bar, kb * 32, r0);
                     } else {
-                        tma_load_2d(c_tile(s), &map_a, bar, r0 / 2, kb * 64);
+                        tma_load_2d(codes_buf(it), &map_a, bar, r0 / 2, kb * 64);
                     }
                     // operand B
                     if constexpr (BSRC == SRC_TMA_K) {
-                        tma_load_2d(b_tile(s), &map_b, bar, kb * 64, c0);
+                        tma_load_2d(b_buf(it), &map_b, bar, kb * 64, c0);
                     } else if constexpr (BSRC == SRC_TMA_MN) {
 #pragma unroll
                         for (int c = 0; c < BN / 64; ++c)
-                            tma_load_2d(b_tile(s) + c * 8192, &map_b, bar, c0 + c * 64, kb * 64);
+                            tma_load_2d(b_buf(it) + c * 8192, &map_b, bar, c0 + c * 64, kb * 64);
                     } else if constexpr (BSRC == SRC_DEC_K) {
-                        tma_load_2d(c_tile(s), &map_b, bar, kb * 32, c0);
+                        tma_load_2d(codes_buf(it), &map_b, bar, kb * 32, c0);
                     } else {
-                        tma_load_2d(c_tile(s), &map_b, bar, c0 / 2, kb * 64);
+                        tma_load_2d(codes_buf(it), &map_b, bar, c0 / 2, kb * 64);
                     }
                 } else {
                     const int j = it - n_main;
+                    // an extension tile on the decoded side lands in a decode slot
+                    if (C::kHasDec && it >= DS &&
+                        !mbar_wait(&bar_dempty[it % DS], ((it / DS) & 1u) ^ 1u, abort_flag))
+                        break;
+                    // the extension operand comes from the preceding kernel
+                    if (j == 0 && args.pdl) grid_dependency_wait();
                     const int ja = args.ext_wrap_a > 0 ? j % args.ext_wrap_a : j;
                     const int jb = args.ext_wrap_b > 0 ? j % args.ext_wrap_b : j;
                     mbar_arrive_expect_tx(bar, C::kTxExt);
                     if constexpr (AE_MN) {
-                        tma_load_2d(a_tile(s), &map_ae, bar, r0, ja * 64);
-                        tma_load_2d(a_tile(s) + 8192, &map_ae, bar, r0 + 64, ja * 64);
+                        tma_load_2d(a_buf(it), &map_ae, bar, r0, ja * 64);
+                        tma_load_2d(a_buf(it) + 8192, &map_ae, bar, r0 + 64, ja * 64);
                     } else {
-                        tma_load_2d(a_tile(s), &map_ae, bar, ja * 64, r0);
+                        tma_load_2d(a_buf(it), &map_ae, bar, ja * 64, r0);
                     }
                     if constexpr (BE_MN) {
 #pragma unroll
                         for (int c = 0; c < BN / 64; ++c)
-                            tma_load_2d(b_tile(s) + c * 8192, &map_be, bar, c0 + c * 64, jb * 64);
+                            tma_load_2d(b_buf(it) + c * 8192, &map_be, bar, c0 + c * 64, jb * 64);
                     } else {
-                        tma_load_2d(b_tile(s), &map_be, bar, jb * 64, c0);
+                        tma_load_2d(b_buf(it), &map_be, bar, jb * 64, c0);
                     }
                 }
                 ++issued;
             }
             if (*abort_flag) {
                 // let the copies already issued land before the CTA exits
-                const int first = issued > S ? issued - S : 0;
-                for (int it = first; it < issued; ++it) mbar_drain(&bar_full[it % S], (it / S) & 1u);
+                const int first = issued > LS ? issued - LS : 0;
+                for (int it = first; it < issued; ++it) mbar_drain(&bar_full[it % LS], (it / LS) & 1u);
             }
         }
     } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
+        // ------------------------------------------------------------ TMEM + MMA issuer
+        tmem_alloc(&s_tmem, C::kTmemCols);
+        tmem_relinquish();
+        tc_fence_before();
+        // hand the tensor-memory address to the epilogue warps
+        asm volatile("bar.arrive 2, %0;" ::"r"(32 + kEpiThreads) : "memory");
+        __syncwarp();
+        tc_fence_after();
+        const uint32_t tmem_d = s_tmem;
         if (lane == 0) {
             for (int it = 0; it < n_iter; ++it) {
-                const int s = it % S;
-                const uint32_t ph = (it / S) & 1u;
-                if (!mbar_wait(&bar_full[s], ph, abort_flag)) break;
+                if (!mbar_wait(&bar_full[it % LS], (it / LS) & 1u, abort_flag)) break;
                 const bool is_main = it < n_main;
-                if (C::kHasDec && is_main && !mbar_wait(&bar_dec[s], ph, abort_flag)) break;
+                if (C::kHasDec && is_main && !mbar_wait(&bar_dfull[it % DS], (it / DS) & 1u, abort_flag)) break;
                 tc_fence_after();
-                const uint32_t a_base = smem_u32(a_tile(s));
-                const uint32_t b_base = smem_u32(b_tile(s));
+                const uint32_t a_base = smem_u32(a_buf(it));
+                const uint32_t b_base = smem_u32(b_buf(it));
                 const bool a_mn = is_main ? OpTraits<ASRC>::kMN : (AE_MN != 0);
                 const bool b_mn = is_main ? OpTraits<BSRC>::kMN : (BE_MN != 0);
                 const uint32_t idesc = is_main ? C::kIdescMain : C::kIdescExt;
@@ -286,7 +365,8 @@ __global__ void __launch_bounds__(GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI>:
                     mma_bf16_ss(tmem_d, tile_desc(a_base, a_mn, kk), tile_desc(b_base, b_mn, kk), idesc,
                                 (it > 0 || kk > 0) ? 1u : 0u);
                 }
-                mma_commit(&bar_empty[s]);
+                mma_commit(&bar_empty[it % LS]);
+                if (C::kHasDec) mma_commit(&bar_dempty[it % DS]);
             }
             mma_commit(&bar_accum);
         }
@@ -295,46 +375,79 @@ __global__ void __launch_bounds__(GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI>:
         // ------------------------------------------------------------ decoders
         if constexpr (C::kHasDec) {
             if (ew < C::kDecWarps) {
-                const int dt = threadIdx.x - 64;
-                const float mu = *args.scale_mean;
+                const int team = ew / C::kTeamWarps;
+                const int dt = threadIdx.x - 64 - team * C::kTeamThreads;
+                const float mu = __ldg(args.scale_mean);
                 constexpr bool kMNdec = C::kDecA ? (ASRC == SRC_DEC_MN) : (BSRC == SRC_DEC_MN);
                 constexpr int kCB = C::kDecMN / 64;           // 64-blocks across the decoded tile
                 const int tile_mn0 = C::kDecA ? r0 : c0;
-                for (int it = 0; it < n_main; ++it) {
-                    const int s = it % S;
-                    const uint32_t ph = (it / S) & 1u;
+                // (weight row, 64-block) decoded by this thread at main step `it`
+                auto unit = [&](int it, int64_t& wrow, int64_t& wblk) {
                     const int kb = kb_begin + it;
-                    int64_t wrow, wblk;
-                    int dst_off, swz;
                     if constexpr (!kMNdec) {
                         wrow = tile_mn0 + dt;
                         wblk = kb;
-                        dst_off = dt * 128;
-                        swz = dt & 7;
                     } else {
-                        const int n_local = dt / kCB, c = dt % kCB;
-                        wrow = static_cast<int64_t>(kb) * 64 + n_local;
-                        wblk = tile_mn0 / 64 + c;
-                        dst_off = c * 8192 + n_local * 128;
-                        swz = n_local & 7;
+                        wrow = static_cast<int64_t>(kb) * 64 + dt / kCB;
+                        wblk = tile_mn0 / 64 + dt % kCB;
                     }
-                    const bool valid = wrow < args.w_rows && wblk < args.w_blocks_per_row;
-                    float sc = 0.0f;
-                    if (valid) {
+                };
+                int dst_off, swz;
+                if constexpr (!kMNdec) {
+                    dst_off = dt * 128;
+                    swz = dt & 7;
+                } else {
+                    const int n_local = dt / kCB, c = dt % kCB;
+                    dst_off = c * 8192 + n_local * 128;
+                    swz = n_local & 7;
+                }
+                // Block scales are prefetched kPf of this team's steps ahead
+                // into registers, so no decode waits on a dependent load.
+                constexpr int kPf = 4;
+                constexpr int kStride = C::kTeams;
+                int8_t q_pf[kPf];
+                float a2_pf[kPf];
+                bool ok_pf[kPf];
+                auto fetch = [&](int it, int slot) {
+                    int64_t wrow, wblk;
+                    unit(it, wrow, wblk);
+                    ok_pf[slot] = it < n_main && wrow < args.w_rows && wblk < args.w_blocks_per_row;
+                    if (ok_pf[slot]) {
                         const int64_t bidx = wrow * args.w_blocks_per_row + wblk;
-                        sc = nf4_block_scale(__ldg(args.qscale + bidx), __ldg(args.scale2 + (bidx >> 8)), mu);
+                        q_pf[slot] = __ldg(args.qscale + bidx);
+                        a2_pf[slot] = __ldg(args.scale2 + (bidx >> 8));
                     }
-                    if (!mbar_wait(&bar_full[s], ph, abort_flag)) break;
-                    uint8_t* dst = (C::kDecA ? a_tile(s) : b_tile(s)) + dst_off;
-                    if (valid) decode_unit(c_tile(s) + dt * 32, sc, dst, swz, s_lut);
-                    else zero_row(dst);
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&bar_dec[s]);
+                };
+#pragma unroll
+                for (int u = 0; u < kPf; ++u) fetch(team + u * kStride, u);
+                bool stop = false;
+                for (int base_it = team; base_it < n_main && !stop; base_it += kPf * kStride) {
+#pragma unroll
+                    for (int u = 0; u < kPf; ++u) {
+                        const int it = base_it + u * kStride;
+                        if (it >= n_main) break;
+                        const bool valid = ok_pf[u];
+                        const float sc = valid ? nf4_block_scale(q_pf[u], a2_pf[u], mu) : 0.0f;
+                        fetch(it + kPf * kStride, u);
+                        if (!mbar_wait(&bar_full[it % LS], (it / LS) & 1u, abort_flag) ||
+                            (it >= DS && !mbar_wait(&bar_dempty[it % DS], ((it / DS) & 1u) ^ 1u, abort_flag))) {
+                            stop = true;
+                            break;
+                        }
+                        uint8_t* dst = dec_slot(it) + dst_off;
+                        if (valid) decode_unit(codes_buf(it) + dt * 32, sc, dst, swz, s_lut);
+                        else zero_row(dst);
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&bar_dfull[it % DS]);
+                    }
                 }
             }
         }
         // ------------------------------------------------------------ epilogue
+        asm volatile("bar.sync 2, %0;" ::"r"(32 + kEpiThreads) : "memory");
+        tc_fence_after();
+        const uint32_t tmem_d = s_tmem;
         const int q = warp & 3;                       // TMEM lane quadrant of this warp
         constexpr int kColSplit = C::kWorkWarps / 4;  // warps sharing one quadrant
         const int part_idx = ew / 4;
@@ -342,7 +455,7 @@ __global__ void __launch_bounds__(GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI>:
         const int cbeg = part_idx * cw;
         const bool ok = mbar_wait(&bar_accum, 0, abort_flag);
         tc_fence_after();
-        if (ok && !*abort_flag) {
+        if constexpr (EPI != EPI_CLUSTER_BF16_T) if (ok && !*abort_flag) {
             const int row = r0 + q * 32 + lane;
             const bool row_ok = row < args.rows;
             for (int cc = cbeg; cc < cbeg + cw; cc += 32) {
@@ -388,7 +501,7 @@ __global__ void __launch_bounds__(GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI>:
                                 if (col + j < args.cols) dst[j] = __uint_as_float(v[j]);
                         }
                     }
-                } else {
+                } else {  // EPI_F32_PART_T
                     if (row_ok) {
                         float* dst = args.part + z * args.part_slice + row;
 #pragma unroll
@@ -398,13 +511,72 @@ __global__ void __launch_bounds__(GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI>:
                 }
             }
         }
+        if constexpr (EPI == EPI_CLUSTER_BF16_T) {
+            // this CTA's fp32 partial tile [128 rows][BN], row-major, into the
+            // partial buffer (one slot per (tile, split); coalesced 16 B stores)
+            if (ew < 4 && ok && !*abort_flag) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tmem_d + (static_cast<uint32_t>(q * 32) << 16), v);
+                tmem_ld_wait();
+                float* dst = args.part + (static_cast<int64_t>(blockIdx.x) * gridDim.z + z) * (C::kBM * BN) +
+                             (q * 32 + lane) * BN;
+#pragma unroll
+                for (int j = 0; j < BN; j += 4)
+                    __stcg(reinterpret_cast<float4*>(dst + j),
+                           make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]),
+                                       __uint_as_float(v[j + 3])));
+            }
+        }
     }
 
+    if constexpr (EPI == EPI_CLUSTER_BF16_T) {
+        // one cluster barrier (release / acquire at cluster scope) makes every
+        // split's partial visible to rank 0, which adds them in split order
+        cluster_sync_all();
+        const int ew = warp - 2;
+        if (cluster_ctarank() == 0 && ew >= 0 && ew < 4 && !*abort_flag) {
+            const int rr = threadIdx.x - 64;              // one row per thread
+            const int row = r0 + rr;
+            const int splits = static_cast<int>(gridDim.z);
+            const float* src = args.part + static_cast<int64_t>(blockIdx.x) * splits * (C::kBM * BN) + rr * BN;
+            float acc[BN];
+#pragma unroll
+            for (int j = 0; j < BN; ++j) acc[j] = 0.0f;
+            for (int z0 = 0; z0 < splits; z0 += 4) {
+                float4 t[4][BN / 4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    if (z0 + u < splits)
+#pragma unroll
+                        for (int j = 0; j < BN / 4; ++j)
+                            t[u][j] = __ldcg(reinterpret_cast<const float4*>(src + (z0 + u) * (C::kBM * BN)) + j);
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    if (z0 + u < splits)
+#pragma unroll
+                        for (int j = 0; j < BN / 4; ++j) {
+                            acc[4 * j] += t[u][j].x;
+                            acc[4 * j + 1] += t[u][j].y;
+                            acc[4 * j + 2] += t[u][j].z;
+                            acc[4 * j + 3] += t[u][j].w;
+                        }
+            }
+            if (row < args.rows) {
+#pragma unroll
+                for (int j = 0; j < BN; ++j) {
+                    if (j < args.cols) {
+                        const __nv_bfloat16 h = __float2bfloat16_rn(acc[j] * args.alpha);
+                        args.out[static_cast<int64_t>(j) * args.ldo + row] = *reinterpret_cast<const uint16_t*>(&h);
+                    }
+                }
+            }
+        }
+    }
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_d, C::kTmemCols);
+        tmem_dealloc(s_tmem, C::kTmemCols);
     }
 }
 

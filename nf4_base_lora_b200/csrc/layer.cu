@@ -23,6 +23,7 @@
 #include <mutex>
 
 #include "gemm.cuh"
+#include "kernels.h"
 #include "layer.h"
 #include "trace.h"
 
@@ -84,11 +85,12 @@ static bool map_codes(CUtensorMap* m, const uint8_t* codes, int64_t d_out, int64
 }
 
 // ------------------------------------------------------------------ launch
-template <int BN, int ASRC, int BSRC, int AE, int BE, int EPI>
+template <int BN, int ASRC, int BSRC, int AE, int BE, int EPI, int LSTAGES = 0, int DSTAGES = 0, int TEAMS = 1>
 static cudaError_t launch(const char* name, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& ae,
-                          const CUtensorMap& be, const GemmArgs& args, dim3 grid, cudaStream_t st) {
-    using C = GemmConfig<BN, ASRC, BSRC, AE, BE, EPI>;
-    auto kern = k_gemm<BN, ASRC, BSRC, AE, BE, EPI>;
+                          const CUtensorMap& be, const GemmArgs& args, dim3 grid, cudaStream_t st,
+                          int cluster_z = 1) {
+    using C = GemmConfig<BN, ASRC, BSRC, AE, BE, EPI, LSTAGES, DSTAGES, TEAMS>;
+    auto kern = k_gemm<BN, ASRC, BSRC, AE, BE, EPI, LSTAGES, DSTAGES, TEAMS>;
     // the shared-memory opt-in is per device; set it once (also keeps it out of
     // stream captures)
     static bool configured[64] = {};
@@ -98,6 +100,11 @@ static cudaError_t launch(const char* name, const CUtensorMap& a, const CUtensor
     if (dev < 0 || dev >= 64 || !configured[dev]) {
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
         if (e != cudaSuccess) return note(e);
+        // all of the unified L1/shared array as shared memory, so that two
+        // ~100 KB CTAs (and clusters of them) fit on one SM
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess) return note(e);
         if (dev >= 0 && dev < 64) configured[dev] = true;
     }
     cudaLaunchConfig_t cfg{};
@@ -105,6 +112,25 @@ static cudaError_t launch(const char* name, const CUtensorMap& a, const CUtensor
     cfg.blockDim = dim3(C::kThreads);
     cfg.dynamicSmemBytes = C::kSmemBytes;
     cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    int n_attr = 0;
+    if (args.pdl) {
+        // may start while the previous kernel on the stream still runs; the
+        // kernel waits for it (griddepcontrol.wait) where it needs its output
+        attr[n_attr].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[n_attr].val.programmaticStreamSerializationAllowed = 1;
+        ++n_attr;
+    }
+    if (cluster_z > 1) {
+        // the split-K slices of one tile form a cluster along grid.z
+        attr[n_attr].id = cudaLaunchAttributeClusterDimension;
+        attr[n_attr].val.clusterDim.x = 1;
+        attr[n_attr].val.clusterDim.y = 1;
+        attr[n_attr].val.clusterDim.z = cluster_z;
+        ++n_attr;
+    }
+    cfg.attrs = n_attr ? attr : nullptr;
+    cfg.numAttrs = n_attr;
     TraceScope trace(name, st);
     return note(cudaLaunchKernelEx(&cfg, kern, a, b, ae, be, args));
 }
@@ -225,6 +251,25 @@ static inline int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + 
 static int bn_for(int cols) { return cols <= 64 ? 64 : (cols <= 128 ? 128 : 256); }
 
 static constexpr int kSmallM = 16;
+// few-token kernels: 6 load slots of 6 KB + 4 decoded tiles of 16 KB = 100 KB
+// (two CTAs per SM), two decode teams on alternate k-steps
+static constexpr int kFewLoad = 6;
+static constexpr int kFewDec = 4;
+static constexpr int kFewTeams = 2;
+
+// Split-K of the few-token kernels: a power of two <= 8 (the portable cluster
+// size) so that the splits of a tile form one cluster, filling about two CTAs
+// per SM and keeping at least two k-steps per split.
+static Split few_split(int tiles, int k_steps, int sms) {
+    int s = 1;
+    while (s < 8 && tiles * (s * 2) <= 2 * sms && k_steps >= 2 * (s * 2)) s *= 2;
+    int kps = (k_steps + s - 1) / s;
+    while (s > 1 && (s - 1) * kps >= k_steps) {  // never leave a split empty
+        s /= 2;
+        kps = (k_steps + s - 1) / s;
+    }
+    return {s, kps};
+}
 
 // The splits each split-K GEMM uses (the workspace query and the calls share them).
 static Split split_down(int64_t M, int64_t d_in, int sms) {
@@ -238,7 +283,7 @@ static Split split_tokens(int64_t rows, int r64, int64_t M, int sms) {
     return choose_split(tiles, ceil_div(M, 64), sms, 4);
 }
 static Split split_small(int64_t rows, int64_t k, int sms) {
-    return choose_split(ceil_div(rows, 128), ceil_div(k, 64), 2 * sms, 4);
+    return few_split(ceil_div(rows, 128), ceil_div(k, 64), sms);
 }
 
 // ------------------------------------------------------------------ layer ops
@@ -285,7 +330,8 @@ static int lora_down(const LayerCtx& c, const uint16_t* A, int r, float s, const
 int64_t fwd_workspace_bytes(int64_t M, int64_t d_out, int64_t d_in, int r, int num_sms) {
     const int r64 = round64(r);
     int64_t part = int64_t(split_down(M, d_in, num_sms).splits) * M * r64;
-    if (M <= kSmallM) part = std::max<int64_t>(part, int64_t(split_small(d_out, d_in, num_sms).splits) * M * d_out);
+    if (M <= kSmallM)
+        part = std::max<int64_t>(part, int64_t(split_small(d_out, d_in, num_sms).splits) * ceil_div(d_out, 128) * 128 * 16);
     return align256(M * r64 * 4) + align256(part * 4);
 }
 
@@ -294,8 +340,6 @@ int layer_fwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, fl
     const int r64 = round64(r), kx = r64 / 64;
     uint16_t* T2 = reinterpret_cast<uint16_t*>(ws);
     float* part = reinterpret_cast<float*>(ws + align256(M * r64 * 4));
-    int rc = lora_down(c, A, r, s, X, M, T2, T_saved, part);
-    if (rc) return rc;
     Maps m;
     GemmArgs g{};
     g.qscale = c.qscale;
@@ -307,27 +351,33 @@ int layer_fwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, fl
     g.k_ext = 2 * kx;
     g.alpha = 1.0f;
     if (M <= kSmallM) {
-        // swapped: D[n, m] = W_hat[n, :] . X[m, :] + B[n, :] . T[m, :]
+        // T on CUDA cores, then the swapped fused GEMM as its programmatic
+        // dependent: D[n, m] = W_hat[n, :] . X[m, :] + B[n, :] . T[m, :],
+        // split-K over a cluster per 128-row tile, reduced in the cluster.
+        const int tiles = ceil_div(c.d_out, 128);
+        if (note(launch_few_down(X, A, static_cast<int>(M), static_cast<int>(c.d_in), r, r64, s, T2, T_saved,
+                                 c.stream)) != cudaSuccess)
+            return -2;
         if (!map_codes(&m.a, c.codes, c.d_out, c.d_in, 32, 128) || !map_bf16(&m.b, X, c.d_in, M, c.d_in, 16) ||
             !map_bf16(&m.ae, B, r, c.d_out, r, 128) || !map_bf16(&m.be, T2, 2 * r64, M, 2 * r64, 16))
             return -1;
-        const int tiles = ceil_div(c.d_out, 128);
         const Split sp = split_small(c.d_out, c.d_in, c.num_sms);
         g.ext_wrap_a = kx;
         g.rows = static_cast<int>(c.d_out);
         g.cols = static_cast<int>(M);
         g.k_per_split = sp.k_per_split;
+        g.out = Y;
+        g.ldo = c.d_out;
         g.part = part;
-        g.ldp = c.d_out;
-        g.part_slice = M * c.d_out;
+        g.pdl = 1;
         dim3 grid(tiles, 1, sp.splits);
-        if (launch<16, SRC_DEC_K, SRC_TMA_K, 0, 0, EPI_F32_PART_T>("nf4_gemm_fwd_few", m.a, m.b, m.ae, m.be, g, grid, c.stream) !=
-            cudaSuccess)
+        if (launch<16, SRC_DEC_K, SRC_TMA_K, 0, 0, EPI_CLUSTER_BF16_T, kFewLoad, kFewDec, kFewTeams>(
+                "nf4_gemm_fwd_few", m.a, m.b, m.ae, m.be, g, grid, c.stream, sp.splits) != cudaSuccess)
             return -2;
-        ReduceArgs ra = reduce_args(part, sp.splits, M * c.d_out, static_cast<int>(M), static_cast<int>(c.d_out),
-                                    c.d_out, 1.0f, Y, c.d_out);
-        return reduce(ra, c.num_sms, c.stream) == cudaSuccess ? 0 : -2;
+        return 0;
     }
+    int rc = lora_down(c, A, r, s, X, M, T2, T_saved, part);
+    if (rc) return rc;
     if (!map_bf16(&m.a, X, c.d_in, M, c.d_in, 128) || !map_codes(&m.b, c.codes, c.d_out, c.d_in, 32, 256) ||
         !map_bf16(&m.ae, T2, 2 * r64, M, 2 * r64, 128) || !map_bf16(&m.be, B, r, c.d_out, r, 256))
         return -1;
@@ -349,7 +399,8 @@ int64_t bwd_workspace_bytes(int64_t M, int64_t d_out, int64_t d_in, int r, int n
     part = std::max<int64_t>(part, int64_t(split_v(M, d_out, num_sms).splits) * M * r64);
     part = std::max<int64_t>(part, int64_t(split_tokens(d_out, r64, M, num_sms).splits) * d_out * 2 * r64);
     part = std::max<int64_t>(part, int64_t(split_tokens(d_in, r64, M, num_sms).splits) * d_in * 2 * r64);
-    if (M <= kSmallM) part = std::max<int64_t>(part, int64_t(split_small(d_in, d_out, num_sms).splits) * M * d_in);
+    if (M <= kSmallM)
+        part = std::max<int64_t>(part, int64_t(split_small(d_in, d_out, num_sms).splits) * ceil_div(d_in, 128) * 128 * 16);
     return 2 * align256(M * r64 * 4) + align256(part * 4);
 }
 
@@ -360,9 +411,14 @@ int layer_bwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, fl
     uint16_t* V2 = reinterpret_cast<uint16_t*>(ws);
     uint16_t* T2 = reinterpret_cast<uint16_t*>(ws + align256(M * r64 * 4));
     float* part = reinterpret_cast<float*>(ws + 2 * align256(M * r64 * 4));
+    const bool few = M <= kSmallM;
 
     // ---- V = s dY B, held as hi | lo: D[m, j] = sum_n dY[m, n] B[n, j]
-    if (dX != nullptr || dA != nullptr) {
+    if (few && (dX != nullptr || dA != nullptr)) {
+        if (note(launch_few_v(dY, B, static_cast<int>(M), static_cast<int>(c.d_out), r, r64, s, V2, c.stream)) !=
+            cudaSuccess)
+            return -2;
+    } else if (dX != nullptr || dA != nullptr) {
         const int bn = bn_for(r64);
         Maps m;
         if (!map_bf16(&m.a, dY, c.d_out, M, c.d_out, 128) || !map_bf16(&m.b, B, r, c.d_out, r, 64)) return -1;
@@ -394,8 +450,9 @@ int layer_bwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, fl
         g.k_main = ceil_div(c.d_out, 64);
         g.k_ext = 2 * kx;
         g.alpha = 1.0f;
-        if (M <= kSmallM) {
-            // swapped: D[k, m] = sum_n W_hat[n, k] dY[m, n] + sum_j A[j, k] V[m, j]
+        if (few) {
+            // swapped: D[k, m] = sum_n W_hat[n, k] dY[m, n] + sum_j A[j, k] V[m, j],
+            // a programmatic dependent of the V kernel just launched
             if (!map_codes(&m.a, c.codes, c.d_out, c.d_in, 64, 64) || !map_bf16(&m.b, dY, c.d_out, M, c.d_out, 16) ||
                 !map_bf16(&m.ae, A, c.d_in, r, c.d_in, 64) || !map_bf16(&m.be, V2, 2 * r64, M, 2 * r64, 16))
                 return -1;
@@ -405,16 +462,14 @@ int layer_bwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, fl
             g.rows = static_cast<int>(c.d_in);
             g.cols = static_cast<int>(M);
             g.k_per_split = sp.k_per_split;
+            g.out = dX;
+            g.ldo = c.d_in;
             g.part = part;
-            g.ldp = c.d_in;
-            g.part_slice = M * c.d_in;
+            g.pdl = 1;
             dim3 grid(tiles, 1, sp.splits);
-            if (launch<16, SRC_DEC_MN, SRC_TMA_K, 1, 0, EPI_F32_PART_T>("nf4_gemm_dx_few", m.a, m.b, m.ae, m.be, g, grid, c.stream) !=
-                cudaSuccess)
+            if (launch<16, SRC_DEC_MN, SRC_TMA_K, 1, 0, EPI_CLUSTER_BF16_T, kFewLoad, kFewDec, kFewTeams>(
+                    "nf4_gemm_dx_few", m.a, m.b, m.ae, m.be, g, grid, c.stream, sp.splits) != cudaSuccess)
                 return -2;
-            ReduceArgs ra = reduce_args(part, sp.splits, M * c.d_in, static_cast<int>(M), static_cast<int>(c.d_in),
-                                        c.d_in, 1.0f, dX, c.d_in);
-            if (reduce(ra, c.num_sms, c.stream) != cudaSuccess) return -2;
         } else {
             if (!map_bf16(&m.a, dY, c.d_out, M, c.d_out, 128) || !map_codes(&m.b, c.codes, c.d_out, c.d_in, 128, 64) ||
                 !map_bf16(&m.ae, V2, 2 * r64, M, 2 * r64, 128) || !map_bf16(&m.be, A, c.d_in, r, c.d_in, 64))
@@ -442,6 +497,10 @@ int layer_bwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, fl
             cfg.blockDim = dim3(256);
             cfg.stream = c.stream;
             if (note(cudaLaunchKernelEx(&cfg, k_split_from_f32, T_saved, M, r, r64, T2)) != cudaSuccess) return -2;
+        } else if (few) {
+            if (note(launch_few_down(X, A, static_cast<int>(M), static_cast<int>(c.d_in), r, r64, s, T2, nullptr,
+                                     c.stream)) != cudaSuccess)
+                return -2;
         } else {
             int rc = lora_down(c, A, r, s, X, M, T2, nullptr, part);
             if (rc) return rc;

@@ -12,7 +12,7 @@
 
 #include <mutex>
 
-#include "../../include/nf4lora.h"
+#include "nf4lora.h"
 #include "kernels.h"
 
 namespace nf4lora {

@@ -8,7 +8,7 @@
 #include <string>
 #include <vector>
 
-#include "../../include/nf4lora.h"
+#include "nf4lora.h"
 #include "trace.h"
 
 namespace nf4lora {
