@@ -3,7 +3,8 @@
 //   D[rows, cols] (fp32, TMEM) = sum_k A[rows, k] * B[cols, k]
 //                              + sum_j A_ext[rows, j] * B_ext[cols, j]
 //
-// One CTA computes a 128 x BN tile (MMA M = 128, N = BN) over a range of
+// One CTA computes a (128 MSUB) x BN tile -- MSUB accumulators of 128 x BN
+// (MMA M = 128, N = BN) that share every B tile -- over a range of
 // 64-wide k-steps ("split"), followed -- in split 0 only -- by the extension
 // k-steps that carry the rank-r LoRA product, so that X W_hat^T + T B^T (or
 // dY W_hat + V A) lands in ONE accumulator without a second pass over the
@@ -85,18 +86,21 @@ struct OpTraits {
     static constexpr bool kMN = (SRC == SRC_TMA_MN || SRC == SRC_DEC_MN);
 };
 
-template <int BN, int ASRC, int BSRC, int AE_MN, int BE_MN, int EPI, int LSTAGES = 0, int DSTAGES = 0, int TEAMS = 1>
+template <int BN, int ASRC, int BSRC, int AE_MN, int BE_MN, int EPI, int LSTAGES = 0, int DSTAGES = 0, int TEAMS = 1,
+          int MSUB = 1>
 struct GemmConfig {
-    static constexpr int kBM = 128;
+    static constexpr int kBM = 128;                           // rows of one MMA / accumulator
+    static constexpr int kMSub = MSUB;                        // accumulators (128-row sub-tiles) per CTA
+    static constexpr int kRows = kBM * MSUB;                  // rows of D per CTA
     static constexpr int kBK = 64;
     static constexpr bool kDecA = OpTraits<ASRC>::kDecoded;
     static constexpr bool kDecB = OpTraits<BSRC>::kDecoded;
     static_assert(!(kDecA && kDecB), "at most one decoded operand");
     static constexpr bool kHasDec = kDecA || kDecB;
     static constexpr int kTeams = kHasDec ? TEAMS : 1;
-    static constexpr int kABytes = kBM * kBK * 2;             // 16 KB
+    static constexpr int kABytes = kRows * kBK * 2;           // 16 KB per sub-tile
     static constexpr int kBBytes = BN * kBK * 2;
-    static constexpr int kDecMN = kDecA ? kBM : (kDecB ? BN : 0);  // decoded tile's M/N width
+    static constexpr int kDecMN = kDecA ? kRows : (kDecB ? BN : 0);  // decoded tile's M/N width
     static constexpr int kCBytes = kDecMN * 32;               // packed codes per k-step
     // load slot: [A tile or A codes | B tile or B codes]; decode slot: the decoded tile
     static constexpr int kLoadA = kDecA ? kCBytes : kABytes;
@@ -121,7 +125,9 @@ struct GemmConfig {
     static constexpr int kDecWarps = kTeamWarps * kTeams;
     static constexpr int kWorkWarps = kDecWarps > 4 ? kDecWarps : 4;
     static constexpr int kThreads = 64 + 32 * kWorkWarps;
-    static constexpr int kTmemCols = BN < 32 ? 32 : BN;
+    static constexpr int kTmemCols = (BN < 32 ? 32 : BN) * MSUB;
+    static_assert(kTmemCols <= 512, "accumulators exceed tensor memory");
+    static_assert(MSUB == 1 || (ASRC == SRC_TMA_K && !AE_MN && EPI == EPI_BF16), "two sub-tiles: K-major A, bf16 out");
     static constexpr int kSmemBytes = kLS * kLoadSlot + (kHasDec ? kDS * kDecSlot : 0) + 1024;
     // CTAs per SM the configuration is built for (registers are capped to fit)
     static constexpr int kMinBlocks = kSmemBytes <= 110 * 1024 ? 2 : 1;
@@ -159,6 +165,46 @@ __device__ __forceinline__ void decode_unit(const uint8_t* src, float s, uint8_t
     }
 }
 
+// The same decode with the codebook held in registers: the 16 scaled levels
+// bf16(level_j * s) are formed once per unit and split into byte planes
+// (P: low bytes, H: high bytes, four entries per register); each group of
+// four codes is then looked up with byte permutes, entries 0-7 and 8-15
+// separately and merged on bit 3 of the code.  No shared-memory reads, so the
+// shared-memory port stays free for TMA, the decoded stores and the MMAs.
+__device__ __forceinline__ void decode_unit_reg(const uint8_t* src, float s, uint8_t* dst_row, int swz) {
+    uint32_t P[4], H[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t t0 = pack_bf16x2(__fmul_rn(nf4_level(4 * i), s), __fmul_rn(nf4_level(4 * i + 1), s));
+        const uint32_t t1 = pack_bf16x2(__fmul_rn(nf4_level(4 * i + 2), s), __fmul_rn(nf4_level(4 * i + 3), s));
+        P[i] = __byte_perm(t0, t1, 0x6420);
+        H[i] = __byte_perm(t0, t1, 0x7531);
+    }
+    const uint4 c0 = *reinterpret_cast<const uint4*>(src);
+    const uint4 c1 = *reinterpret_cast<const uint4*>(src + 16);
+    const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        uint32_t o[4];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            // nibbles of xs, low first: e1 e0 e3 e2 (byte b = e_2b << 4 | e_2b+1)
+            const uint32_t xs = words[j] >> (16 * h);
+            const uint32_t sel = xs & 0x7777u;                          // index within 0-7 / 8-15
+            const uint32_t pick = ((xs >> 1) & 0x4444u) | 0x3210u;      // byte i from the 8-15 half if bit 3
+            const uint32_t lo = __byte_perm(__byte_perm(P[0], P[1], sel), __byte_perm(P[2], P[3], sel), pick);
+            const uint32_t hi = __byte_perm(__byte_perm(H[0], H[1], sel), __byte_perm(H[2], H[3], sel), pick);
+            o[2 * h] = __byte_perm(lo, hi, 0x4051);      // (e0, e1): lo.b1 hi.b1 lo.b0 hi.b0
+            o[2 * h + 1] = __byte_perm(lo, hi, 0x6273);  // (e2, e3): lo.b3 hi.b3 lo.b2 hi.b2
+        }
+        *reinterpret_cast<uint4*>(dst_row + ((j ^ swz) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
+// Codebook used by the engine's decode warps: registers (true) or a 16-word
+// shared-memory table (false).
+constexpr bool kRegisterCodebook = true;
+
 __device__ __forceinline__ void zero_row(uint8_t* dst_row) {
 #pragma unroll
     for (int j = 0; j < 8; ++j) *reinterpret_cast<uint4*>(dst_row + (j << 4)) = make_uint4(0, 0, 0, 0);
@@ -184,13 +230,14 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
     }
 }
 
-template <int BN, int ASRC, int BSRC, int AE_MN, int BE_MN, int EPI, int LSTAGES = 0, int DSTAGES = 0, int TEAMS = 1>
-__global__ void __launch_bounds__(GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI, LSTAGES, DSTAGES, TEAMS>::kThreads,
-                                  GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI, LSTAGES, DSTAGES, TEAMS>::kMinBlocks)
+template <int BN, int ASRC, int BSRC, int AE_MN, int BE_MN, int EPI, int LSTAGES = 0, int DSTAGES = 0, int TEAMS = 1,
+          int MSUB = 1>
+__global__ void __launch_bounds__(GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI, LSTAGES, DSTAGES, TEAMS, MSUB>::kThreads,
+                                  GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI, LSTAGES, DSTAGES, TEAMS, MSUB>::kMinBlocks)
     k_gemm(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
            const __grid_constant__ CUtensorMap map_ae, const __grid_constant__ CUtensorMap map_be,
            const GemmArgs args) {
-    using C = GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI, LSTAGES, DSTAGES, TEAMS>;
+    using C = GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI, LSTAGES, DSTAGES, TEAMS, MSUB>;
     constexpr int LS = C::kLS;
     constexpr int DS = C::kDS;
     constexpr int kEpiThreads = C::kWorkWarps * 32;
@@ -211,7 +258,7 @@ __global__ void __launch_bounds__(GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI, 
     auto b_buf = [&](int it) { return C::kDecB ? dec_slot(it) : load_slot(it) + C::kLoadA; };
     auto codes_buf = [&](int it) { return load_slot(it) + (C::kDecA ? 0 : C::kLoadA); };
 
-    const int r0 = blockIdx.x * C::kBM;
+    const int r0 = blockIdx.x * C::kRows;
     const int c0 = blockIdx.y * BN;
     const int z = blockIdx.z;
     int kb_begin, kb_end;
@@ -285,7 +332,9 @@ __global__ void __launch_bounds__(GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI, 
                     mbar_arrive_expect_tx(bar, C::kTxMain);
                     // operand A
                     if constexpr (ASRC == SRC_TMA_K) {
-                        tma_load_2d(a_buf(it), &map_a, bar, kb * 64, r0);
+#pragma unroll
+                        for (int ms = 0; ms < MSUB; ++ms)
+                            tma_load_2d(a_buf(it) + ms * (C::kBM * 128), &map_a, bar, kb * 64, r0 + ms * C::kBM);
                     } else if constexpr (ASRC == SRC_TMA_MN) {
                         tma_load_2d(a_buf(it), &map_a, bar, r0, kb * 64);
                         tma_load_2d(a_buf(it) + 8192, &map_a, bar, r0 + 64, kb * 64);
@@ -321,7 +370,9 @@ __global__ void __launch_bounds__(GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI, 
                         tma_load_2d(a_buf(it), &map_ae, bar, r0, ja * 64);
                         tma_load_2d(a_buf(it) + 8192, &map_ae, bar, r0 + 64, ja * 64);
                     } else {
-                        tma_load_2d(a_buf(it), &map_ae, bar, ja * 64, r0);
+#pragma unroll
+                        for (int ms = 0; ms < MSUB; ++ms)
+                            tma_load_2d(a_buf(it) + ms * (C::kBM * 128), &map_ae, bar, ja * 64, r0 + ms * C::kBM);
                     }
                     if constexpr (BE_MN) {
 #pragma unroll
@@ -362,8 +413,11 @@ __global__ void __launch_bounds__(GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI, 
                 const uint32_t idesc = is_main ? C::kIdescMain : C::kIdescExt;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                    mma_bf16_ss(tmem_d, tile_desc(a_base, a_mn, kk), tile_desc(b_base, b_mn, kk), idesc,
-                                (it > 0 || kk > 0) ? 1u : 0u);
+                    const uint64_t bdesc = tile_desc(b_base, b_mn, kk);
+#pragma unroll
+                    for (int ms = 0; ms < MSUB; ++ms)   // sub-tile ms: rows 128 ms.., columns ms BN..
+                        mma_bf16_ss(tmem_d + ms * (C::kTmemCols / MSUB), tile_desc(a_base + ms * C::kBM * 128, a_mn, kk),
+                                    bdesc, idesc, (it > 0 || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(&bar_empty[it % LS]);
                 if (C::kHasDec) mma_commit(&bar_dempty[it % DS]);
@@ -435,8 +489,9 @@ __global__ void __launch_bounds__(GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI, 
                             break;
                         }
                         uint8_t* dst = dec_slot(it) + dst_off;
-                        if (valid) decode_unit(codes_buf(it) + dt * 32, sc, dst, swz, s_lut);
-                        else zero_row(dst);
+                        if (!valid) zero_row(dst);
+                        else if constexpr (kRegisterCodebook) decode_unit_reg(codes_buf(it) + dt * 32, sc, dst, swz);
+                        else decode_unit(codes_buf(it) + dt * 32, sc, dst, swz, s_lut);
                         fence_proxy_async_smem();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&bar_dfull[it % DS]);
@@ -456,11 +511,12 @@ __global__ void __launch_bounds__(GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI, 
         const bool ok = mbar_wait(&bar_accum, 0, abort_flag);
         tc_fence_after();
         if constexpr (EPI != EPI_CLUSTER_BF16_T) if (ok && !*abort_flag) {
-            const int row = r0 + q * 32 + lane;
+          for (int ms = 0; ms < MSUB; ++ms) {
+            const int row = r0 + ms * C::kBM + q * 32 + lane;
             const bool row_ok = row < args.rows;
             for (int cc = cbeg; cc < cbeg + cw; cc += 32) {
                 uint32_t v[32];
-                tmem_ld_32x32b_x32(tmem_d + (static_cast<uint32_t>(q * 32) << 16) + cc, v);
+                tmem_ld_32x32b_x32(tmem_d + (static_cast<uint32_t>(q * 32) << 16) + ms * (C::kTmemCols / MSUB) + cc, v);
                 tmem_ld_wait();
                 const int col = c0 + cc;
                 if constexpr (EPI == EPI_BF16) {
@@ -510,6 +566,7 @@ __global__ void __launch_bounds__(GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI, 
                     }
                 }
             }
+          }
         }
         if constexpr (EPI == EPI_CLUSTER_BF16_T) {
             // this CTA's fp32 partial tile [128 rows][BN], row-major, into the

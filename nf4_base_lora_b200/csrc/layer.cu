@@ -85,12 +85,13 @@ static bool map_codes(CUtensorMap* m, const uint8_t* codes, int64_t d_out, int64
 }
 
 // ------------------------------------------------------------------ launch
-template <int BN, int ASRC, int BSRC, int AE, int BE, int EPI, int LSTAGES = 0, int DSTAGES = 0, int TEAMS = 1>
+template <int BN, int ASRC, int BSRC, int AE, int BE, int EPI, int LSTAGES = 0, int DSTAGES = 0, int TEAMS = 1,
+          int MSUB = 1>
 static cudaError_t launch(const char* name, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& ae,
                           const CUtensorMap& be, const GemmArgs& args, dim3 grid, cudaStream_t st,
                           int cluster_z = 1) {
-    using C = GemmConfig<BN, ASRC, BSRC, AE, BE, EPI, LSTAGES, DSTAGES, TEAMS>;
-    auto kern = k_gemm<BN, ASRC, BSRC, AE, BE, EPI, LSTAGES, DSTAGES, TEAMS>;
+    using C = GemmConfig<BN, ASRC, BSRC, AE, BE, EPI, LSTAGES, DSTAGES, TEAMS, MSUB>;
+    auto kern = k_gemm<BN, ASRC, BSRC, AE, BE, EPI, LSTAGES, DSTAGES, TEAMS, MSUB>;
     // the shared-memory opt-in is per device; set it once (also keeps it out of
     // stream captures)
     static bool configured[64] = {};
@@ -251,6 +252,18 @@ static inline int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + 
 static int bn_for(int cols) { return cols <= 64 ? 64 : (cols <= 128 ? 128 : 256); }
 
 static constexpr int kSmallM = 16;
+
+// Many-token fused GEMMs: 256-row CTA tiles (two accumulators sharing each
+// decoded weight tile, which halves the decode work per MMA) once there are
+// enough of them to cover every SM, else 128-row tiles.
+static bool wide_tiles(int64_t M, int64_t cols, int sms) {
+    return int64_t(ceil_div(M, 256)) * ceil_div(cols, 256) >= sms;
+}
+// 256 x 256 tiles: 4 load slots of 40 KB + 2 decoded tiles of 32 KB, one per
+// decode team, teams on alternate k-steps
+static constexpr int kWideLoad = 4;
+static constexpr int kWideDec = 2;
+static constexpr int kWideTeams = 2;
 // few-token kernels: 6 load slots of 6 KB + 4 decoded tiles of 16 KB = 100 KB
 // (two CTAs per SM), two decode teams on alternate k-steps
 static constexpr int kFewLoad = 6;
@@ -387,10 +400,16 @@ int layer_fwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, fl
     g.k_per_split = g.k_main;
     g.out = Y;
     g.ldo = c.d_out;
-    dim3 grid(ceil_div(M, 128), ceil_div(c.d_out, 256), 1);
-    if (launch<256, SRC_TMA_K, SRC_DEC_K, 0, 0, EPI_BF16>("nf4_gemm_fwd", m.a, m.b, m.ae, m.be, g, grid, c.stream) != cudaSuccess)
-        return -2;
-    return 0;
+    cudaError_t e;
+    if (wide_tiles(M, c.d_out, c.num_sms)) {
+        dim3 grid(ceil_div(M, 256), ceil_div(c.d_out, 256), 1);
+        e = launch<256, SRC_TMA_K, SRC_DEC_K, 0, 0, EPI_BF16, kWideLoad, kWideDec, kWideTeams, 2>(
+            "nf4_gemm_fwd", m.a, m.b, m.ae, m.be, g, grid, c.stream);
+    } else {
+        dim3 grid(ceil_div(M, 128), ceil_div(c.d_out, 256), 1);
+        e = launch<256, SRC_TMA_K, SRC_DEC_K, 0, 0, EPI_BF16>("nf4_gemm_fwd", m.a, m.b, m.ae, m.be, g, grid, c.stream);
+    }
+    return e == cudaSuccess ? 0 : -2;
 }
 
 int64_t bwd_workspace_bytes(int64_t M, int64_t d_out, int64_t d_in, int r, int num_sms) {
@@ -480,10 +499,17 @@ int layer_bwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, fl
             g.k_per_split = g.k_main;
             g.out = dX;
             g.ldo = c.d_in;
-            dim3 grid(ceil_div(M, 128), ceil_div(c.d_in, 256), 1);
-            if (launch<256, SRC_TMA_K, SRC_DEC_MN, 0, 1, EPI_BF16>("nf4_gemm_dx", m.a, m.b, m.ae, m.be, g, grid, c.stream) !=
-                cudaSuccess)
-                return -2;
+            cudaError_t e;
+            if (wide_tiles(M, c.d_in, c.num_sms)) {
+                dim3 grid(ceil_div(M, 256), ceil_div(c.d_in, 256), 1);
+                e = launch<256, SRC_TMA_K, SRC_DEC_MN, 0, 1, EPI_BF16, kWideLoad, kWideDec, kWideTeams, 2>(
+                    "nf4_gemm_dx", m.a, m.b, m.ae, m.be, g, grid, c.stream);
+            } else {
+                dim3 grid(ceil_div(M, 128), ceil_div(c.d_in, 256), 1);
+                e = launch<256, SRC_TMA_K, SRC_DEC_MN, 0, 1, EPI_BF16>("nf4_gemm_dx", m.a, m.b, m.ae, m.be, g, grid,
+                                                                       c.stream);
+            }
+            if (e != cudaSuccess) return -2;
         }
     }
 

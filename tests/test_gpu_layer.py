@@ -39,6 +39,7 @@ CASES = [
     (512, 768, 300, 128),
     (1024, 512, 256, 24),
     (384, 1024, 200, 192),
+    (4736, 4800, 2000, 16),   # enough tiles for the 256-row CTA tile; ragged tokens
 ]
 
 
