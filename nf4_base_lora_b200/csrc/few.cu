@@ -1,15 +1,17 @@
-// Rank-r intermediates for few tokens (M <= 16), on CUDA cores:
-//   T = s X A^T   (forward, "第 04 篇：QLoRA 原理" §6.3, the LoRA down product)
-//   V = s dY B    (backward, §2.4, the input-gradient branch through B)
-// Each writes the bf16 hi | lo pair the tensor-core extension steps consume
-// (and T in fp32 for reuse by the backward) and lets the fused dequant-GEMM
-// that follows launch at once (programmatic dependent launch): the GEMM
-// streams and decodes the weight while these run, and waits for them only
+// Rank-r intermediates for few tokens (M <= 16):
+//   T = s X A^T   (forward, "第 04 篇：QLoRA 原理" §6.3, the LoRA down product;
+//                  warp-level tensor instructions)
+//   V = s dY B    (backward, §2.4, the input-gradient branch through B; CUDA cores)
+// Each writes the bf16 hi | lo pair the fused products' extension steps
+// consume (and T in fp32 for reuse by the backward) and lets the fused
+// dequant-GEMM that follows launch early (programmatic dependent launch): the
+// GEMM streams and decodes the weight while these run, and waits for them only
 // before its extension steps.  The contraction is split over a thread-block
 // cluster and summed through distributed shared memory in rank order.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
 
 #include "common.cuh"
@@ -36,74 +38,145 @@ __device__ __forceinline__ void store_split(uint16_t* dst_hi, uint16_t* dst_lo, 
     *dst_lo = *reinterpret_cast<const uint16_t*>(&lo);
 }
 
-constexpr int kDownSplit = 4;   // cluster size along K for T
-constexpr int kVSplit = 8;      // cluster size along d_out for V
+// T on the warp-level tensor instructions: D[t, j] = sum_k X[t, k] A[j, k]
+// (m16n8k16: A operand = X, 16 tokens x 16 k; B operand = 8 rows of A).
+// One cluster of up to 8 CTAs splits K.  A CTA copies its slice of X and of A
+// (64 rows of A at a time, up to 512 k) into shared memory with asynchronous
+// copies issued all at once -- one memory latency per slice -- and releases
+// the dependent launch as soon as the first slice is requested, so that these
+// loads queue ahead of the dependent kernel's.  Warp w then owns the 8-column
+// tile (w & 7) of the 64 and every other 16-wide chunk of the slice (w >> 3).
+// Partials are added in a fixed order: the two chunk halves in shared memory,
+// then the cluster ranks by rank 0 reading the others' shared memory.
+constexpr int kDownThreads = 512;
+constexpr int kDownMaxSplit = 8;
+constexpr int kDownBatch = 512;                 // k per staged slice
+constexpr int kDownStride = kDownBatch + 8;     // row stride (elements): 1040 bytes, conflict-free fragments
+constexpr int kDownSmem = (kMaxFewTokens + 64) * kDownStride * 2 + 2 * kMaxFewTokens * 256 * 4;
 
-// T: cluster (1, kDownSplit) per column j of T (j < r64; j >= r written as
-// zeros).  CTA rank ks covers k in [ks K / kDownSplit, (ks + 1) K / kDownSplit);
-// thread t accumulates k = k0 + 8t, k0 + 8t + 1024, ... for every token.
-__global__ void __launch_bounds__(128) k_few_down(const uint16_t* __restrict__ X, const uint16_t* __restrict__ A,
-                                                  int M, int K, int r, int r64, float s,
-                                                  uint16_t* __restrict__ T2, float* __restrict__ T_saved) {
-    allow_dependents();
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int j = blockIdx.x;
-    const int ks = static_cast<int>(cluster_ctarank());
-    const int k_len = (K / 8 + kDownSplit - 1) / kDownSplit * 8;
-    const int k0 = ks * k_len;
-    const int k1 = min(K, k0 + k_len);
-    float acc[kMaxFewTokens];
+__device__ __forceinline__ void mma_m16n8k16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                             uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(kDownThreads, 1) k_few_down(const uint16_t* __restrict__ X,
+                                                               const uint16_t* __restrict__ A, int M, int K, int r,
+                                                               int r64, float s, uint16_t* __restrict__ T2,
+                                                               float* __restrict__ T_saved) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    uint16_t* sX = reinterpret_cast<uint16_t*>(smem);              // [16][kDownStride]
+    uint16_t* sA = sX + kMaxFewTokens * kDownStride;               // [64][kDownStride]
+    float* s_half = reinterpret_cast<float*>(sA + 64 * kDownStride);  // [16][256]
+    float* s_p = s_half + kMaxFewTokens * 256;                       // [16][256]
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, q = lane & 3;
+    const int nt = warp & 7, kg = warp >> 3;
+    const int splits = static_cast<int>(gridDim.z);
+    const int rank = static_cast<int>(cluster_ctarank());
+    const int bpr = K / 64;
+    const int per = bpr / splits, extra = bpr % splits;
+    const int k_begin = 64 * (rank * per + (rank < extra ? rank : extra));
+    const int k_end = k_begin + 64 * (per + (rank < extra ? 1 : 0));
+    const int npass = r64 / 64;  // 64 columns of T per pass (<= 4)
+    float acc[4][4];
 #pragma unroll
-    for (int m = 0; m < kMaxFewTokens; ++m) acc[m] = 0.0f;
-    if (j < r) {
-        for (int k = k0 + tid * 8; k < k1; k += 128 * 8) {
-            const uint4 a = __ldg(reinterpret_cast<const uint4*>(A + static_cast<int64_t>(j) * K + k));
-            const float af[8] = {bf16_lo(a.x), bf16_hi(a.x), bf16_lo(a.y), bf16_hi(a.y),
-                                 bf16_lo(a.z), bf16_hi(a.z), bf16_lo(a.w), bf16_hi(a.w)};
+    for (int p = 0; p < 4; ++p)
 #pragma unroll
-            for (int m = 0; m < kMaxFewTokens; ++m) {
-                if (m < M) {
-                    const uint4 x = __ldg(reinterpret_cast<const uint4*>(X + static_cast<int64_t>(m) * K + k));
-                    float d = acc[m];
-                    d = fmaf(bf16_lo(x.x), af[0], d);
-                    d = fmaf(bf16_hi(x.x), af[1], d);
-                    d = fmaf(bf16_lo(x.y), af[2], d);
-                    d = fmaf(bf16_hi(x.y), af[3], d);
-                    d = fmaf(bf16_lo(x.z), af[4], d);
-                    d = fmaf(bf16_hi(x.z), af[5], d);
-                    d = fmaf(bf16_lo(x.w), af[6], d);
-                    d = fmaf(bf16_hi(x.w), af[7], d);
-                    acc[m] = d;
+        for (int i = 0; i < 4; ++i) acc[p][i] = 0.0f;
+
+    bool released = false;
+    for (int k0 = k_begin; k0 < k_end; k0 += kDownBatch) {
+        const int kn = min(kDownBatch, k_end - k0);  // a multiple of 64
+        const int pieces = kn / 8;                   // 16-byte pieces per row
+        for (int p = 0; p < npass; ++p) {
+            __syncthreads();  // the previous slice is no longer read
+            // rows of X (first pass of the slice only) and rows 64 p .. 64 p + 63 of A
+            const int xrows = p == 0 ? kMaxFewTokens : 0;
+            for (int i = tid; i < (xrows + 64) * pieces; i += kDownThreads) {
+                const int row = i / pieces, pc = i - row * pieces;
+                if (row < xrows) {
+                    uint16_t* dst = sX + row * kDownStride + pc * 8;
+                    if (row < M) cp_async16(dst, X + static_cast<int64_t>(row) * K + k0 + pc * 8);
+                    else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+                } else {
+                    const int j = 64 * p + (row - xrows);
+                    uint16_t* dst = sA + (row - xrows) * kDownStride + pc * 8;
+                    if (j < r) cp_async16(dst, A + static_cast<int64_t>(j) * K + k0 + pc * 8);
+                    else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
                 }
+            }
+            if (!released) {
+                allow_dependents();
+                released = true;
+            }
+            cp_async_wait_all();
+            __syncthreads();
+            const uint16_t* xr0 = sX + g * kDownStride + 2 * q;
+            const uint16_t* xr8 = xr0 + 8 * kDownStride;
+            const uint16_t* ar = sA + (8 * nt + g) * kDownStride + 2 * q;
+            for (int c = kg; c < kn / 16; c += 2) {
+                const int k = 16 * c;
+                mma_m16n8k16(acc[p], *reinterpret_cast<const uint32_t*>(xr0 + k), *reinterpret_cast<const uint32_t*>(xr8 + k),
+                             *reinterpret_cast<const uint32_t*>(xr0 + k + 8), *reinterpret_cast<const uint32_t*>(xr8 + k + 8),
+                             *reinterpret_cast<const uint32_t*>(ar + k), *reinterpret_cast<const uint32_t*>(ar + k + 8));
             }
         }
     }
-    __shared__ float red[4][kMaxFewTokens];
-    __shared__ float part[kMaxFewTokens];
-#pragma unroll
-    for (int m = 0; m < kMaxFewTokens; ++m) {
-        float v = acc[m];
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0) red[warp][m] = v;
-    }
+    if (!released) allow_dependents();
+
+    // acc[p]: tokens g (0, 1) and g + 8 (2, 3) at columns 64 p + 8 nt + 2q + {0, 1}
+    auto put = [&](float* dst, int p) {
+        const int j = 64 * p + 8 * nt + 2 * q;
+        dst[g * 256 + j] = acc[p][0];
+        dst[g * 256 + j + 1] = acc[p][1];
+        dst[(g + 8) * 256 + j] = acc[p][2];
+        dst[(g + 8) * 256 + j + 1] = acc[p][3];
+    };
+    if (kg == 1)
+        for (int p = 0; p < npass; ++p) put(s_half, p);
     __syncthreads();
-    if (tid < kMaxFewTokens) part[tid] = ((red[0][tid] + red[1][tid]) + red[2][tid]) + red[3][tid];
-    cluster_sync_all();
-    if (ks == 0 && tid < M) {
-        float t[kDownSplit];
+    if (kg == 0)
+        for (int p = 0; p < npass; ++p) {
+            const int j = 64 * p + 8 * nt + 2 * q;
+            acc[p][0] += s_half[g * 256 + j];
+            acc[p][1] += s_half[g * 256 + j + 1];
+            acc[p][2] += s_half[(g + 8) * 256 + j];
+            acc[p][3] += s_half[(g + 8) * 256 + j + 1];
+            put(s_p, p);
+        }
+    cluster_sync_all();  // every rank's partial is complete and visible
+    if (rank == 0) {
+        for (int i = tid; i < M * r64; i += kDownThreads) {
+            const int t = i / r64, j = i - t * r64;
+            float part[kDownMaxSplit];
+            const uint32_t addr = smem_u32(&s_p[t * 256 + j]);
 #pragma unroll
-        for (int rk = 0; rk < kDownSplit; ++rk) t[rk] = ld_cluster_f32(cluster_map(smem_u32(&part[tid]), rk));
-        float v = 0.0f;
+            for (int rk = 1; rk < kDownMaxSplit; ++rk)
+                if (rk < splits) part[rk] = ld_cluster_f32(cluster_map(addr, rk));
+            float v = s_p[t * 256 + j];
 #pragma unroll
-        for (int rk = 0; rk < kDownSplit; ++rk) v += t[rk];
-        v *= s;
-        uint16_t* row = T2 + static_cast<int64_t>(tid) * 2 * r64;
-        store_split(row + j, row + r64 + j, v);
-        if (T_saved != nullptr && j < r) T_saved[static_cast<int64_t>(tid) * r + j] = v;
+            for (int rk = 1; rk < kDownMaxSplit; ++rk)
+                if (rk < splits) v += part[rk];
+            v *= s;
+            uint16_t* row = T2 + static_cast<int64_t>(t) * 2 * r64;
+            store_split(row + j, row + r64 + j, j < r ? v : 0.0f);
+            if (T_saved != nullptr && j < r) T_saved[static_cast<int64_t>(t) * r + j] = v;
+        }
     }
-    cluster_sync_all();
+    cluster_sync_all();  // rank 0 has read the other ranks' shared memory
 }
+
+constexpr int kVSplit = 8;      // cluster size along d_out for V
 
 // V: cluster (1, kVSplit) per 4 columns of V; CTA rank ns covers rows
 // n in [ns N / kVSplit, (ns + 1) N / kVSplit); thread t takes rows t, t + 128, ...
@@ -187,8 +260,29 @@ static cudaLaunchConfig_t cluster_config(dim3 grid, int split, cudaLaunchAttribu
 
 cudaError_t launch_few_down(const uint16_t* X, const uint16_t* A, int M, int K, int r, int r64, float s,
                             uint16_t* T2, float* T_saved, cudaStream_t stream) {
+    if (M < 1 || M > kMaxFewTokens || K % 64 != 0 || r64 > 256) return cudaErrorInvalidValue;
+    static bool configured[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64 || !configured[dev]) {
+        e = cudaFuncSetAttribute(k_few_down, cudaFuncAttributeMaxDynamicSharedMemorySize, kDownSmem);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) configured[dev] = true;
+    }
+    const int splits = std::max(1, std::min(kDownMaxSplit, K / 64));
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(1, 1, splits);
+    cfg.blockDim = dim3(kDownThreads);
+    cfg.dynamicSmemBytes = kDownSmem;
+    cfg.stream = stream;
     cudaLaunchAttribute attr[1];
-    cudaLaunchConfig_t cfg = cluster_config(dim3(r64, kDownSplit), kDownSplit, attr, stream);
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = splits;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     TraceScope trace("few_lora_down", stream);
     return cudaLaunchKernelEx(&cfg, k_few_down, X, A, M, K, r, r64, s, T2, T_saved);
 }

@@ -1,0 +1,382 @@
+// Few-token (M <= 16) fused NF4-LoRA forward, weights decoded straight into
+// the operand registers of warp-level tensor instructions (mma.sync
+// m16n8k16, bf16 in, fp32 accumulate):
+//
+//   Y[t, n] = sum_k X[t, k] W_hat[n, k] + sum_j T2[t, j] [B | B][n, j]
+//
+// ("第 04 篇：QLoRA 原理" §6.1-§6.3; T2 holds the rank-r intermediate
+// s X A^T as a bf16 hi | lo pair.)
+//
+// With at most 16 tokens the layer is a streamed matrix-vector product: per
+// weight the GPU reads 4.127 bits and decodes them, and the 16 dot products
+// are a small tail.  One thread (TMA) streams the CTA's packed codes into
+// shared memory; each thread then decodes its slice with the 16-level table,
+// restores bf16(level[code] * s_b) in registers and hands the pairs to the
+// tensor instruction as its A fragment (16 weight rows x 16 k; the activations
+// are the B fragment, 16 k x 8 tokens).  A decoded weight never goes back to
+// memory.
+//
+// The contraction index inside each 16-wide MMA chunk is permuted so that a
+// thread's operand comes from whole 64-blocks (one scale per row and block):
+// thread (g, q) of a warp covers weight rows g and g + 8 of a 16-row group
+// and block q of four consecutive blocks; chunk c takes k = 4c .. 4c+3 of each
+// thread's block.  The activation fragment uses the same permutation, which
+// leaves the sums unchanged.
+//
+// Split-K: the CTAs that share one output tile form a thread-block cluster
+// along grid.z.  Inside a CTA the two warps of a row group add their fp32
+// partials through shared memory; every CTA of rank > 0 then pushes its
+// partial tile into a slot of rank 0 (distributed shared memory) and arrives
+// on an mbarrier there; rank 0 adds the slots in rank order, adds the rank-r
+// extension once the kernel that produced T2 has finished (programmatic
+// dependent launch), and writes bf16.  The summation order is fixed, so the
+// result is the same on every run.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "nf4_levels.cuh"
+#include "trace.h"
+
+namespace nf4lora {
+
+namespace {
+
+constexpr int kThreads = 512;      // 16 warps
+constexpr int kTile = 128;         // weight rows per CTA
+constexpr int kTok = 16;           // token rows of the MMA
+constexpr int kMaxSplit = 8;       // CTAs per cluster (portable cluster size)
+constexpr int kPartFloats = kTile * kTok;  // one CTA's partial tile, fp32
+
+// contraction blocks staged per segment (four block quads: two per warp of a
+// row group, 16 x 16 x 64 activations = 4 16-byte pieces per thread)
+constexpr int kFwdSegBlocks = 16;
+
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void wait_prerequisites() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Even split of `total` units over `parts`; part p gets [begin, end).
+__device__ __forceinline__ void split_range(int total, int parts, int p, int& begin, int& end) {
+    const int per = total / parts, extra = total % parts;
+    begin = p * per + (p < extra ? p : extra);
+    end = begin + per + (p < extra ? 1 : 0);
+}
+
+// Tensor-instruction roles: A = 16 weight rows x 16 k (decoded), B = 16 k x 8
+// tokens (activations), D = 16 rows x 8 tokens; two MMAs cover 16 tokens.
+// A warp works on 16 weight rows (thread (g, q): rows g and g + 8) and four
+// consecutive 64-blocks at a time (thread q streams block q whole: 32 bytes
+// per row, one scale per row); MMA chunk c of the quad takes k = 4c .. 4c+3
+// of each thread's block.
+//
+// Activations are staged as [token][block][64 + 4] with a token stride of
+// 16 x 68 + 16 elements (2208 bytes): the 8-byte fragment loads of a
+// half-warp (4 tokens x 4 blocks) then fall in 16 different bank pairs.
+constexpr int kFwdBlockStride = 68;
+constexpr int kFwdTokStride = kFwdSegBlocks * kFwdBlockStride + 16;
+constexpr int kFwdQuadBytes = kTile * 128;  // codes of 4 blocks x 128 rows
+constexpr int kFwdMaxSplit = kMaxSplit;      // partial-tile slots of rank 0: kFwdMaxSplit - 1
+constexpr int kFwdSmemV2 =
+    1024 + 4 * kFwdQuadBytes + (kFwdMaxSplit - 1) * kPartFloats * 4 + 8 * 8 * 32 * 4 + kTok * kFwdTokStride * 2;
+
+// Bytes 2h and 2h + 1 of word w (4 weights) to two bf16 pairs, with the level
+// table read by byte offset (code * 4) straight from the shifted word.
+__device__ __forceinline__ void decode_quarter(uint32_t w, int h, float s, const uint8_t* lut_bytes, uint32_t& p0,
+                                               uint32_t& p1) {
+    const uint32_t hi_off = (w >> 2) & 0x3C3C3C3Cu;  // 4 * high nibble of each byte
+    const uint32_t lo_off = (w << 2) & 0x3C3C3C3Cu;  // 4 * low nibble of each byte
+    const uint32_t sel0 = 0x4440u + 2 * h, sel1 = 0x4441u + 2 * h;  // byte 2h / 2h + 1, zero-extended
+    const float e0 = *reinterpret_cast<const float*>(lut_bytes + __byte_perm(hi_off, 0u, sel0));
+    const float o0 = *reinterpret_cast<const float*>(lut_bytes + __byte_perm(lo_off, 0u, sel0));
+    const float e1 = *reinterpret_cast<const float*>(lut_bytes + __byte_perm(hi_off, 0u, sel1));
+    const float o1 = *reinterpret_cast<const float*>(lut_bytes + __byte_perm(lo_off, 0u, sel1));
+    p0 = pack_bf16x2(__fmul_rn(e0, s), __fmul_rn(o0, s));
+    p1 = pack_bf16x2(__fmul_rn(e1, s), __fmul_rn(o1, s));
+}
+
+// Registers capped at 96 (48K of the SM's 64K) so that the CTAs of the kernel
+// producing T2, which this one overlaps, keep room on the same SM.
+__global__ void __maxnreg__(96) k_few_fwd(const __grid_constant__ CUtensorMap map_codes, const FewArgs a) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    __shared__ __align__(16) float s_lut[16];
+    __shared__ uint64_t bar_part, bar_q[4];
+    __shared__ int s_abort;
+    // [codes: 4 quads x 128 rows x 128 B, 128-byte swizzle][partial slots][warp reduction][activations]
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t* s_codes = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    float* s_part = reinterpret_cast<float*>(s_codes + 4 * kFwdQuadBytes);  // [kFwdMaxSplit - 1][8 values][256 threads]
+    float* s_red = s_part + (kFwdMaxSplit - 1) * kPartFloats;               // [8 row groups][8 values][32 lanes]
+    uint16_t* sX = reinterpret_cast<uint16_t*>(s_red + 8 * 8 * 32);          // [16][kFwdTokStride]
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, q = lane & 3;
+    const int rgp = warp & 7;  // 16-row group of the CTA's 128 rows
+    const int qs = warp >> 3;  // which block quads: qs, qs + 2
+    const int splits = static_cast<int>(gridDim.z);
+    const int rank = static_cast<int>(cluster_ctarank());
+    const int M = a.M, N = a.N, K = a.K;
+    const int bpr = K / 64;
+    int kb0, kb1;
+    split_range(bpr, splits, rank, kb0, kb1);
+    const int row0 = blockIdx.x * kTile;
+    // thread 0: barriers, then the first segment's codes in flight at once
+    auto issue_codes = [&](int seg0, int nquads) {
+        for (int j = 0; j < nquads; ++j) {
+            mbar_arrive_expect_tx(&bar_q[j], kFwdQuadBytes);
+            tma_load_2d(s_codes + j * kFwdQuadBytes, &map_codes, &bar_q[j], 32 * (seg0 + 4 * j), row0);
+        }
+    };
+    const int nq_first = (min(kb1 - kb0, kFwdSegBlocks) + 3) / 4;
+    if (tid == 0) {
+        mbar_init(&bar_part, splits > 1 ? (splits - 1) * 256 : 1);
+        for (int j = 0; j < 4; ++j) mbar_init(&bar_q[j], 1);
+        s_abort = 0;
+        fence_barrier_init();
+        if (kb0 < kb1) {
+            tma_prefetch_desc(&map_codes);
+            issue_codes(kb0, nq_first);
+        }
+    }
+    if (tid < 16) s_lut[tid] = nf4_level(tid);
+
+    const int lr = 16 * rgp + g;  // local row of nA (nB = nA + 8 is local row lr + 8)
+    const int nA = row0 + lr, nB = nA + 8;
+    const bool okA = nA < N, okB = nB < N;
+    const bool two_halves = M > 8;
+
+    float acc0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, acc1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    __syncthreads();
+    cluster_arrive_relaxed();  // barriers initialised (made visible by the init fence)
+    const float mu = __ldg(a.scale_mean);
+    const uint8_t* lut_bytes = reinterpret_cast<const uint8_t*>(s_lut);
+    volatile int* abort_flag = &s_abort;
+
+    int seg_i = 0, issued_seg = 0, issued_nq = kb0 < kb1 ? nq_first : 0;
+    for (int seg0 = kb0; seg0 < kb1; seg0 += kFwdSegBlocks, ++seg_i) {
+        const int nb = min(kb1 - seg0, kFwdSegBlocks);
+        const int nquads = (nb + 3) / 4;
+        const int nbp = 4 * nquads;  // staged blocks; nb .. nbp - 1 and tokens >= M are zeros
+        if (seg_i > 0) {
+            __syncthreads();  // the previous segment's codes and activations are no longer read
+            if (*abort_flag) break;  // the same value in every thread: no wait can set it here
+            if (tid == 0) issue_codes(seg0, nquads);
+            issued_seg = seg_i;
+            issued_nq = nquads;
+        }
+        // activations of the segment (L2 hits) and this thread's block scales
+        uint4 xv[4];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const int i = tid + p * kThreads;
+            const int t = i / (nbp * 8), pc = i - t * (nbp * 8);
+            xv[p] = make_uint4(0, 0, 0, 0);
+            if (t < M && pc < nb * 8)
+                xv[p] = __ldg(reinterpret_cast<const uint4*>(a.act + static_cast<int64_t>(t) * K + seg0 * 64) + pc);
+        }
+        int qA[2], qB[2];
+        float aA[2], aB[2];
+        bool inA[2], inB[2];  // the item's block exists (else its weights are zero)
+#pragma unroll
+        for (int it = 0; it < 2; ++it) {
+            const int j = qs + 2 * it, lb = 4 * j + q, blk = seg0 + lb;
+            const bool in = j < nquads && lb < nb;
+            const int64_t biA = static_cast<int64_t>(nA) * bpr + blk, biB = static_cast<int64_t>(nB) * bpr + blk;
+            inA[it] = in && okA;
+            inB[it] = in && okB;
+            qA[it] = inA[it] ? static_cast<int>(__ldg(a.qscale + biA)) : 0;
+            qB[it] = inB[it] ? static_cast<int>(__ldg(a.qscale + biB)) : 0;
+            aA[it] = inA[it] ? __ldg(a.scale2 + (biA >> 8)) : 0.0f;
+            aB[it] = inB[it] ? __ldg(a.scale2 + (biB >> 8)) : 0.0f;
+        }
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const int i = tid + p * kThreads;
+            const int t = i / (nbp * 8), pc = i - t * (nbp * 8);
+            if (t < kTok) {
+                const int lb = pc >> 3, kk = (pc & 7) * 8;
+                uint2* dst = reinterpret_cast<uint2*>(sX + t * kFwdTokStride + lb * kFwdBlockStride + kk);
+                dst[0] = make_uint2(xv[p].x, xv[p].y);
+                dst[1] = make_uint2(xv[p].z, xv[p].w);
+            }
+        }
+        __syncthreads();
+        // decode and multiply as each quad's codes land
+#pragma unroll
+        for (int it = 0; it < 2; ++it) {
+            const int j = qs + 2 * it;
+            if (j >= nquads) break;
+            if (!mbar_wait(&bar_q[j], seg_i & 1, abort_flag)) break;
+            const int lb = 4 * j + q;
+            const float sA = inA[it] ? nf4_block_scale(static_cast<int8_t>(qA[it]), aA[it], mu) : 0.0f;
+            const float sB = inB[it] ? nf4_block_scale(static_cast<int8_t>(qB[it]), aB[it], mu) : 0.0f;
+            // rows lr and lr + 8 of the quad, 16-byte chunks 2q and 2q + 1 (block q), swizzled by row
+            const uint8_t* qbase = s_codes + j * kFwdQuadBytes;
+            const uint4 cA0 = *reinterpret_cast<const uint4*>(qbase + lr * 128 + (((2 * q) ^ g) << 4));
+            const uint4 cA1 = *reinterpret_cast<const uint4*>(qbase + lr * 128 + (((2 * q + 1) ^ g) << 4));
+            const uint4 cB0 = *reinterpret_cast<const uint4*>(qbase + (lr + 8) * 128 + (((2 * q) ^ g) << 4));
+            const uint4 cB1 = *reinterpret_cast<const uint4*>(qbase + (lr + 8) * 128 + (((2 * q + 1) ^ g) << 4));
+            const uint16_t* x0 = sX + g * kFwdTokStride + lb * kFwdBlockStride;
+            const uint16_t* x8 = x0 + 8 * kFwdTokStride;
+            const uint32_t wA[8] = {cA0.x, cA0.y, cA0.z, cA0.w, cA1.x, cA1.y, cA1.z, cA1.w};
+            const uint32_t wB[8] = {cB0.x, cB0.y, cB0.z, cB0.w, cB1.x, cB1.y, cB1.z, cB1.w};
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                uint32_t a0, a1, a2, a3;  // rows g (a0, a2) and g + 8 (a1, a3), k = 4c + {0,1} / {2,3}
+                decode_quarter(wA[c >> 1], c & 1, sA, lut_bytes, a0, a2);
+                decode_quarter(wB[c >> 1], c & 1, sB, lut_bytes, a1, a3);
+                const uint2 xb = *reinterpret_cast<const uint2*>(x0 + 4 * c);
+                mma_16816(acc0, a0, a1, a2, a3, xb.x, xb.y);
+                if (two_halves) {
+                    const uint2 xc = *reinterpret_cast<const uint2*>(x8 + 4 * c);
+                    mma_16816(acc1, a0, a1, a2, a3, xc.x, xc.y);
+                }
+            }
+        }
+    }
+    if (tid == 0 && *abort_flag) {
+        // let the copies still in flight land before the CTA can exit
+        for (int j = 0; j < issued_nq; ++j) mbar_drain(&bar_q[j], issued_seg & 1);
+    }
+
+    // rank-r extension on rank 0: [B | B] rows of this CTA against T2, once the
+    // kernel producing T2 has finished (programmatic dependent launch)
+    if (rank == 0 && a.ext_act != nullptr) {
+        if (a.pdl) wait_prerequisites();
+        const int nchunks = 2 * a.r64 / 16;
+        const uint16_t* bA = a.ext_w + static_cast<int64_t>(nA) * a.r;
+        const uint16_t* bB = a.ext_w + static_cast<int64_t>(nB) * a.r;
+        for (int ch = qs; ch < nchunks; ch += 2) {
+            const int j0 = ch * 16;
+            const int jj = (j0 % a.r64) + 2 * q;  // column of B (same in both halves of T2)
+            const bool lo_ok = jj < a.r, hi_ok = jj + 8 < a.r;
+            const uint32_t a0 = (okA && lo_ok) ? __ldg(reinterpret_cast<const uint32_t*>(bA + jj)) : 0u;
+            const uint32_t a1 = (okB && lo_ok) ? __ldg(reinterpret_cast<const uint32_t*>(bB + jj)) : 0u;
+            const uint32_t a2 = (okA && hi_ok) ? __ldg(reinterpret_cast<const uint32_t*>(bA + jj + 8)) : 0u;
+            const uint32_t a3 = (okB && hi_ok) ? __ldg(reinterpret_cast<const uint32_t*>(bB + jj + 8)) : 0u;
+            const uint16_t* t0 = a.ext_act + static_cast<int64_t>(g) * 2 * a.r64 + j0 + 2 * q;
+            const uint32_t b0 = g < M ? __ldg(reinterpret_cast<const uint32_t*>(t0)) : 0u;
+            const uint32_t b1 = g < M ? __ldg(reinterpret_cast<const uint32_t*>(t0 + 8)) : 0u;
+            mma_16816(acc0, a0, a1, a2, a3, b0, b1);
+            if (two_halves) {
+                const uint16_t* t8 = t0 + 8 * 2 * a.r64;
+                const uint32_t c0 = g + 8 < M ? __ldg(reinterpret_cast<const uint32_t*>(t8)) : 0u;
+                const uint32_t c1 = g + 8 < M ? __ldg(reinterpret_cast<const uint32_t*>(t8 + 8)) : 0u;
+                mma_16816(acc1, a0, a1, a2, a3, c0, c1);
+            }
+        }
+    }
+
+    // the two warps of a row group add up (qs 1 into qs 0), then ranks > 0
+    // push to rank 0, which adds the ranks in order
+    float v[8] = {acc0[0], acc0[1], acc0[2], acc0[3], acc1[0], acc1[1], acc1[2], acc1[3]};
+    if (qs == 1) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) s_red[(rgp * 8 + i) * 32 + lane] = v[i];
+    }
+    __syncthreads();
+    bool waited = false;
+    if (qs == 0) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] += s_red[(rgp * 8 + i) * 32 + lane];
+        const int slot = tid;  // 0..255
+        if (rank != 0) {
+            cluster_wait_acquire();
+            waited = true;
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                st_cluster_f32(cluster_map(smem_u32(s_part + ((rank - 1) * 8 + i) * 256 + slot), 0), v[i]);
+            mbar_arrive_remote(cluster_map(smem_u32(&bar_part), 0));
+        } else {
+            const bool got = splits == 1 || mbar_wait_cluster(&bar_part, 0, &s_abort);
+            if (got) {
+                for (int rk = 1; rk < splits; ++rk)
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) v[i] += s_part[((rk - 1) * 8 + i) * 256 + slot];
+                // v[0..3]: tokens 2q, 2q+1 of rows nA (0, 1) and nB (2, 3); v[4..7]: tokens + 8
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int t0 = 2 * q + 8 * h;
+                    auto put = [&](int t, int n, float x) {
+                        if (t < M && n < N) {
+                            const __nv_bfloat16 b = __float2bfloat16_rn(x);
+                            a.out[static_cast<int64_t>(t) * N + n] = *reinterpret_cast<const uint16_t*>(&b);
+                        }
+                    };
+                    put(t0, nA, v[4 * h + 0]);
+                    put(t0 + 1, nA, v[4 * h + 1]);
+                    put(t0, nB, v[4 * h + 2]);
+                    put(t0 + 1, nB, v[4 * h + 3]);
+                }
+            }
+        }
+    }
+    // no CTA leaves while another may still write into its shared memory
+    if (!waited) cluster_wait_acquire();
+    cluster_arrive_release();
+    cluster_wait_acquire();
+}
+
+// `configured`: per-device flags of this kernel (both kernels have the same
+// type, so the flags cannot live in the template)
+template <typename Kern, typename... Params>
+cudaError_t launch_cluster(Kern kern, bool (&configured)[64], int smem, const char* name, const FewArgs& a, int tiles,
+                           int splits, cudaStream_t stream, const Params&... params) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64 || !configured[dev]) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) configured[dev] = true;
+    }
+    if (splits < 1 || splits > kMaxSplit) return cudaErrorInvalidValue;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(tiles, 1, splits);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    int n = 0;
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = 1;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = splits;
+    ++n;
+    if (a.pdl) {
+        attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[n].val.programmaticStreamSerializationAllowed = 1;
+        ++n;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    TraceScope trace(name, stream);
+    return cudaLaunchKernelEx(&cfg, kern, params..., a);
+}
+
+}  // namespace
+
+int few_max_split(bool forward) { return forward ? kFwdMaxSplit : kMaxSplit; }
+
+cudaError_t launch_few_fwd(const CUtensorMap& map_codes, const FewArgs& a, int splits, cudaStream_t stream) {
+    if (a.M < 1 || a.M > kTok || a.K % 64 != 0 || a.N % 8 != 0 || splits > a.K / 64 || splits > kFwdMaxSplit)
+        return cudaErrorInvalidValue;
+    static bool configured[64] = {};
+    return launch_cluster(k_few_fwd, configured, kFwdSmemV2, "nf4_gemm_fwd_few", a, (a.N + kTile - 1) / kTile, splits,
+                          stream, map_codes);
+}
+
+}  // namespace nf4lora

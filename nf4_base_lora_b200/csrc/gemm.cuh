@@ -38,9 +38,10 @@
 // decoded tiles occupy shared memory.  Every wait is bounded (common.cuh).
 //
 // Split-K over few tokens: the splits of one tile form a thread-block cluster
-// along grid.z; each CTA writes its fp32 partial tile to the workspace, one
-// cluster barrier makes them visible, and CTA rank 0 adds them in split order
-// -- no atomics or counters, the same sum on every run.
+// along grid.z; every CTA of rank > 0 pushes its fp32 partial tile straight
+// into a shared-memory slot of rank 0 (distributed shared memory) and arrives
+// on an mbarrier there; rank 0 adds the slots in rank order -- no atomics, no
+// round trip through global memory, the same sum on every run.
 #pragma once
 
 #include <cstdint>
@@ -109,7 +110,10 @@ struct GemmConfig {
     static constexpr int kDecSlot = kDecA ? kABytes : (kDecB ? kBBytes : 0);
     static constexpr int kDS = kHasDec ? (DSTAGES > 0 ? DSTAGES : 3 * kTeams) : 1;
     static_assert(kDS % kTeams == 0, "each team must own whole decode slots");
-    static constexpr int kBudget = 225 * 1024 - (kHasDec ? kDS * kDecSlot : 0);
+    // cluster split-K: rank 0 receives the partial tiles of ranks 1 .. kPushMax - 1
+    static constexpr int kPushMax = 4;
+    static constexpr int kPartBytes = EPI == EPI_CLUSTER_BF16_T ? (kPushMax - 1) * kBM * BN * 4 : 0;
+    static constexpr int kBudget = 225 * 1024 - (kHasDec ? kDS * kDecSlot : 0) - kPartBytes;
     static constexpr int kLSRaw = kBudget / kLoadSlot;
     static constexpr int kLSCap = kHasDec ? 2 * kDS : 8;
     static constexpr int kLSAuto = kLSRaw < kLSCap ? kLSRaw : kLSCap;
@@ -125,10 +129,17 @@ struct GemmConfig {
     static constexpr int kDecWarps = kTeamWarps * kTeams;
     static constexpr int kWorkWarps = kDecWarps > 4 ? kDecWarps : 4;
     static constexpr int kThreads = 64 + 32 * kWorkWarps;
-    static constexpr int kTmemCols = (BN < 32 ? 32 : BN) * MSUB;
-    static_assert(kTmemCols <= 512, "accumulators exceed tensor memory");
+    // Few-token tiles (N = 16) rotate their MMAs over kAcc independent
+    // accumulators: one small MMA finishes long before the next one on the same
+    // accumulator could start, so a single chain would leave the tensor core
+    // idle.  The epilogue adds the accumulators in a fixed order.
+    static constexpr int kAcc = EPI == EPI_CLUSTER_BF16_T ? 8 : 1;
+    static_assert(kAcc == 1 || MSUB == 1, "rotating accumulators or two sub-tiles, not both");
+    static constexpr int kAccCols = BN * MSUB * kAcc;
+    static constexpr int kTmemCols = kAccCols <= 32 ? 32 : kAccCols <= 64 ? 64 : kAccCols <= 128 ? 128 : kAccCols <= 256 ? 256 : 512;
+    static_assert(kAccCols <= 512, "accumulators exceed tensor memory");
     static_assert(MSUB == 1 || (ASRC == SRC_TMA_K && !AE_MN && EPI == EPI_BF16), "two sub-tiles: K-major A, bf16 out");
-    static constexpr int kSmemBytes = kLS * kLoadSlot + (kHasDec ? kDS * kDecSlot : 0) + 1024;
+    static constexpr int kSmemBytes = kLS * kLoadSlot + (kHasDec ? kDS * kDecSlot : 0) + kPartBytes + 1024;
     // CTAs per SM the configuration is built for (registers are capped to fit)
     static constexpr int kMinBlocks = kSmemBytes <= 110 * 1024 ? 2 : 1;
     static constexpr int kTxMain = kLoadA + kLoadB;            // bytes TMA lands per main k-step
@@ -221,15 +232,6 @@ __device__ __forceinline__ void named_barrier_sync(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
-// Bounded wait that ignores the abort flag: used only to drain copies that
-// are still in flight when a CTA gives up.
-__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
-    const uint64_t t0 = global_timer_ns();
-    while (!mbar_try_wait(bar, parity)) {
-        if (global_timer_ns() - t0 > kWaitLimitNs / 20) break;
-    }
-}
-
 template <int BN, int ASRC, int BSRC, int AE_MN, int BE_MN, int EPI, int LSTAGES = 0, int DSTAGES = 0, int TEAMS = 1,
           int MSUB = 1>
 __global__ void __launch_bounds__(GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI, LSTAGES, DSTAGES, TEAMS, MSUB>::kThreads,
@@ -242,12 +244,13 @@ __global__ void __launch_bounds__(GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI, 
     constexpr int DS = C::kDS;
     constexpr int kEpiThreads = C::kWorkWarps * 32;
     extern __shared__ uint8_t smem_raw[];
-    __shared__ uint64_t bar_full[LS], bar_empty[LS], bar_dfull[DS], bar_dempty[DS], bar_accum;
+    __shared__ uint64_t bar_full[LS], bar_empty[LS], bar_dfull[DS], bar_dempty[DS], bar_accum, bar_part;
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
     __shared__ float s_lut[16];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    bool cluster_waited = false;  // this thread has passed the cluster barrier's first phase
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base_u32 = (raw + 1023u) & ~1023u;
     uint8_t* base = smem_raw + (base_u32 - raw);
@@ -297,6 +300,8 @@ __global__ void __launch_bounds__(GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI, 
             mbar_init(&bar_dempty[i], 1);
         }
         mbar_init(&bar_accum, 1);
+        // rank 0 of a split-K cluster: one arrival per row from every other rank
+        mbar_init(&bar_part, gridDim.z > 1 ? (gridDim.z - 1) * C::kBM : 1);
         s_abort = 0;
         fence_barrier_init();
     }
@@ -311,6 +316,9 @@ __global__ void __launch_bounds__(GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI, 
         asm volatile("barrier.sync 3, %0;" ::"r"(C::kThreads) : "memory");
     }
     volatile int* abort_flag = &s_abort;
+    // split-K cluster: announce that this CTA's barriers are initialised; the
+    // matching wait comes before the first access to another CTA's memory
+    if constexpr (EPI == EPI_CLUSTER_BF16_T) cluster_arrive_release();
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -415,9 +423,13 @@ __global__ void __launch_bounds__(GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI, 
                 for (int kk = 0; kk < 4; ++kk) {
                     const uint64_t bdesc = tile_desc(b_base, b_mn, kk);
 #pragma unroll
-                    for (int ms = 0; ms < MSUB; ++ms)   // sub-tile ms: rows 128 ms.., columns ms BN..
-                        mma_bf16_ss(tmem_d + ms * (C::kTmemCols / MSUB), tile_desc(a_base + ms * C::kBM * 128, a_mn, kk),
-                                    bdesc, idesc, (it > 0 || kk > 0) ? 1u : 0u);
+                    for (int ms = 0; ms < MSUB; ++ms) {  // sub-tile ms: rows 128 ms.., columns ms BN..
+                        const int mi = it * 4 + kk;      // MMA index; with kAcc > 1 it picks the accumulator
+                        const uint32_t dcol = C::kAcc > 1 ? (mi % C::kAcc) * BN : ms * BN;
+                        const uint32_t accumulate = C::kAcc > 1 ? (mi >= C::kAcc ? 1u : 0u) : (mi > 0 ? 1u : 0u);
+                        mma_bf16_ss(tmem_d + dcol, tile_desc(a_base + ms * C::kBM * 128, a_mn, kk), bdesc, idesc,
+                                    accumulate);
+                    }
                 }
                 mma_commit(&bar_empty[it % LS]);
                 if (C::kHasDec) mma_commit(&bar_dempty[it % DS]);
@@ -516,7 +528,7 @@ __global__ void __launch_bounds__(GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI, 
             const bool row_ok = row < args.rows;
             for (int cc = cbeg; cc < cbeg + cw; cc += 32) {
                 uint32_t v[32];
-                tmem_ld_32x32b_x32(tmem_d + (static_cast<uint32_t>(q * 32) << 16) + ms * (C::kTmemCols / MSUB) + cc, v);
+                tmem_ld_32x32b_x32(tmem_d + (static_cast<uint32_t>(q * 32) << 16) + ms * BN + cc, v);
                 tmem_ld_wait();
                 const int col = c0 + cc;
                 if constexpr (EPI == EPI_BF16) {
@@ -569,65 +581,83 @@ __global__ void __launch_bounds__(GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI, 
           }
         }
         if constexpr (EPI == EPI_CLUSTER_BF16_T) {
-            // this CTA's fp32 partial tile [128 rows][BN], row-major, into the
-            // partial buffer (one slot per (tile, split); coalesced 16 B stores)
-            if (ew < 4 && ok && !*abort_flag) {
-                uint32_t v[32];
-                tmem_ld_32x32b_x32(tmem_d + (static_cast<uint32_t>(q * 32) << 16), v);
-                tmem_ld_wait();
-                float* dst = args.part + (static_cast<int64_t>(blockIdx.x) * gridDim.z + z) * (C::kBM * BN) +
-                             (q * 32 + lane) * BN;
+            // ranks > 0 push their fp32 partial tile into slot rank - 1 of
+            // rank 0; rank 0 adds the slots to its own tile in rank order
+            if (ew < 4) {
+                const int rl = q * 32 + lane;  // row within the tile
+                const uint32_t rank = cluster_ctarank();
+                const int splits = static_cast<int>(gridDim.z);
+                float* s_part = reinterpret_cast<float*>(base + LS * C::kLoadSlot + DS * C::kDecSlot);
+                const bool have = ok && !*abort_flag;
+                // this CTA's partial: the used accumulators added in index order
+                float part[BN];
 #pragma unroll
-                for (int j = 0; j < BN; j += 4)
-                    __stcg(reinterpret_cast<float4*>(dst + j),
-                           make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]),
-                                       __uint_as_float(v[j + 3])));
+                for (int j = 0; j < BN; ++j) part[j] = 0.0f;
+                if (have) {
+                    const int used = n_iter * 4 < C::kAcc ? n_iter * 4 : C::kAcc;
+                    static_assert(32 % BN == 0 && (C::kAcc * BN) % 32 == 0, "accumulator loads of 32 columns");
+#pragma unroll
+                    for (int c = 0; c < C::kAcc * BN; c += 32) {
+                        uint32_t v[32];
+                        tmem_ld_32x32b_x32(tmem_d + (static_cast<uint32_t>(q * 32) << 16) + c, v);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if ((c + j) / BN < used) part[(c + j) % BN] += __uint_as_float(v[j]);
+                    }
+                }
+                if (rank != 0) {
+                    cluster_wait_acquire();  // rank 0's barrier is initialised
+                    cluster_waited = true;
+                    if (have) {
+                        const uint32_t dst = cluster_map(smem_u32(s_part + ((rank - 1) * C::kBM + rl) * BN), 0);
+#pragma unroll
+                        for (int j = 0; j < BN; j += 4)
+                            st_cluster_f4(dst + 4 * j, part[j], part[j + 1], part[j + 2], part[j + 3]);
+                    }
+                    // arrive even without data, so that rank 0 never waits out
+                    // the time limit for a rank that gave up (the device status
+                    // word already reports it)
+                    mbar_arrive_remote(cluster_map(smem_u32(&bar_part), 0));
+                } else {
+                    const bool got = splits == 1 || mbar_wait_cluster(&bar_part, 0, abort_flag);
+                    if (have && got && !*abort_flag) {
+                        float acc[BN];
+#pragma unroll
+                        for (int j = 0; j < BN; ++j) acc[j] = part[j];
+                        for (int rk = 1; rk < splits; ++rk) {
+                            const float4* src = reinterpret_cast<const float4*>(s_part + ((rk - 1) * C::kBM + rl) * BN);
+#pragma unroll
+                            for (int j = 0; j < BN / 4; ++j) {
+                                const float4 t = src[j];
+                                acc[4 * j] += t.x;
+                                acc[4 * j + 1] += t.y;
+                                acc[4 * j + 2] += t.z;
+                                acc[4 * j + 3] += t.w;
+                            }
+                        }
+                        const int row = r0 + rl;
+                        if (row < args.rows) {
+#pragma unroll
+                            for (int j = 0; j < BN; ++j) {
+                                if (j < args.cols) {
+                                    const __nv_bfloat16 h = __float2bfloat16_rn(acc[j] * args.alpha);
+                                    args.out[static_cast<int64_t>(j) * args.ldo + row] =
+                                        *reinterpret_cast<const uint16_t*>(&h);
+                                }
+                            }
+                        }
+                    }
+                }
             }
         }
     }
 
     if constexpr (EPI == EPI_CLUSTER_BF16_T) {
-        // one cluster barrier (release / acquire at cluster scope) makes every
-        // split's partial visible to rank 0, which adds them in split order
-        cluster_sync_all();
-        const int ew = warp - 2;
-        if (cluster_ctarank() == 0 && ew >= 0 && ew < 4 && !*abort_flag) {
-            const int rr = threadIdx.x - 64;              // one row per thread
-            const int row = r0 + rr;
-            const int splits = static_cast<int>(gridDim.z);
-            const float* src = args.part + static_cast<int64_t>(blockIdx.x) * splits * (C::kBM * BN) + rr * BN;
-            float acc[BN];
-#pragma unroll
-            for (int j = 0; j < BN; ++j) acc[j] = 0.0f;
-            for (int z0 = 0; z0 < splits; z0 += 4) {
-                float4 t[4][BN / 4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u)
-                    if (z0 + u < splits)
-#pragma unroll
-                        for (int j = 0; j < BN / 4; ++j)
-                            t[u][j] = __ldcg(reinterpret_cast<const float4*>(src + (z0 + u) * (C::kBM * BN)) + j);
-#pragma unroll
-                for (int u = 0; u < 4; ++u)
-                    if (z0 + u < splits)
-#pragma unroll
-                        for (int j = 0; j < BN / 4; ++j) {
-                            acc[4 * j] += t[u][j].x;
-                            acc[4 * j + 1] += t[u][j].y;
-                            acc[4 * j + 2] += t[u][j].z;
-                            acc[4 * j + 3] += t[u][j].w;
-                        }
-            }
-            if (row < args.rows) {
-#pragma unroll
-                for (int j = 0; j < BN; ++j) {
-                    if (j < args.cols) {
-                        const __nv_bfloat16 h = __float2bfloat16_rn(acc[j] * args.alpha);
-                        args.out[static_cast<int64_t>(j) * args.ldo + row] = *reinterpret_cast<const uint16_t*>(&h);
-                    }
-                }
-            }
-        }
+        // no CTA leaves while another may still write into its shared memory
+        if (!cluster_waited) cluster_wait_acquire();
+        cluster_arrive_release();
+        cluster_wait_acquire();
     }
     tc_fence_before();
     __syncthreads();

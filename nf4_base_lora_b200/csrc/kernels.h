@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 namespace nf4lora {
@@ -20,5 +21,25 @@ cudaError_t launch_few_down(const uint16_t* X, const uint16_t* A, int M, int K, 
                             uint16_t* T2, float* T_saved, cudaStream_t stream);
 cudaError_t launch_few_v(const uint16_t* dY, const uint16_t* B, int M, int N, int r, int r64, float s,
                          uint16_t* V2, cudaStream_t stream);
+
+// Few-token (M <= 16) fused products on warp-level tensor instructions with
+// the weight decoded in registers (fewmma.cu).
+struct FewArgs {
+    const uint16_t* act;       // forward: X [M, K]; input grad: dY [M, N]
+    const uint8_t* codes;      // packed NF4 codes [N, K / 2]
+    const int8_t* qscale;      // [N K / 64]
+    const float* scale2;       // [ceil(N K / 64 / 256)]
+    const float* scale_mean;   // [1]
+    int M, N, K;               // tokens, d_out, d_in
+    const uint16_t* ext_act;   // T2 / V2 [M, 2 r64] (bf16 hi | lo)
+    const uint16_t* ext_w;     // forward: B [N, r]; input grad: A [r, K]
+    int r, r64;
+    uint16_t* out;             // forward: Y [M, N]; input grad: dX [M, K]
+    int pdl;                   // launched as a programmatic dependent of the ext_act producer
+};
+int few_max_split(bool forward);
+// map_codes: the packed codes as bytes [N, K / 2], box {128 bytes, 128 rows},
+// 128-byte swizzle
+cudaError_t launch_few_fwd(const CUtensorMap& map_codes, const FewArgs& a, int splits, cudaStream_t stream);
 
 }  // namespace nf4lora

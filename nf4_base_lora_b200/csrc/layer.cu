@@ -72,7 +72,7 @@ static bool map_bf16(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t o
 
 // Packed NF4 codes viewed as bytes [d_out, d_in / 2], box {box_inner bytes, box_outer rows}.
 static bool map_codes(CUtensorMap* m, const uint8_t* codes, int64_t d_out, int64_t d_in,
-                      uint32_t box_inner, uint32_t box_outer) {
+                      uint32_t box_inner, uint32_t box_outer, bool swizzle128 = false) {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(d_in / 2), static_cast<cuuint64_t>(d_out)};
@@ -80,7 +80,7 @@ static bool map_codes(CUtensorMap* m, const uint8_t* codes, int64_t d_out, int64
     cuuint32_t box[2] = {box_inner, box_outer};
     cuuint32_t estr[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -92,6 +92,9 @@ static cudaError_t launch(const char* name, const CUtensorMap& a, const CUtensor
                           int cluster_z = 1) {
     using C = GemmConfig<BN, ASRC, BSRC, AE, BE, EPI, LSTAGES, DSTAGES, TEAMS, MSUB>;
     auto kern = k_gemm<BN, ASRC, BSRC, AE, BE, EPI, LSTAGES, DSTAGES, TEAMS, MSUB>;
+    // rank 0 of a split-K cluster has partial-tile slots for kPushMax - 1 other ranks
+    if (EPI == EPI_CLUSTER_BF16_T && (static_cast<int>(grid.z) > C::kPushMax || cluster_z != static_cast<int>(grid.z)))
+        return note(cudaErrorInvalidValue);
     // the shared-memory opt-in is per device; set it once (also keeps it out of
     // stream captures)
     static bool configured[64] = {};
@@ -264,24 +267,39 @@ static bool wide_tiles(int64_t M, int64_t cols, int sms) {
 static constexpr int kWideLoad = 4;
 static constexpr int kWideDec = 2;
 static constexpr int kWideTeams = 2;
-// few-token kernels: 6 load slots of 6 KB + 4 decoded tiles of 16 KB = 100 KB
-// (two CTAs per SM), two decode teams on alternate k-steps
-static constexpr int kFewLoad = 6;
-static constexpr int kFewDec = 4;
-static constexpr int kFewTeams = 2;
+// Split of the contraction of the few-token kernels: the splits of one tile
+// form a cluster; as many (up to the cluster limit) as keep every tile's
+// cluster resident at once with one CTA per SM.
+static int few_splits(int tiles, int units, int sms, bool forward) {
+    return std::max(1, std::min({few_max_split(forward), sms / std::max(1, tiles), units}));
+}
 
-// Split-K of the few-token kernels: a power of two <= 8 (the portable cluster
-// size) so that the splits of a tile form one cluster, filling about two CTAs
-// per SM and keeping at least two k-steps per split.
-static Split few_split(int tiles, int k_steps, int sms) {
-    int s = 1;
-    while (s < 8 && tiles * (s * 2) <= 2 * sms && k_steps >= 2 * (s * 2)) s *= 2;
-    int kps = (k_steps + s - 1) / s;
-    while (s > 1 && (s - 1) * kps >= k_steps) {  // never leave a split empty
-        s /= 2;
-        kps = (k_steps + s - 1) / s;
-    }
-    return {s, kps};
+// few-token input gradient on the tcgen05 engine (one CTA per SM): 12 load
+// slots of 6 KB + 8 decoded tiles of 16 KB + partial-tile slots; four decode
+// teams, each on every fourth k-step; at most 4 splits (the slots of rank 0)
+static constexpr int kDxLoad = 12;
+static constexpr int kDxDec = 8;
+static constexpr int kDxTeams = 4;
+static constexpr int kDxMaxSplit = 4;
+
+static FewArgs few_args(const LayerCtx& c, const uint16_t* act, int M, const uint16_t* ext_act,
+                        const uint16_t* ext_w, int r, int r64, uint16_t* out) {
+    FewArgs a{};
+    a.act = act;
+    a.codes = c.codes;
+    a.qscale = c.qscale;
+    a.scale2 = c.scale2;
+    a.scale_mean = c.scale_mean;
+    a.M = M;
+    a.N = static_cast<int>(c.d_out);
+    a.K = static_cast<int>(c.d_in);
+    a.ext_act = ext_act;
+    a.ext_w = ext_w;
+    a.r = r;
+    a.r64 = r64;
+    a.out = out;
+    a.pdl = 1;
+    return a;
 }
 
 // The splits each split-K GEMM uses (the workspace query and the calls share them).
@@ -294,9 +312,6 @@ static Split split_v(int64_t M, int64_t d_out, int sms) {
 static Split split_tokens(int64_t rows, int r64, int64_t M, int sms) {
     const int tiles = ceil_div(rows, 128) * ceil_div(2 * r64, bn_for(2 * r64));
     return choose_split(tiles, ceil_div(M, 64), sms, 4);
-}
-static Split split_small(int64_t rows, int64_t k, int sms) {
-    return few_split(ceil_div(rows, 128), ceil_div(k, 64), sms);
 }
 
 // ------------------------------------------------------------------ layer ops
@@ -342,9 +357,7 @@ static int lora_down(const LayerCtx& c, const uint16_t* A, int r, float s, const
 
 int64_t fwd_workspace_bytes(int64_t M, int64_t d_out, int64_t d_in, int r, int num_sms) {
     const int r64 = round64(r);
-    int64_t part = int64_t(split_down(M, d_in, num_sms).splits) * M * r64;
-    if (M <= kSmallM)
-        part = std::max<int64_t>(part, int64_t(split_small(d_out, d_in, num_sms).splits) * ceil_div(d_out, 128) * 128 * 16);
+    const int64_t part = M <= kSmallM ? 0 : int64_t(split_down(M, d_in, num_sms).splits) * M * r64;
     return align256(M * r64 * 4) + align256(part * 4);
 }
 
@@ -364,30 +377,16 @@ int layer_fwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, fl
     g.k_ext = 2 * kx;
     g.alpha = 1.0f;
     if (M <= kSmallM) {
-        // T on CUDA cores, then the swapped fused GEMM as its programmatic
-        // dependent: D[n, m] = W_hat[n, :] . X[m, :] + B[n, :] . T[m, :],
-        // split-K over a cluster per 128-row tile, reduced in the cluster.
-        const int tiles = ceil_div(c.d_out, 128);
+        // T (hi | lo) first; the fused product as its programmatic dependent
+        // streams and decodes the weight meanwhile and waits for T only before
+        // the rank-r extension.
         if (note(launch_few_down(X, A, static_cast<int>(M), static_cast<int>(c.d_in), r, r64, s, T2, T_saved,
                                  c.stream)) != cudaSuccess)
             return -2;
-        if (!map_codes(&m.a, c.codes, c.d_out, c.d_in, 32, 128) || !map_bf16(&m.b, X, c.d_in, M, c.d_in, 16) ||
-            !map_bf16(&m.ae, B, r, c.d_out, r, 128) || !map_bf16(&m.be, T2, 2 * r64, M, 2 * r64, 16))
-            return -1;
-        const Split sp = split_small(c.d_out, c.d_in, c.num_sms);
-        g.ext_wrap_a = kx;
-        g.rows = static_cast<int>(c.d_out);
-        g.cols = static_cast<int>(M);
-        g.k_per_split = sp.k_per_split;
-        g.out = Y;
-        g.ldo = c.d_out;
-        g.part = part;
-        g.pdl = 1;
-        dim3 grid(tiles, 1, sp.splits);
-        if (launch<16, SRC_DEC_K, SRC_TMA_K, 0, 0, EPI_CLUSTER_BF16_T, kFewLoad, kFewDec, kFewTeams>(
-                "nf4_gemm_fwd_few", m.a, m.b, m.ae, m.be, g, grid, c.stream, sp.splits) != cudaSuccess)
-            return -2;
-        return 0;
+        const FewArgs fa = few_args(c, X, static_cast<int>(M), T2, B, r, r64, Y);
+        const int splits = few_splits(ceil_div(c.d_out, 128), static_cast<int>(c.d_in / 64), c.num_sms, true);
+        if (!map_codes(&m.a, c.codes, c.d_out, c.d_in, 128, 128, true)) return -1;
+        return note(launch_few_fwd(m.a, fa, splits, c.stream)) == cudaSuccess ? 0 : -2;
     }
     int rc = lora_down(c, A, r, s, X, M, T2, T_saved, part);
     if (rc) return rc;
@@ -418,8 +417,6 @@ int64_t bwd_workspace_bytes(int64_t M, int64_t d_out, int64_t d_in, int r, int n
     part = std::max<int64_t>(part, int64_t(split_v(M, d_out, num_sms).splits) * M * r64);
     part = std::max<int64_t>(part, int64_t(split_tokens(d_out, r64, M, num_sms).splits) * d_out * 2 * r64);
     part = std::max<int64_t>(part, int64_t(split_tokens(d_in, r64, M, num_sms).splits) * d_in * 2 * r64);
-    if (M <= kSmallM)
-        part = std::max<int64_t>(part, int64_t(split_small(d_in, d_out, num_sms).splits) * ceil_div(d_in, 128) * 128 * 16);
     return 2 * align256(M * r64 * 4) + align256(part * 4);
 }
 
@@ -470,24 +467,24 @@ int layer_bwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, fl
         g.k_ext = 2 * kx;
         g.alpha = 1.0f;
         if (few) {
-            // swapped: D[k, m] = sum_n W_hat[n, k] dY[m, n] + sum_j A[j, k] V[m, j],
-            // a programmatic dependent of the V kernel just launched
+            // swapped: D[k, m] = sum_n W_hat[n, k] dY[m, n] + sum_j A[j, k] V[m, j] on the
+            // tcgen05 engine (the decoded tile goes to shared memory in the MN-major
+            // layout the tensor core reads transposed), split-K over a cluster, a
+            // programmatic dependent of the V kernel just launched
             if (!map_codes(&m.a, c.codes, c.d_out, c.d_in, 64, 64) || !map_bf16(&m.b, dY, c.d_out, M, c.d_out, 16) ||
                 !map_bf16(&m.ae, A, c.d_in, r, c.d_in, 64) || !map_bf16(&m.be, V2, 2 * r64, M, 2 * r64, 16))
                 return -1;
             const int tiles = ceil_div(c.d_in, 128);
-            const Split sp = split_small(c.d_in, c.d_out, c.num_sms);
+            const int splits = std::max(1, std::min({kDxMaxSplit, c.num_sms / tiles, ceil_div(c.d_out, 64) / 2}));
             g.ext_wrap_a = kx;
             g.rows = static_cast<int>(c.d_in);
             g.cols = static_cast<int>(M);
-            g.k_per_split = sp.k_per_split;
             g.out = dX;
             g.ldo = c.d_in;
-            g.part = part;
             g.pdl = 1;
-            dim3 grid(tiles, 1, sp.splits);
-            if (launch<16, SRC_DEC_MN, SRC_TMA_K, 1, 0, EPI_CLUSTER_BF16_T, kFewLoad, kFewDec, kFewTeams>(
-                    "nf4_gemm_dx_few", m.a, m.b, m.ae, m.be, g, grid, c.stream, sp.splits) != cudaSuccess)
+            dim3 grid(tiles, 1, splits);
+            if (launch<16, SRC_DEC_MN, SRC_TMA_K, 1, 0, EPI_CLUSTER_BF16_T, kDxLoad, kDxDec, kDxTeams>(
+                    "nf4_gemm_dx_few", m.a, m.b, m.ae, m.be, g, grid, c.stream, splits) != cudaSuccess)
                 return -2;
         } else {
             if (!map_bf16(&m.a, dY, c.d_out, M, c.d_out, 128) || !map_codes(&m.b, c.codes, c.d_out, c.d_in, 128, 64) ||

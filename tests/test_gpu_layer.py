@@ -40,6 +40,7 @@ CASES = [
     (1024, 512, 256, 24),
     (384, 1024, 200, 192),
     (4736, 4800, 2000, 16),   # enough tiles for the 256-row CTA tile; ragged tokens
+    (9472, 1408, 5, 16),      # few tokens: two splits of 11 blocks (a ragged block quad)
 ]
 
 
