@@ -96,10 +96,15 @@ def load_peaks():
 
 
 def kernel_source_hash():
+    """Hash of every CUDA source of the library (a traffic figure is used only
+    while the kernels are the ones it was measured on)."""
     h = hashlib.sha256()
-    for name in ("gemm.cuh", "common.cuh", "nf4_levels.cuh", "layer.cu"):
-        with open(os.path.join(ROOT, "nf4_base_lora_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+    csrc = os.path.join(ROOT, "nf4_base_lora_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode())
+                h.update(f.read())
     return h.hexdigest()[:16]
 
 

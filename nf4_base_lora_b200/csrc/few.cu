@@ -40,19 +40,22 @@ __device__ __forceinline__ void store_split(uint16_t* dst_hi, uint16_t* dst_lo, 
 
 // T on the warp-level tensor instructions: D[t, j] = sum_k X[t, k] A[j, k]
 // (m16n8k16: A operand = X, 16 tokens x 16 k; B operand = 8 rows of A).
-// One cluster of up to 8 CTAs splits K.  A CTA copies its slice of X and of A
-// (64 rows of A at a time, up to 512 k) into shared memory with asynchronous
-// copies issued all at once -- one memory latency per slice -- and releases
-// the dependent launch as soon as the first slice is requested, so that these
-// loads queue ahead of the dependent kernel's.  Warp w then owns the 8-column
-// tile (w & 7) of the 64 and every other 16-wide chunk of the slice (w >> 3).
-// Partials are added in a fixed order: the two chunk halves in shared memory,
-// then the cluster ranks by rank 0 reading the others' shared memory.
-constexpr int kDownThreads = 512;
+// CTA (x, z) computes columns 16x .. 16x + 15 of T over the z-th of up to 8
+// slices of K; the slices of one column group form a cluster.  A CTA copies
+// its part of X and its 16 rows of A (up to 512 k at a time) into shared
+// memory with asynchronous copies issued all at once, and releases the
+// dependent launch as soon as they are requested, so that these loads queue
+// ahead of the dependent kernel's.  The CTAs are small (four warps, 37 KB of
+// shared memory) and many (one per SM for r = 64), so that the loads are
+// spread over SMs and the CTAs share SMs with the dependent kernel's.  Warp w
+// takes every fourth 16-wide chunk; partials are added in a fixed order: the
+// four warps in shared memory, then the cluster ranks by rank 0 reading the
+// others' shared memory.
+constexpr int kDownThreads = 128;
 constexpr int kDownMaxSplit = 8;
 constexpr int kDownBatch = 512;                 // k per staged slice
 constexpr int kDownStride = kDownBatch + 8;     // row stride (elements): 1040 bytes, conflict-free fragments
-constexpr int kDownSmem = (kMaxFewTokens + 64) * kDownStride * 2 + 2 * kMaxFewTokens * 256 * 4;
+constexpr int kDownSmem = 2 * kMaxFewTokens * kDownStride * 2 + 4 * kMaxFewTokens * 16 * 4;
 
 __device__ __forceinline__ void mma_m16n8k16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                              uint32_t b0, uint32_t b1) {
@@ -70,107 +73,97 @@ __device__ __forceinline__ void cp_async_wait_all() {
     asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
-__global__ void __launch_bounds__(kDownThreads, 1) k_few_down(const uint16_t* __restrict__ X,
-                                                               const uint16_t* __restrict__ A, int M, int K, int r,
-                                                               int r64, float s, uint16_t* __restrict__ T2,
-                                                               float* __restrict__ T_saved) {
+__global__ void __launch_bounds__(kDownThreads) k_few_down(const uint16_t* __restrict__ X,
+                                                            const uint16_t* __restrict__ A, int M, int K, int r,
+                                                            int r64, float s, uint16_t* __restrict__ T2,
+                                                            float* __restrict__ T_saved) {
     extern __shared__ __align__(16) uint8_t smem[];
-    uint16_t* sX = reinterpret_cast<uint16_t*>(smem);              // [16][kDownStride]
-    uint16_t* sA = sX + kMaxFewTokens * kDownStride;               // [64][kDownStride]
-    float* s_half = reinterpret_cast<float*>(sA + 64 * kDownStride);  // [16][256]
-    float* s_p = s_half + kMaxFewTokens * 256;                       // [16][256]
+    uint16_t* sX = reinterpret_cast<uint16_t*>(smem);                // [16][kDownStride]
+    uint16_t* sA = sX + kMaxFewTokens * kDownStride;                 // [16][kDownStride]
+    float* s_w = reinterpret_cast<float*>(sA + 16 * kDownStride);    // [4 warps][16 t][16 j]
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, q = lane & 3;
-    const int nt = warp & 7, kg = warp >> 3;
     const int splits = static_cast<int>(gridDim.z);
     const int rank = static_cast<int>(cluster_ctarank());
+    const int j0 = 16 * blockIdx.x;  // this CTA's columns of T
     const int bpr = K / 64;
     const int per = bpr / splits, extra = bpr % splits;
     const int k_begin = 64 * (rank * per + (rank < extra ? rank : extra));
     const int k_end = k_begin + 64 * (per + (rank < extra ? 1 : 0));
-    const int npass = r64 / 64;  // 64 columns of T per pass (<= 4)
-    float acc[4][4];
-#pragma unroll
-    for (int p = 0; p < 4; ++p)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[p][i] = 0.0f;
+    float acc[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
 
     bool released = false;
     for (int k0 = k_begin; k0 < k_end; k0 += kDownBatch) {
         const int kn = min(kDownBatch, k_end - k0);  // a multiple of 64
         const int pieces = kn / 8;                   // 16-byte pieces per row
-        for (int p = 0; p < npass; ++p) {
-            __syncthreads();  // the previous slice is no longer read
-            // rows of X (first pass of the slice only) and rows 64 p .. 64 p + 63 of A
-            const int xrows = p == 0 ? kMaxFewTokens : 0;
-            for (int i = tid; i < (xrows + 64) * pieces; i += kDownThreads) {
-                const int row = i / pieces, pc = i - row * pieces;
-                if (row < xrows) {
-                    uint16_t* dst = sX + row * kDownStride + pc * 8;
-                    if (row < M) cp_async16(dst, X + static_cast<int64_t>(row) * K + k0 + pc * 8);
-                    else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
-                } else {
-                    const int j = 64 * p + (row - xrows);
-                    uint16_t* dst = sA + (row - xrows) * kDownStride + pc * 8;
-                    if (j < r) cp_async16(dst, A + static_cast<int64_t>(j) * K + k0 + pc * 8);
-                    else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
-                }
+        __syncthreads();                             // the previous slice is no longer read
+        for (int i = tid; i < 2 * kMaxFewTokens * pieces; i += kDownThreads) {
+            const int row = i / pieces, pc = i - row * pieces;
+            if (row < kMaxFewTokens) {
+                uint16_t* dst = sX + row * kDownStride + pc * 8;
+                if (row < M) cp_async16(dst, X + static_cast<int64_t>(row) * K + k0 + pc * 8);
+                else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+            } else {
+                const int j = j0 + row - kMaxFewTokens;
+                uint16_t* dst = sA + (row - kMaxFewTokens) * kDownStride + pc * 8;
+                if (j < r) cp_async16(dst, A + static_cast<int64_t>(j) * K + k0 + pc * 8);
+                else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
             }
-            if (!released) {
-                allow_dependents();
-                released = true;
-            }
-            cp_async_wait_all();
-            __syncthreads();
-            const uint16_t* xr0 = sX + g * kDownStride + 2 * q;
-            const uint16_t* xr8 = xr0 + 8 * kDownStride;
-            const uint16_t* ar = sA + (8 * nt + g) * kDownStride + 2 * q;
-            for (int c = kg; c < kn / 16; c += 2) {
-                const int k = 16 * c;
-                mma_m16n8k16(acc[p], *reinterpret_cast<const uint32_t*>(xr0 + k), *reinterpret_cast<const uint32_t*>(xr8 + k),
-                             *reinterpret_cast<const uint32_t*>(xr0 + k + 8), *reinterpret_cast<const uint32_t*>(xr8 + k + 8),
-                             *reinterpret_cast<const uint32_t*>(ar + k), *reinterpret_cast<const uint32_t*>(ar + k + 8));
-            }
+        }
+        if (!released) {
+            allow_dependents();
+            released = true;
+        }
+        cp_async_wait_all();
+        __syncthreads();
+        const uint16_t* xr0 = sX + g * kDownStride + 2 * q;
+        const uint16_t* xr8 = xr0 + 8 * kDownStride;
+        const uint16_t* ar0 = sA + g * kDownStride + 2 * q;  // columns j0 .. j0 + 7
+        const uint16_t* ar1 = ar0 + 8 * kDownStride;         // columns j0 + 8 .. j0 + 15
+#pragma unroll 4
+        for (int c = warp; c < kn / 16; c += 4) {
+            const int k = 16 * c;
+            const uint32_t a0 = *reinterpret_cast<const uint32_t*>(xr0 + k), a1 = *reinterpret_cast<const uint32_t*>(xr8 + k);
+            const uint32_t a2 = *reinterpret_cast<const uint32_t*>(xr0 + k + 8), a3 = *reinterpret_cast<const uint32_t*>(xr8 + k + 8);
+            mma_m16n8k16(acc[0], a0, a1, a2, a3, *reinterpret_cast<const uint32_t*>(ar0 + k),
+                         *reinterpret_cast<const uint32_t*>(ar0 + k + 8));
+            mma_m16n8k16(acc[1], a0, a1, a2, a3, *reinterpret_cast<const uint32_t*>(ar1 + k),
+                         *reinterpret_cast<const uint32_t*>(ar1 + k + 8));
         }
     }
     if (!released) allow_dependents();
 
-    // acc[p]: tokens g (0, 1) and g + 8 (2, 3) at columns 64 p + 8 nt + 2q + {0, 1}
-    auto put = [&](float* dst, int p) {
-        const int j = 64 * p + 8 * nt + 2 * q;
-        dst[g * 256 + j] = acc[p][0];
-        dst[g * 256 + j + 1] = acc[p][1];
-        dst[(g + 8) * 256 + j] = acc[p][2];
-        dst[(g + 8) * 256 + j + 1] = acc[p][3];
-    };
-    if (kg == 1)
-        for (int p = 0; p < npass; ++p) put(s_half, p);
+    // acc[u]: tokens g (0, 1) and g + 8 (2, 3) at columns 8u + 2q + {0, 1}; the
+    // four warps' partials added in order by warp 0 into s_w[0]
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        float* dst = s_w + warp * 256;
+        const int j = 8 * u + 2 * q;
+        dst[g * 16 + j] = acc[u][0];
+        dst[g * 16 + j + 1] = acc[u][1];
+        dst[(g + 8) * 16 + j] = acc[u][2];
+        dst[(g + 8) * 16 + j + 1] = acc[u][3];
+    }
     __syncthreads();
-    if (kg == 0)
-        for (int p = 0; p < npass; ++p) {
-            const int j = 64 * p + 8 * nt + 2 * q;
-            acc[p][0] += s_half[g * 256 + j];
-            acc[p][1] += s_half[g * 256 + j + 1];
-            acc[p][2] += s_half[(g + 8) * 256 + j];
-            acc[p][3] += s_half[(g + 8) * 256 + j + 1];
-            put(s_p, p);
-        }
-    cluster_sync_all();  // every rank's partial is complete and visible
+    for (int i = tid; i < 256; i += kDownThreads) s_w[i] = ((s_w[i] + s_w[256 + i]) + s_w[512 + i]) + s_w[768 + i];
+    cluster_sync_all();  // every rank's partial (s_w[0 .. 255]) is complete and visible
     if (rank == 0) {
-        for (int i = tid; i < M * r64; i += kDownThreads) {
-            const int t = i / r64, j = i - t * r64;
+        for (int i = tid; i < M * 16; i += kDownThreads) {
+            const int t = i >> 4, jl = i & 15, j = j0 + jl;
             float part[kDownMaxSplit];
-            const uint32_t addr = smem_u32(&s_p[t * 256 + j]);
+            const uint32_t addr = smem_u32(&s_w[t * 16 + jl]);
 #pragma unroll
             for (int rk = 1; rk < kDownMaxSplit; ++rk)
                 if (rk < splits) part[rk] = ld_cluster_f32(cluster_map(addr, rk));
-            float v = s_p[t * 256 + j];
+            float v = s_w[t * 16 + jl];
 #pragma unroll
             for (int rk = 1; rk < kDownMaxSplit; ++rk)
                 if (rk < splits) v += part[rk];
             v *= s;
-            uint16_t* row = T2 + static_cast<int64_t>(t) * 2 * r64;
-            store_split(row + j, row + r64 + j, j < r ? v : 0.0f);
-            if (T_saved != nullptr && j < r) T_saved[static_cast<int64_t>(t) * r + j] = v;
+            if (j < r64) {
+                uint16_t* row = T2 + static_cast<int64_t>(t) * 2 * r64;
+                store_split(row + j, row + r64 + j, j < r ? v : 0.0f);
+                if (T_saved != nullptr && j < r) T_saved[static_cast<int64_t>(t) * r + j] = v;
+            }
         }
     }
     cluster_sync_all();  // rank 0 has read the other ranks' shared memory
@@ -268,11 +261,16 @@ cudaError_t launch_few_down(const uint16_t* X, const uint16_t* A, int M, int K, 
     if (dev < 0 || dev >= 64 || !configured[dev]) {
         e = cudaFuncSetAttribute(k_few_down, cudaFuncAttributeMaxDynamicSharedMemorySize, kDownSmem);
         if (e != cudaSuccess) return e;
+        // the same shared-memory carveout as the dependent kernel, so that an SM
+        // running this kernel can also take a CTA of that one
+        e = cudaFuncSetAttribute(k_few_down, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) configured[dev] = true;
     }
     const int splits = std::max(1, std::min(kDownMaxSplit, K / 64));
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(1, 1, splits);
+    cfg.gridDim = dim3(r64 / 16, 1, splits);
     cfg.blockDim = dim3(kDownThreads);
     cfg.dynamicSmemBytes = kDownSmem;
     cfg.stream = stream;
@@ -289,6 +287,17 @@ cudaError_t launch_few_down(const uint16_t* X, const uint16_t* A, int M, int K, 
 
 cudaError_t launch_few_v(const uint16_t* dY, const uint16_t* B, int M, int N, int r, int r64, float s,
                          uint16_t* V2, cudaStream_t stream) {
+    static bool configured[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64 || !configured[dev]) {
+        // the dependent kernel's shared-memory carveout (see launch_few_down)
+        e = cudaFuncSetAttribute(k_few_v, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) configured[dev] = true;
+    }
     cudaLaunchAttribute attr[1];
     cudaLaunchConfig_t cfg = cluster_config(dim3(r64 / 4, kVSplit), kVSplit, attr, stream);
     TraceScope trace("few_lora_v", stream);

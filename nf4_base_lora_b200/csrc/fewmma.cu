@@ -37,6 +37,7 @@
 #include <cstdint>
 
 #include "common.cuh"
+#include "decode.cuh"
 #include "kernels.h"
 #include "nf4_levels.cuh"
 #include "trace.h"
@@ -328,6 +329,269 @@ __global__ void __maxnreg__(96) k_few_fwd(const __grid_constant__ CUtensorMap ma
     cluster_wait_acquire();
 }
 
+// ---------------------------------------------------------------- input gradient
+// dX^T[k, t] = sum_n W_hat[n, k] dY[t, n] + sum_j [A ; A][j, k] V2[t, j]:
+// tensor-instruction roles A = 16 columns k x 16 rows n of W_hat (transposed),
+// B = 16 rows n x 8 tokens (dY), D = 16 columns x 8 tokens.  The operand pairs
+// of A run along n, i.e. across two code bytes of different rows, so the
+// decode goes through shared memory: each thread decodes one whole 64-block
+// of one weight row (one scale) with the register codebook into its warp's
+// padded tile [32 rows][64 + 8], and ldmatrix.trans hands out the transposed
+// pairs.  Warp w works on 64-column block (w & 1) of the CTA's 128 columns and
+// on every eighth 32-row chunk of the CTA's rows (w >> 1); the codes of up to
+// 1024 rows x 128 columns come in by TMA (64-byte swizzle) in four boxes.
+constexpr int kDxRowsSeg = 1024;
+constexpr int kDxTileStride = 144;                 // bytes per tile row: 64 bf16 + 16 bytes padding
+constexpr int kDxTileBytes = 32 * kDxTileStride;   // one warp's tile
+constexpr int kDxYStride = kDxRowsSeg + 8;         // dY staging, elements (2064 bytes: conflict-free)
+constexpr int kDxMaxSplit = 4;
+constexpr int kDxSmem = 1024 + kDxRowsSeg * 64 + 16 * kDxTileBytes + kTok * kDxYStride * 2 +
+                        (kDxMaxSplit - 1) * kPartFloats * 4;
+static_assert(7 * 2 * 32 * 32 * 4 <= 16 * kDxTileBytes, "warp reduction reuses the tiles");
+static_assert(kTok * (2 * 256 + 8) <= kTok * kDxYStride, "V2 staging reuses the dY staging");
+
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                                  uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+// The MMAs of one 32-row chunk held in the warp's tile, against activation
+// rows row0 .. row0 + 31 of the staged [16][ystride] array.
+__device__ __forceinline__ void dx_chunk_mma(float (&acc)[4][2][4], uint32_t tile_u32, const uint16_t* sy,
+                                             int ystride, int row0, int lane, bool two_halves) {
+    const int g = lane >> 2, q = lane & 3;
+    const int mi = lane >> 3, i = lane & 7;  // ldmatrix: this lane's row address of matrix mi
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+        const uint16_t* y0 = sy + g * ystride + row0 + 16 * s + 2 * q;
+        const uint16_t* y8 = y0 + 8 * ystride;
+        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(y0), b1 = *reinterpret_cast<const uint32_t*>(y0 + 8);
+        const uint32_t c0 = *reinterpret_cast<const uint32_t*>(y8), c1 = *reinterpret_cast<const uint32_t*>(y8 + 8);
+        const uint32_t row_addr = tile_u32 + (16 * s + 8 * (mi >> 1) + i) * kDxTileStride + 16 * (mi & 1);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            uint32_t a0, a1, a2, a3;
+            ldmatrix_x4_trans(row_addr + 32 * m, a0, a1, a2, a3);
+            mma_16816(acc[m][0], a0, a1, a2, a3, b0, b1);
+            if (two_halves) mma_16816(acc[m][1], a0, a1, a2, a3, c0, c1);
+        }
+    }
+}
+
+__global__ void __maxnreg__(128) k_few_dx(const __grid_constant__ CUtensorMap map_codes, const FewArgs a) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    __shared__ uint64_t bar_part, bar_c[4];
+    __shared__ int s_abort;
+    // [codes: kDxRowsSeg rows x 64 B, 64-byte swizzle][16 warp tiles][dY staging][partial slots]
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t* s_codes = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    uint8_t* s_tiles = s_codes + kDxRowsSeg * 64;
+    uint16_t* sY = reinterpret_cast<uint16_t*>(s_tiles + 16 * kDxTileBytes);
+    float* s_part = reinterpret_cast<float*>(sY + kTok * kDxYStride);  // [kDxMaxSplit - 1][32 values][64 threads]
+    float* s_red = reinterpret_cast<float*>(s_tiles);                   // [7][2][32 values][32 lanes], after the loop
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, q = lane & 3;
+    const int cb = warp & 1, rw = warp >> 1;
+    const int splits = static_cast<int>(gridDim.z);
+    const int rank = static_cast<int>(cluster_ctarank());
+    const int M = a.M, N = a.N, K = a.K;
+    const int bpr = K / 64;
+    const int blk = 2 * blockIdx.x + cb;
+    const bool blk_ok = blk < bpr;
+    int ch0, ch1;  // this rank's 32-row chunks
+    split_range((N + 31) / 32, splits, rank, ch0, ch1);
+    auto issue_codes = [&](int sc0, int sc1) {
+        for (int b = 0; 8 * b < sc1 - sc0; ++b) {
+            mbar_arrive_expect_tx(&bar_c[b], 256 * 64);
+            tma_load_2d(s_codes + b * 256 * 64, &map_codes, &bar_c[b], 64 * blockIdx.x, 32 * (sc0 + 8 * b));
+        }
+    };
+    if (tid == 0) {
+        mbar_init(&bar_part, splits > 1 ? (splits - 1) * 64 : 1);
+        for (int b = 0; b < 4; ++b) mbar_init(&bar_c[b], 1);
+        s_abort = 0;
+        fence_barrier_init();
+        if (ch0 < ch1) {
+            tma_prefetch_desc(&map_codes);
+            issue_codes(ch0, min(ch1, ch0 + kDxRowsSeg / 32));
+        }
+    }
+    const bool two_halves = M > 8;
+    float acc[4][2][4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m)
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[m][h][e] = 0.0f;
+    __syncthreads();
+    cluster_arrive_relaxed();  // barriers initialised (made visible by the init fence)
+    const float mu = __ldg(a.scale_mean);
+    volatile int* abort_flag = &s_abort;
+    uint8_t* my_tile = s_tiles + warp * kDxTileBytes;
+    const uint32_t my_tile_u32 = smem_u32(my_tile);
+
+    int seg_i = 0, issued_seg = 0, issued_boxes = ch0 < ch1 ? (min(ch1, ch0 + kDxRowsSeg / 32) - ch0 + 7) / 8 : 0;
+    for (int sc0 = ch0; sc0 < ch1; sc0 += kDxRowsSeg / 32, ++seg_i) {
+        const int sc1 = min(ch1, sc0 + kDxRowsSeg / 32);
+        const int rows = 32 * (sc1 - sc0);  // staged rows (the last ones may lie beyond N)
+        if (seg_i > 0) {
+            __syncthreads();  // the previous segment's codes, tiles and dY are no longer read
+            if (*abort_flag) break;
+            if (tid == 0) issue_codes(sc0, sc1);
+            issued_seg = seg_i;
+            issued_boxes = (sc1 - sc0 + 7) / 8;
+        }
+        // dY[:, 32 sc0 : 32 sc1] (rows >= N, tokens >= M as zeros) and this thread's scales
+        uint2 yv[8];
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+            const int i = tid + p * kThreads, t = i / (rows / 4), pc = i - t * (rows / 4);
+            const int n = 32 * sc0 + 4 * pc;
+            yv[p] = make_uint2(0, 0);
+            if (t < M && n < N) yv[p] = __ldg(reinterpret_cast<const uint2*>(a.act + static_cast<int64_t>(t) * N + n));
+        }
+        int qv[4];
+        float a2v[4];
+#pragma unroll
+        for (int it = 0; it < 4; ++it) {
+            const int c = sc0 + rw + 8 * it, n = 32 * c + lane;
+            const bool ok = c < sc1 && n < N && blk_ok;
+            const int64_t bi = static_cast<int64_t>(n) * bpr + blk;
+            qv[it] = ok ? static_cast<int>(__ldg(a.qscale + bi)) : 0;
+            a2v[it] = ok ? __ldg(a.scale2 + (bi >> 8)) : 0.0f;
+        }
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+            const int i = tid + p * kThreads, t = i / (rows / 4), pc = i - t * (rows / 4);
+            if (t < kTok) *reinterpret_cast<uint2*>(sY + t * kDxYStride + 4 * pc) = yv[p];
+        }
+        __syncthreads();
+#pragma unroll 1
+        for (int it = 0; it < 4; ++it) {
+            const int c = sc0 + rw + 8 * it;
+            if (c >= sc1) break;
+            const int lr = 32 * (c - sc0) + lane;  // staged row of this thread
+            if (!mbar_wait(&bar_c[(c - sc0) / 8], seg_i & 1, abort_flag)) break;
+            const int n = 32 * c + lane;
+            const bool ok = n < N && blk_ok;
+            const float sc = ok ? nf4_block_scale(static_cast<int8_t>(qv[it]), a2v[it], mu) : 0.0f;
+            // the row's 32 code bytes of block cb: 16-byte chunks 2 cb, 2 cb + 1, swizzled by row
+            const uint8_t* crow = s_codes + lr * 64;
+            const int sw = (lr >> 1) & 3;
+            const uint4 u0 = *reinterpret_cast<const uint4*>(crow + (((2 * cb) ^ sw) << 4));
+            const uint4 u1 = *reinterpret_cast<const uint4*>(crow + (((2 * cb + 1) ^ sw) << 4));
+            const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+            uint32_t d[32];
+            nf4_decode_block(w, sc, d);
+            uint4* trow = reinterpret_cast<uint4*>(my_tile + lane * kDxTileStride);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) trow[j] = make_uint4(d[4 * j], d[4 * j + 1], d[4 * j + 2], d[4 * j + 3]);
+            __syncwarp();
+            dx_chunk_mma(acc, my_tile_u32, sY, kDxYStride, 32 * (c - sc0), lane, two_halves);
+            __syncwarp();
+        }
+    }
+    if (tid == 0 && *abort_flag) {
+        for (int b = 0; b < issued_boxes; ++b) mbar_drain(&bar_c[b], issued_seg & 1);
+    }
+
+    // rank-r extension on rank 0: the rows of [A ; A] as 32-row chunks through
+    // the same tiles, against V2 staged in place of dY, once the kernel
+    // producing V2 has finished
+    if (rank == 0 && a.ext_act != nullptr) {
+        if (a.pdl) wait_prerequisites();
+        const int vstride = 2 * a.r64 + 8;
+        __syncthreads();  // dY staging and tiles are free
+        for (int i = tid; i < kTok * (2 * a.r64 / 4); i += kThreads) {
+            const int t = i / (2 * a.r64 / 4), pc = i - t * (2 * a.r64 / 4);
+            uint2 v = make_uint2(0, 0);
+            if (t < M) v = __ldg(reinterpret_cast<const uint2*>(a.ext_act + static_cast<int64_t>(t) * 2 * a.r64) + pc);
+            *reinterpret_cast<uint2*>(sY + t * vstride + 4 * pc) = v;
+        }
+        __syncthreads();
+        for (int c = rw; c < 2 * a.r64 / 32; c += 8) {
+            const int j = (32 * c + lane) % a.r64;  // row of A (the same in both halves)
+            uint4* trow = reinterpret_cast<uint4*>(my_tile + lane * kDxTileStride);
+            const uint4* arow = reinterpret_cast<const uint4*>(a.ext_w + static_cast<int64_t>(j) * K + 64 * blk);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) trow[k] = (j < a.r && blk_ok) ? __ldg(arow + k) : make_uint4(0, 0, 0, 0);
+            __syncwarp();
+            dx_chunk_mma(acc, my_tile_u32, sY, vstride, 32 * c, lane, two_halves);
+            __syncwarp();
+        }
+    }
+
+    // the eight row warps of a block add up in order (into row warp 0), then
+    // ranks > 0 push to rank 0, which adds the ranks in order
+    __syncthreads();  // tiles are free for the reduction
+    if (rw > 0) {
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    s_red[(((rw - 1) * 2 + cb) * 32 + (m * 8 + h * 4 + e)) * 32 + lane] = acc[m][h][e];
+    }
+    __syncthreads();
+    bool waited = false;
+    if (rw == 0) {
+        for (int k = 0; k < 7; ++k)
+#pragma unroll
+            for (int m = 0; m < 4; ++m)
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) acc[m][h][e] += s_red[((k * 2 + cb) * 32 + (m * 8 + h * 4 + e)) * 32 + lane];
+        const int slot = cb * 32 + lane;  // 0..63
+        if (rank != 0) {
+            cluster_wait_acquire();
+            waited = true;
+#pragma unroll
+            for (int m = 0; m < 4; ++m)
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        st_cluster_f32(cluster_map(smem_u32(s_part + ((rank - 1) * 32 + (m * 8 + h * 4 + e)) * 64 + slot), 0),
+                                       acc[m][h][e]);
+            mbar_arrive_remote(cluster_map(smem_u32(&bar_part), 0));
+        } else {
+            const bool got = splits == 1 || mbar_wait_cluster(&bar_part, 0, &s_abort);
+            if (got && blk_ok) {
+                for (int rk = 1; rk < splits; ++rk)
+#pragma unroll
+                    for (int m = 0; m < 4; ++m)
+#pragma unroll
+                        for (int h = 0; h < 2; ++h)
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                acc[m][h][e] += s_part[((rk - 1) * 32 + (m * 8 + h * 4 + e)) * 64 + slot];
+                // acc[m][h]: columns 16m + g (e = 0, 1) and + 8 (e = 2, 3), tokens 2q + 8h + (e & 1)
+#pragma unroll
+                for (int m = 0; m < 4; ++m)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int t = 2 * q + 8 * h + (e & 1);
+                            const int col = 64 * blk + 16 * m + g + 8 * (e >> 1);
+                            if (t < M) {
+                                const __nv_bfloat16 b = __float2bfloat16_rn(acc[m][h][e]);
+                                a.out[static_cast<int64_t>(t) * K + col] = *reinterpret_cast<const uint16_t*>(&b);
+                            }
+                        }
+            }
+        }
+    }
+    if (!waited) cluster_wait_acquire();
+    cluster_arrive_release();
+    cluster_wait_acquire();
+}
+
 // `configured`: per-device flags of this kernel (both kernels have the same
 // type, so the flags cannot live in the template)
 template <typename Kern, typename... Params>
@@ -369,7 +633,7 @@ cudaError_t launch_cluster(Kern kern, bool (&configured)[64], int smem, const ch
 
 }  // namespace
 
-int few_max_split(bool forward) { return forward ? kFwdMaxSplit : kMaxSplit; }
+int few_max_split(bool forward) { return forward ? kFwdMaxSplit : kDxMaxSplit; }
 
 cudaError_t launch_few_fwd(const CUtensorMap& map_codes, const FewArgs& a, int splits, cudaStream_t stream) {
     if (a.M < 1 || a.M > kTok || a.K % 64 != 0 || a.N % 8 != 0 || splits > a.K / 64 || splits > kFwdMaxSplit)
@@ -377,6 +641,15 @@ cudaError_t launch_few_fwd(const CUtensorMap& map_codes, const FewArgs& a, int s
     static bool configured[64] = {};
     return launch_cluster(k_few_fwd, configured, kFwdSmemV2, "nf4_gemm_fwd_few", a, (a.N + kTile - 1) / kTile, splits,
                           stream, map_codes);
+}
+
+cudaError_t launch_few_dx(const CUtensorMap& map_codes, const FewArgs& a, int splits, cudaStream_t stream) {
+    if (a.M < 1 || a.M > kTok || a.K % 64 != 0 || a.N % 8 != 0 || splits > (a.N + 31) / 32 || splits > kDxMaxSplit ||
+        a.r64 > 256)
+        return cudaErrorInvalidValue;
+    static bool configured[64] = {};
+    return launch_cluster(k_few_dx, configured, kDxSmem, "nf4_gemm_dx_few", a, (a.K + 127) / 128, splits, stream,
+                          map_codes);
 }
 
 }  // namespace nf4lora

@@ -41,5 +41,8 @@ int few_max_split(bool forward);
 // map_codes: the packed codes as bytes [N, K / 2], box {128 bytes, 128 rows},
 // 128-byte swizzle
 cudaError_t launch_few_fwd(const CUtensorMap& map_codes, const FewArgs& a, int splits, cudaStream_t stream);
+// map_codes: the packed codes as bytes [N, K / 2], box {64 bytes, 256 rows},
+// 64-byte swizzle
+cudaError_t launch_few_dx(const CUtensorMap& map_codes, const FewArgs& a, int splits, cudaStream_t stream);
 
 }  // namespace nf4lora

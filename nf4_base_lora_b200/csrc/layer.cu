@@ -72,7 +72,8 @@ static bool map_bf16(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t o
 
 // Packed NF4 codes viewed as bytes [d_out, d_in / 2], box {box_inner bytes, box_outer rows}.
 static bool map_codes(CUtensorMap* m, const uint8_t* codes, int64_t d_out, int64_t d_in,
-                      uint32_t box_inner, uint32_t box_outer, bool swizzle128 = false) {
+                      uint32_t box_inner, uint32_t box_outer,
+                      CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_NONE) {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(d_in / 2), static_cast<cuuint64_t>(d_out)};
@@ -80,7 +81,7 @@ static bool map_codes(CUtensorMap* m, const uint8_t* codes, int64_t d_out, int64
     cuuint32_t box[2] = {box_inner, box_outer};
     cuuint32_t estr[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -274,14 +275,6 @@ static int few_splits(int tiles, int units, int sms, bool forward) {
     return std::max(1, std::min({few_max_split(forward), sms / std::max(1, tiles), units}));
 }
 
-// few-token input gradient on the tcgen05 engine (one CTA per SM): 12 load
-// slots of 6 KB + 8 decoded tiles of 16 KB + partial-tile slots; four decode
-// teams, each on every fourth k-step; at most 4 splits (the slots of rank 0)
-static constexpr int kDxLoad = 12;
-static constexpr int kDxDec = 8;
-static constexpr int kDxTeams = 4;
-static constexpr int kDxMaxSplit = 4;
-
 static FewArgs few_args(const LayerCtx& c, const uint16_t* act, int M, const uint16_t* ext_act,
                         const uint16_t* ext_w, int r, int r64, uint16_t* out) {
     FewArgs a{};
@@ -385,7 +378,7 @@ int layer_fwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, fl
             return -2;
         const FewArgs fa = few_args(c, X, static_cast<int>(M), T2, B, r, r64, Y);
         const int splits = few_splits(ceil_div(c.d_out, 128), static_cast<int>(c.d_in / 64), c.num_sms, true);
-        if (!map_codes(&m.a, c.codes, c.d_out, c.d_in, 128, 128, true)) return -1;
+        if (!map_codes(&m.a, c.codes, c.d_out, c.d_in, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return -1;
         return note(launch_few_fwd(m.a, fa, splits, c.stream)) == cudaSuccess ? 0 : -2;
     }
     int rc = lora_down(c, A, r, s, X, M, T2, T_saved, part);
@@ -467,25 +460,11 @@ int layer_bwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, fl
         g.k_ext = 2 * kx;
         g.alpha = 1.0f;
         if (few) {
-            // swapped: D[k, m] = sum_n W_hat[n, k] dY[m, n] + sum_j A[j, k] V[m, j] on the
-            // tcgen05 engine (the decoded tile goes to shared memory in the MN-major
-            // layout the tensor core reads transposed), split-K over a cluster, a
-            // programmatic dependent of the V kernel just launched
-            if (!map_codes(&m.a, c.codes, c.d_out, c.d_in, 64, 64) || !map_bf16(&m.b, dY, c.d_out, M, c.d_out, 16) ||
-                !map_bf16(&m.ae, A, c.d_in, r, c.d_in, 64) || !map_bf16(&m.be, V2, 2 * r64, M, 2 * r64, 16))
-                return -1;
-            const int tiles = ceil_div(c.d_in, 128);
-            const int splits = std::max(1, std::min({kDxMaxSplit, c.num_sms / tiles, ceil_div(c.d_out, 64) / 2}));
-            g.ext_wrap_a = kx;
-            g.rows = static_cast<int>(c.d_in);
-            g.cols = static_cast<int>(M);
-            g.out = dX;
-            g.ldo = c.d_in;
-            g.pdl = 1;
-            dim3 grid(tiles, 1, splits);
-            if (launch<16, SRC_DEC_MN, SRC_TMA_K, 1, 0, EPI_CLUSTER_BF16_T, kDxLoad, kDxDec, kDxTeams>(
-                    "nf4_gemm_dx_few", m.a, m.b, m.ae, m.be, g, grid, c.stream, splits) != cudaSuccess)
-                return -2;
+            // a programmatic dependent of the V kernel just launched
+            const FewArgs fa = few_args(c, dY, static_cast<int>(M), V2, A, r, r64, dX);
+            const int splits = few_splits(ceil_div(c.d_in, 128), ceil_div(c.d_out, 32), c.num_sms, false);
+            if (!map_codes(&m.a, c.codes, c.d_out, c.d_in, 64, 256, CU_TENSOR_MAP_SWIZZLE_64B)) return -1;
+            if (note(launch_few_dx(m.a, fa, splits, c.stream)) != cudaSuccess) return -2;
         } else {
             if (!map_bf16(&m.a, dY, c.d_out, M, c.d_out, 128) || !map_codes(&m.b, c.codes, c.d_out, c.d_in, 128, 64) ||
                 !map_bf16(&m.ae, V2, 2 * r64, M, 2 * r64, 128) || !map_bf16(&m.be, A, c.d_in, r, c.d_in, 64))
