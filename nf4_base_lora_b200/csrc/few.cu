@@ -1,7 +1,6 @@
 // Rank-r intermediates for few tokens (M <= 16):
-//   T = s X A^T   (forward, "第 04 篇：QLoRA 原理" §6.3, the LoRA down product;
-//                  warp-level tensor instructions)
-//   V = s dY B    (backward, §2.4, the input-gradient branch through B; CUDA cores)
+//   T = s X A^T   (forward, "第 04 篇：QLoRA 原理" §6.3, the LoRA down product)
+//   V = s dY B    (backward, §2.4, the input-gradient branch through B)
 // Each writes the bf16 hi | lo pair the fused products' extension steps
 // consume (and T in fp32 for reuse by the backward) and lets the fused
 // dequant-GEMM that follows launch early (programmatic dependent launch): the
@@ -28,8 +27,6 @@ __device__ __forceinline__ void allow_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
 
 __device__ __forceinline__ void store_split(uint16_t* dst_hi, uint16_t* dst_lo, float v) {
     const __nv_bfloat16 hi = __float2bfloat16_rn(v);
@@ -169,87 +166,114 @@ __global__ void __launch_bounds__(kDownThreads) k_few_down(const uint16_t* __res
     cluster_sync_all();  // rank 0 has read the other ranks' shared memory
 }
 
-constexpr int kVSplit = 8;      // cluster size along d_out for V
+// V on the warp-level tensor instructions: D[t, j] = sum_n dY[t, n] B[n, j]
+// (m16n8k16: A operand = dY, 16 tokens x 16 n; B operand = B[n][j] read
+// transposed from shared memory with ldmatrix.trans).  The same layout as the
+// T kernel: CTA (x, z) computes columns 16x .. 16x + 15 of V over the z-th of
+// up to 8 slices of d_out, the slices of one column group form a cluster, the
+// slice of dY and of B (up to 512 rows at a time) comes in by asynchronous
+// copies issued at once, and the dependent launch is released right after.
+constexpr int kVBatch = 512;                    // rows of B per staged slice
+constexpr int kVYStride = kVBatch + 8;          // dY staging row stride (elements)
+constexpr int kVBStride = 24;                   // B staging row stride (elements): 48 bytes, conflict-free ldmatrix
+constexpr int kVSmem = kMaxFewTokens * kVYStride * 2 + kVBatch * kVBStride * 2 + 4 * kMaxFewTokens * 16 * 4;
 
-// V: cluster (1, kVSplit) per 4 columns of V; CTA rank ns covers rows
-// n in [ns N / kVSplit, (ns + 1) N / kVSplit); thread t takes rows t, t + 128, ...
-__global__ void __launch_bounds__(128) k_few_v(const uint16_t* __restrict__ dY, const uint16_t* __restrict__ B,
-                                               int M, int N, int r, int r64, float s, uint16_t* __restrict__ V2) {
-    allow_dependents();
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int j0 = blockIdx.x * 4;
-    const int ns = static_cast<int>(cluster_ctarank());
-    const int n_len = (N + kVSplit - 1) / kVSplit;
-    const int n0 = ns * n_len;
-    const int n1 = min(N, n0 + n_len);
-    float acc[kMaxFewTokens][4];
-#pragma unroll
-    for (int m = 0; m < kMaxFewTokens; ++m)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) acc[m][q] = 0.0f;
-    if (j0 < r) {
+__device__ __forceinline__ void ldmatrix_x2_trans(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
+}
+
+__global__ void __launch_bounds__(kDownThreads) k_few_v(const uint16_t* __restrict__ dY,
+                                                         const uint16_t* __restrict__ B, int M, int N, int r,
+                                                         int r64, float s, uint16_t* __restrict__ V2) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    uint16_t* sY = reinterpret_cast<uint16_t*>(smem);             // [16][kVYStride]
+    uint16_t* sB = sY + kMaxFewTokens * kVYStride;               // [kVBatch][kVBStride]: rows n, columns j0 .. j0 + 15
+    float* s_w = reinterpret_cast<float*>(sB + kVBatch * kVBStride);  // [4 warps][16 t][16 j]
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, q = lane & 3;
+    const int splits = static_cast<int>(gridDim.z);
+    const int rank = static_cast<int>(cluster_ctarank());
+    const int j0 = 16 * blockIdx.x;
+    const int nq = (N + 15) / 16;  // 16-row chunks of d_out
+    const int per = nq / splits, extra = nq % splits;
+    const int n_begin = 16 * (rank * per + (rank < extra ? rank : extra));
+    const int n_end = n_begin + 16 * (per + (rank < extra ? 1 : 0));
+    float acc[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
+
+    bool released = false;
+    for (int n0 = n_begin; n0 < n_end; n0 += kVBatch) {
+        const int nn = min(kVBatch, n_end - n0);  // a multiple of 16
+        __syncthreads();                          // the previous slice is no longer read
+        // dY[:, n0 : n0 + nn] in 16-byte pieces (N is a multiple of 8)
+        for (int i = tid; i < kMaxFewTokens * (nn / 8); i += kDownThreads) {
+            const int t = i / (nn / 8), pc = i - t * (nn / 8), n = n0 + 8 * pc;
+            uint16_t* dst = sY + t * kVYStride + 8 * pc;
+            if (t < M && n < N) cp_async16(dst, dY + static_cast<int64_t>(t) * N + n);
+            else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+        }
+        // B[n0 : n0 + nn, j0 : j0 + 16] in 16-byte pieces (r is a multiple of 8)
+        for (int i = tid; i < nn * 2; i += kDownThreads) {
+            const int row = i >> 1, h = i & 1, n = n0 + row, j = j0 + 8 * h;
+            uint16_t* dst = sB + row * kVBStride + 8 * h;
+            if (n < N && j < r) cp_async16(dst, B + static_cast<int64_t>(n) * r + j);
+            else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+        }
+        if (!released) {
+            allow_dependents();
+            released = true;
+        }
+        cp_async_wait_all();
+        __syncthreads();
+        const uint16_t* y0 = sY + g * kVYStride + 2 * q;
+        const uint16_t* y8 = y0 + 8 * kVYStride;
+        const int mi = lane >> 3, li = lane & 7;  // ldmatrix.x2: matrix mi (rows 8 mi .. 8 mi + 7 of the chunk)
 #pragma unroll 4
-        for (int n = n0 + tid; n < n1; n += 128) {
-            const uint2 b = __ldg(reinterpret_cast<const uint2*>(B + static_cast<int64_t>(n) * r + j0));
-            const float bf[4] = {bf16_lo(b.x), bf16_hi(b.x), bf16_lo(b.y), bf16_hi(b.y)};
-#pragma unroll
-            for (int m = 0; m < kMaxFewTokens; ++m) {
-                if (m < M) {
-                    const float d = __uint_as_float(static_cast<uint32_t>(__ldg(dY + static_cast<int64_t>(m) * N + n))
-                                                    << 16);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) acc[m][q] = fmaf(d, bf[q], acc[m][q]);
-                }
-            }
+        for (int c = warp; c < nn / 16; c += 4) {
+            const int k = 16 * c;
+            const uint32_t a0 = *reinterpret_cast<const uint32_t*>(y0 + k), a1 = *reinterpret_cast<const uint32_t*>(y8 + k);
+            const uint32_t a2 = *reinterpret_cast<const uint32_t*>(y0 + k + 8), a3 = *reinterpret_cast<const uint32_t*>(y8 + k + 8);
+            const uint32_t brow = smem_u32(sB + (k + 8 * (mi & 1) + li) * kVBStride);
+            uint32_t b0, b1, c0, c1;
+            ldmatrix_x2_trans(brow, b0, b1);        // columns j0 .. j0 + 7
+            ldmatrix_x2_trans(brow + 16, c0, c1);   // columns j0 + 8 .. j0 + 15
+            mma_m16n8k16(acc[0], a0, a1, a2, a3, b0, b1);
+            mma_m16n8k16(acc[1], a0, a1, a2, a3, c0, c1);
         }
     }
-    __shared__ float red[4][kMaxFewTokens][4];
-    __shared__ float part[kMaxFewTokens][4];
+    if (!released) allow_dependents();
+
 #pragma unroll
-    for (int m = 0; m < kMaxFewTokens; ++m)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            float v = acc[m][q];
-#pragma unroll
-            for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            if (lane == 0) red[warp][m][q] = v;
-        }
+    for (int u = 0; u < 2; ++u) {
+        float* dst = s_w + warp * 256;
+        const int j = 8 * u + 2 * q;
+        dst[g * 16 + j] = acc[u][0];
+        dst[g * 16 + j + 1] = acc[u][1];
+        dst[(g + 8) * 16 + j] = acc[u][2];
+        dst[(g + 8) * 16 + j + 1] = acc[u][3];
+    }
     __syncthreads();
-    if (tid < 4 * kMaxFewTokens) {
-        const int m = tid >> 2, q = tid & 3;
-        part[m][q] = ((red[0][m][q] + red[1][m][q]) + red[2][m][q]) + red[3][m][q];
-    }
+    for (int i = tid; i < 256; i += kDownThreads) s_w[i] = ((s_w[i] + s_w[256 + i]) + s_w[512 + i]) + s_w[768 + i];
     cluster_sync_all();
-    if (ns == 0 && tid < 4 * M) {
-        const int m = tid >> 2, q = tid & 3, j = j0 + q;
-        float t[kVSplit];
+    if (rank == 0) {
+        for (int i = tid; i < M * 16; i += kDownThreads) {
+            const int t = i >> 4, jl = i & 15, j = j0 + jl;
+            float part[kDownMaxSplit];
+            const uint32_t addr = smem_u32(&s_w[t * 16 + jl]);
 #pragma unroll
-        for (int rk = 0; rk < kVSplit; ++rk) t[rk] = ld_cluster_f32(cluster_map(smem_u32(&part[m][q]), rk));
-        float v = 0.0f;
+            for (int rk = 1; rk < kDownMaxSplit; ++rk)
+                if (rk < splits) part[rk] = ld_cluster_f32(cluster_map(addr, rk));
+            float v = s_w[t * 16 + jl];
 #pragma unroll
-        for (int rk = 0; rk < kVSplit; ++rk) v += t[rk];
-        v *= s;
-        uint16_t* row = V2 + static_cast<int64_t>(m) * 2 * r64;
-        if (j < r64) store_split(row + j, row + r64 + j, j < r ? v : 0.0f);
+            for (int rk = 1; rk < kDownMaxSplit; ++rk)
+                if (rk < splits) v += part[rk];
+            v *= s;
+            uint16_t* row = V2 + static_cast<int64_t>(t) * 2 * r64;
+            if (j < r64) store_split(row + j, row + r64 + j, j < r ? v : 0.0f);
+        }
     }
     cluster_sync_all();
 }
 
 }  // namespace
-
-static cudaLaunchConfig_t cluster_config(dim3 grid, int split, cudaLaunchAttribute* attr, cudaStream_t stream) {
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = grid;
-    cfg.blockDim = dim3(128);
-    cfg.stream = stream;
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 1;
-    attr[0].val.clusterDim.y = split;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cfg;
-}
 
 cudaError_t launch_few_down(const uint16_t* X, const uint16_t* A, int M, int K, int r, int r64, float s,
                             uint16_t* T2, float* T_saved, cudaStream_t stream) {
@@ -287,19 +311,33 @@ cudaError_t launch_few_down(const uint16_t* X, const uint16_t* A, int M, int K, 
 
 cudaError_t launch_few_v(const uint16_t* dY, const uint16_t* B, int M, int N, int r, int r64, float s,
                          uint16_t* V2, cudaStream_t stream) {
+    if (M < 1 || M > kMaxFewTokens || N % 8 != 0 || r % 8 != 0 || r64 > 256) return cudaErrorInvalidValue;
     static bool configured[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64 || !configured[dev]) {
+        e = cudaFuncSetAttribute(k_few_v, cudaFuncAttributeMaxDynamicSharedMemorySize, kVSmem);
+        if (e != cudaSuccess) return e;
         // the dependent kernel's shared-memory carveout (see launch_few_down)
         e = cudaFuncSetAttribute(k_few_v, cudaFuncAttributePreferredSharedMemoryCarveout,
                                  cudaSharedmemCarveoutMaxShared);
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) configured[dev] = true;
     }
+    const int splits = std::max(1, std::min(kDownMaxSplit, (N + 15) / 16));
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(r64 / 16, 1, splits);
+    cfg.blockDim = dim3(kDownThreads);
+    cfg.dynamicSmemBytes = kVSmem;
+    cfg.stream = stream;
     cudaLaunchAttribute attr[1];
-    cudaLaunchConfig_t cfg = cluster_config(dim3(r64 / 4, kVSplit), kVSplit, attr, stream);
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = splits;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     TraceScope trace("few_lora_v", stream);
     return cudaLaunchKernelEx(&cfg, k_few_v, dY, B, M, N, r, r64, s, V2);
 }
