@@ -447,6 +447,17 @@ __global__ void __launch_bounds__(GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI, 
                 constexpr bool kMNdec = C::kDecA ? (ASRC == SRC_DEC_MN) : (BSRC == SRC_DEC_MN);
                 constexpr int kCB = C::kDecMN / 64;           // 64-blocks across the decoded tile
                 const int tile_mn0 = C::kDecA ? r0 : c0;
+                // MN-major: this thread's unit is (k-row n_local of the step, block c
+                // of the tile).  The eight threads of a quarter warp take eight
+                // consecutive rows (their swizzled 16-byte stores hit eight
+                // different bank groups) and blocks spread so that their 32-byte
+                // code reads land at most two to a bank group.
+                int n_local = dt, cblk = 0;
+                if constexpr (kMNdec) {
+                    const int qw = dt >> 3, i = dt & 7;
+                    n_local = 8 * (qw / kCB) + i;
+                    cblk = ((i * kCB) / 4 + qw % kCB) % kCB;
+                }
                 // (weight row, 64-block) decoded by this thread at main step `it`
                 auto unit = [&](int it, int64_t& wrow, int64_t& wblk) {
                     const int kb = kb_begin + it;
@@ -454,18 +465,19 @@ __global__ void __launch_bounds__(GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI, 
                         wrow = tile_mn0 + dt;
                         wblk = kb;
                     } else {
-                        wrow = static_cast<int64_t>(kb) * 64 + dt / kCB;
-                        wblk = tile_mn0 / 64 + dt % kCB;
+                        wrow = static_cast<int64_t>(kb) * 64 + n_local;
+                        wblk = tile_mn0 / 64 + cblk;
                     }
                 };
-                int dst_off, swz;
+                int dst_off, swz, code_off;
                 if constexpr (!kMNdec) {
                     dst_off = dt * 128;
                     swz = dt & 7;
+                    code_off = dt * 32;
                 } else {
-                    const int n_local = dt / kCB, c = dt % kCB;
-                    dst_off = c * 8192 + n_local * 128;
+                    dst_off = cblk * 8192 + n_local * 128;
                     swz = n_local & 7;
+                    code_off = (n_local * kCB + cblk) * 32;  // codes tile: [64 k-rows][kCB blocks x 32 bytes]
                 }
                 // Block scales are prefetched kPf of this team's steps ahead
                 // into registers, so no decode waits on a dependent load.
@@ -502,8 +514,8 @@ __global__ void __launch_bounds__(GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI, 
                         }
                         uint8_t* dst = dec_slot(it) + dst_off;
                         if (!valid) zero_row(dst);
-                        else if constexpr (kRegisterCodebook) decode_unit_reg(codes_buf(it) + dt * 32, sc, dst, swz);
-                        else decode_unit(codes_buf(it) + dt * 32, sc, dst, swz, s_lut);
+                        else if constexpr (kRegisterCodebook) decode_unit_reg(codes_buf(it) + code_off, sc, dst, swz);
+                        else decode_unit(codes_buf(it) + code_off, sc, dst, swz, s_lut);
                         fence_proxy_async_smem();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&bar_dfull[it % DS]);
