@@ -317,9 +317,12 @@ class GpuWorkload:
             enc = d["encs"][(copy_base + p) % len(d["encs"])]
             x = (X[i] if X is not None else d["X"])[:m]
             if kind == "fwd":
-                nf.qlora_linear_fwd(enc, d["A"], d["B"], wl.scaling, x, save_t=False,
-                                    Y=(outs[i]["Y"][m] if outs else d["Y"][m]), workspace=self.ws)
-                # T is produced again by the next pass's forward of the same batch
+                # a full backward follows: the forward keeps T = s X A^T (fp32) for it,
+                # as a training step does; a dX-only backward needs no T
+                keep = wl.backward != "dx"
+                nf.qlora_linear_fwd(enc, d["A"], d["B"], wl.scaling, x, save_t=keep,
+                                    Y=(outs[i]["Y"][m] if outs else d["Y"][m]), workspace=self.ws,
+                                    T=d["T"][m])
             else:
                 dy = (dY[i] if dY is not None else d["dY"])[:m]
                 if kind == "dx":
@@ -327,7 +330,7 @@ class GpuWorkload:
                                         need_db=False, dX=(outs[i]["dX"][m] if outs else d["dX"][m]),
                                         workspace=self.ws)
                 else:
-                    nf.qlora_linear_bwd(enc, d["A"], d["B"], wl.scaling, x, None, dy, dA=d["dA"], dB=d["dB"],
+                    nf.qlora_linear_bwd(enc, d["A"], d["B"], wl.scaling, x, d["T"][m], dy, dA=d["dA"], dB=d["dB"],
                                         dX=(outs[i]["dX"][m] if outs else d["dX"][m]), workspace=self.ws)
 
 

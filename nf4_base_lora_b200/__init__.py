@@ -200,14 +200,21 @@ def nf4_dequantize(w: NF4Tensor, out: Optional[torch.Tensor] = None) -> torch.Te
 
 def qlora_linear_fwd(w: NF4Tensor, A: torch.Tensor, B: torch.Tensor, scaling: float, X: torch.Tensor,
                      save_t: bool = True, Y: Optional[torch.Tensor] = None,
-                     workspace: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+                     workspace: Optional[torch.Tensor] = None,
+                     T: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Y = X W_hat^T + s (X A^T) B^T.  Returns (Y, T) with T = s X A^T in
-    fp32 (or None when save_t is False), for reuse by the backward."""
+    fp32 (or None when save_t is False), for reuse by the backward; T may be
+    given as a contiguous float32 [M, r] output buffer."""
     _bf16(A, "A"), _bf16(B, "B"), _bf16(X, "X")
     r = A.shape[0]
     M = X.shape[0]
     Y = Y if Y is not None else torch.empty((M, w.d_out), dtype=torch.bfloat16, device=X.device)
-    T = torch.empty((M, r), dtype=torch.float32, device=X.device) if save_t else None
+    if not save_t:
+        T = None
+    elif T is None:
+        T = torch.empty((M, r), dtype=torch.float32, device=X.device)
+    elif T.dtype != torch.float32 or not T.is_contiguous() or tuple(T.shape) != (M, r):
+        raise ValueError("T must be a contiguous float32 [M, r] tensor")
     need = qlora_fwd_workspace_bytes(M, w.d_out, w.d_in, r)
     ws = workspace if workspace is not None else _workspace(need, X.device)
     _check(lib.qlora_linear_fwd(ctypes.byref(w.struct), _ptr(A), _ptr(B), r, ctypes.c_float(scaling),

@@ -10,8 +10,8 @@
 // With at most 16 tokens the layer is a streamed matrix-vector product: per
 // weight the GPU reads 4.127 bits and decodes them, and the 16 dot products
 // are a small tail.  One thread (TMA) streams the CTA's packed codes into
-// shared memory; each thread then decodes its slice with the 16-level table,
-// restores bf16(level[code] * s_b) in registers and hands the pairs to the
+// shared memory; each thread then decodes its slice with a register-held
+// codebook (csrc/decode.cuh), restores bf16(level[code] * s_b) and hands the pairs to the
 // tensor instruction as its A fragment (16 weight rows x 16 k; the activations
 // are the B fragment, 16 k x 8 tokens).  A decoded weight never goes back to
 // memory.
@@ -27,10 +27,10 @@
 // along grid.z.  Inside a CTA the two warps of a row group add their fp32
 // partials through shared memory; every CTA of rank > 0 then pushes its
 // partial tile into a slot of rank 0 (distributed shared memory) and arrives
-// on an mbarrier there; rank 0 adds the slots in rank order, adds the rank-r
-// extension once the kernel that produced T2 has finished (programmatic
-// dependent launch), and writes bf16.  The summation order is fixed, so the
-// result is the same on every run.
+// on an mbarrier there; rank 0 adds the slots in rank order and writes bf16.
+// The rank-r extension, once the kernel that produced T2 has finished
+// (programmatic dependent launch), is shared out among the ranks.  The
+// summation order is fixed, so the result is the same on every run.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -93,26 +93,10 @@ constexpr int kFwdMaxSplit = kMaxSplit;      // partial-tile slots of rank 0: kF
 constexpr int kFwdSmemV2 =
     1024 + 4 * kFwdQuadBytes + (kFwdMaxSplit - 1) * kPartFloats * 4 + 8 * 8 * 32 * 4 + kTok * kFwdTokStride * 2;
 
-// Bytes 2h and 2h + 1 of word w (4 weights) to two bf16 pairs, with the level
-// table read by byte offset (code * 4) straight from the shifted word.
-__device__ __forceinline__ void decode_quarter(uint32_t w, int h, float s, const uint8_t* lut_bytes, uint32_t& p0,
-                                               uint32_t& p1) {
-    const uint32_t hi_off = (w >> 2) & 0x3C3C3C3Cu;  // 4 * high nibble of each byte
-    const uint32_t lo_off = (w << 2) & 0x3C3C3C3Cu;  // 4 * low nibble of each byte
-    const uint32_t sel0 = 0x4440u + 2 * h, sel1 = 0x4441u + 2 * h;  // byte 2h / 2h + 1, zero-extended
-    const float e0 = *reinterpret_cast<const float*>(lut_bytes + __byte_perm(hi_off, 0u, sel0));
-    const float o0 = *reinterpret_cast<const float*>(lut_bytes + __byte_perm(lo_off, 0u, sel0));
-    const float e1 = *reinterpret_cast<const float*>(lut_bytes + __byte_perm(hi_off, 0u, sel1));
-    const float o1 = *reinterpret_cast<const float*>(lut_bytes + __byte_perm(lo_off, 0u, sel1));
-    p0 = pack_bf16x2(__fmul_rn(e0, s), __fmul_rn(o0, s));
-    p1 = pack_bf16x2(__fmul_rn(e1, s), __fmul_rn(o1, s));
-}
-
 // Registers capped at 96 (48K of the SM's 64K) so that the CTAs of the kernel
 // producing T2, which this one overlaps, keep room on the same SM.
 __global__ void __maxnreg__(96) k_few_fwd(const __grid_constant__ CUtensorMap map_codes, const FewArgs a) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
-    __shared__ __align__(16) float s_lut[16];
     __shared__ uint64_t bar_part, bar_q[4];
     __shared__ int s_abort;
     // [codes: 4 quads x 128 rows x 128 B, 128-byte swizzle][partial slots][warp reduction][activations]
@@ -150,7 +134,6 @@ __global__ void __maxnreg__(96) k_few_fwd(const __grid_constant__ CUtensorMap ma
             issue_codes(kb0, nq_first);
         }
     }
-    if (tid < 16) s_lut[tid] = nf4_level(tid);
 
     const int lr = 16 * rgp + g;  // local row of nA (nB = nA + 8 is local row lr + 8)
     const int nA = row0 + lr, nB = nA + 8;
@@ -161,7 +144,6 @@ __global__ void __maxnreg__(96) k_few_fwd(const __grid_constant__ CUtensorMap ma
     __syncthreads();
     cluster_arrive_relaxed();  // barriers initialised (made visible by the init fence)
     const float mu = __ldg(a.scale_mean);
-    const uint8_t* lut_bytes = reinterpret_cast<const uint8_t*>(s_lut);
     volatile int* abort_flag = &s_abort;
 
     int seg_i = 0, issued_seg = 0, issued_nq = kb0 < kb1 ? nq_first : 0;
@@ -232,11 +214,14 @@ __global__ void __maxnreg__(96) k_few_fwd(const __grid_constant__ CUtensorMap ma
             const uint16_t* x8 = x0 + 8 * kFwdTokStride;
             const uint32_t wA[8] = {cA0.x, cA0.y, cA0.z, cA0.w, cA1.x, cA1.y, cA1.z, cA1.w};
             const uint32_t wB[8] = {cB0.x, cB0.y, cB0.z, cB0.w, cB1.x, cB1.y, cB1.z, cB1.w};
+            uint32_t PA[4], HA[4], PB[4], HB[4];  // register codebooks of the two rows
+            nf4_table(sA, PA, HA);
+            nf4_table(sB, PB, HB);
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
                 uint32_t a0, a1, a2, a3;  // rows g (a0, a2) and g + 8 (a1, a3), k = 4c + {0,1} / {2,3}
-                decode_quarter(wA[c >> 1], c & 1, sA, lut_bytes, a0, a2);
-                decode_quarter(wB[c >> 1], c & 1, sB, lut_bytes, a1, a3);
+                nf4_lookup4(wA[c >> 1] >> (16 * (c & 1)), PA, HA, a0, a2);
+                nf4_lookup4(wB[c >> 1] >> (16 * (c & 1)), PB, HB, a1, a3);
                 const uint2 xb = *reinterpret_cast<const uint2*>(x0 + 4 * c);
                 mma_16816(acc0, a0, a1, a2, a3, xb.x, xb.y);
                 if (two_halves) {
@@ -251,14 +236,16 @@ __global__ void __maxnreg__(96) k_few_fwd(const __grid_constant__ CUtensorMap ma
         for (int j = 0; j < issued_nq; ++j) mbar_drain(&bar_q[j], issued_seg & 1);
     }
 
-    // rank-r extension on rank 0: [B | B] rows of this CTA against T2, once the
-    // kernel producing T2 has finished (programmatic dependent launch)
-    if (rank == 0 && a.ext_act != nullptr) {
+    // rank-r extension: [B | B] rows of this CTA against T2, once the kernel
+    // producing T2 has finished (programmatic dependent launch).  Its 16-wide
+    // chunks are dealt round-robin to the ranks of the cluster (and to the two
+    // warps of a row group), which add them to the partials they push.
+    if (a.ext_act != nullptr) {
         if (a.pdl) wait_prerequisites();
         const int nchunks = 2 * a.r64 / 16;
         const uint16_t* bA = a.ext_w + static_cast<int64_t>(nA) * a.r;
         const uint16_t* bB = a.ext_w + static_cast<int64_t>(nB) * a.r;
-        for (int ch = qs; ch < nchunks; ch += 2) {
+        for (int ch = rank + splits * qs; ch < nchunks; ch += 2 * splits) {
             const int j0 = ch * 16;
             const int jj = (j0 % a.r64) + 2 * q;  // column of B (same in both halves of T2)
             const bool lo_ok = jj < a.r, hi_ok = jj + 8 < a.r;

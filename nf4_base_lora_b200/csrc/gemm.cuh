@@ -47,6 +47,7 @@
 #include <cstdint>
 
 #include "common.cuh"
+#include "decode.cuh"
 #include "nf4_levels.cuh"
 
 namespace nf4lora {
@@ -176,38 +177,20 @@ __device__ __forceinline__ void decode_unit(const uint8_t* src, float s, uint8_t
     }
 }
 
-// The same decode with the codebook held in registers: the 16 scaled levels
-// bf16(level_j * s) are formed once per unit and split into byte planes
-// (P: low bytes, H: high bytes, four entries per register); each group of
-// four codes is then looked up with byte permutes, entries 0-7 and 8-15
-// separately and merged on bit 3 of the code.  No shared-memory reads, so the
-// shared-memory port stays free for TMA, the decoded stores and the MMAs.
+// The same decode with the codebook held in registers (csrc/decode.cuh): no
+// shared-memory reads, so the shared-memory port stays free for TMA, the
+// decoded stores and the MMAs.
 __device__ __forceinline__ void decode_unit_reg(const uint8_t* src, float s, uint8_t* dst_row, int swz) {
     uint32_t P[4], H[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint32_t t0 = pack_bf16x2(__fmul_rn(nf4_level(4 * i), s), __fmul_rn(nf4_level(4 * i + 1), s));
-        const uint32_t t1 = pack_bf16x2(__fmul_rn(nf4_level(4 * i + 2), s), __fmul_rn(nf4_level(4 * i + 3), s));
-        P[i] = __byte_perm(t0, t1, 0x6420);
-        H[i] = __byte_perm(t0, t1, 0x7531);
-    }
+    nf4_table(s, P, H);
     const uint4 c0 = *reinterpret_cast<const uint4*>(src);
     const uint4 c1 = *reinterpret_cast<const uint4*>(src + 16);
     const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
         uint32_t o[4];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            // nibbles of xs, low first: e1 e0 e3 e2 (byte b = e_2b << 4 | e_2b+1)
-            const uint32_t xs = words[j] >> (16 * h);
-            const uint32_t sel = xs & 0x7777u;                          // index within 0-7 / 8-15
-            const uint32_t pick = ((xs >> 1) & 0x4444u) | 0x3210u;      // byte i from the 8-15 half if bit 3
-            const uint32_t lo = __byte_perm(__byte_perm(P[0], P[1], sel), __byte_perm(P[2], P[3], sel), pick);
-            const uint32_t hi = __byte_perm(__byte_perm(H[0], H[1], sel), __byte_perm(H[2], H[3], sel), pick);
-            o[2 * h] = __byte_perm(lo, hi, 0x4051);      // (e0, e1): lo.b1 hi.b1 lo.b0 hi.b0
-            o[2 * h + 1] = __byte_perm(lo, hi, 0x6273);  // (e2, e3): lo.b3 hi.b3 lo.b2 hi.b2
-        }
+        nf4_lookup4(words[j], P, H, o[0], o[1]);
+        nf4_lookup4(words[j] >> 16, P, H, o[2], o[3]);
         *reinterpret_cast<uint4*>(dst_row + ((j ^ swz) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
     }
 }
