@@ -173,7 +173,7 @@ __global__ void __launch_bounds__(kDownThreads) k_few_down(const uint16_t* __res
 // up to 8 slices of d_out, the slices of one column group form a cluster, the
 // slice of dY and of B (up to 512 rows at a time) comes in by asynchronous
 // copies issued at once, and the dependent launch is released right after.
-constexpr int kVBatch = 512;                    // rows of B per staged slice
+constexpr int kVBatch = 256;                    // rows of B per staged slice (small enough to share an SM with the dX kernel)
 constexpr int kVYStride = kVBatch + 8;          // dY staging row stride (elements)
 constexpr int kVBStride = 24;                   // B staging row stride (elements): 48 bytes, conflict-free ldmatrix
 constexpr int kVSmem = kMaxFewTokens * kVYStride * 2 + kVBatch * kVBStride * 2 + 4 * kMaxFewTokens * 16 * 4;

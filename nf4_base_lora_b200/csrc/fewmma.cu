@@ -367,7 +367,7 @@ __device__ __forceinline__ void dx_chunk_mma(float (&acc)[4][2][4], uint32_t til
     }
 }
 
-__global__ void __maxnreg__(128) k_few_dx(const __grid_constant__ CUtensorMap map_codes, const FewArgs a) {
+__global__ void __maxnreg__(112) k_few_dx(const __grid_constant__ CUtensorMap map_codes, const FewArgs a) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     __shared__ uint64_t bar_part, bar_c[4];
     __shared__ int s_abort;
@@ -485,10 +485,11 @@ __global__ void __maxnreg__(128) k_few_dx(const __grid_constant__ CUtensorMap ma
         for (int b = 0; b < issued_boxes; ++b) mbar_drain(&bar_c[b], issued_seg & 1);
     }
 
-    // rank-r extension on rank 0: the rows of [A ; A] as 32-row chunks through
-    // the same tiles, against V2 staged in place of dY, once the kernel
-    // producing V2 has finished
-    if (rank == 0 && a.ext_act != nullptr) {
+    // rank-r extension: the rows of [A ; A] as 32-row chunks through the same
+    // tiles, against V2 staged in place of dY, once the kernel producing V2
+    // has finished; the chunks are dealt round-robin to the ranks, which add
+    // them to the partials they push
+    if (a.ext_act != nullptr) {
         if (a.pdl) wait_prerequisites();
         const int vstride = 2 * a.r64 + 8;
         __syncthreads();  // dY staging and tiles are free
@@ -499,7 +500,7 @@ __global__ void __maxnreg__(128) k_few_dx(const __grid_constant__ CUtensorMap ma
             *reinterpret_cast<uint2*>(sY + t * vstride + 4 * pc) = v;
         }
         __syncthreads();
-        for (int c = rw; c < 2 * a.r64 / 32; c += 8) {
+        for (int c = rank + splits * rw; c < 2 * a.r64 / 32; c += 8 * splits) {
             const int j = (32 * c + lane) % a.r64;  // row of A (the same in both halves)
             uint4* trow = reinterpret_cast<uint4*>(my_tile + lane * kDxTileStride);
             const uint4* arow = reinterpret_cast<const uint4*>(a.ext_w + static_cast<int64_t>(j) * K + 64 * blk);
