@@ -179,8 +179,10 @@ int nf4_dequantize(const nf4_tensor* w, uint16_t* W_hat, void* stream);
  * arrays hi = bf16(T), lo = bf16(T - hi) (about 16 significant bits), so the
  * adapter branch is not limited to bfloat16 precision ([QP] §6.3: the adapter
  * dtype may be wider than the base compute dtype).
- * Requirements: M >= 1, 1 <= r <= 256, r % 8 == 0, d_in % 64 == 0,
+ * Requirements: 0 <= M < 2^31, 1 <= r <= 256, r % 8 == 0, d_in % 64 == 0,
  * d_out % 8 == 0, ws >= qlora_fwd_workspace_bytes(M, d_out, d_in, r).
+ * M = 0 (an empty batch) does nothing and returns NF4_OK; X, Y and T_saved
+ * may then be NULL.
  */
 int qlora_linear_fwd(const nf4_tensor* w, const uint16_t* A, const uint16_t* B, int r,
                      float scaling, const uint16_t* X, int64_t M, uint16_t* Y,
@@ -201,6 +203,9 @@ int qlora_linear_fwd(const nf4_tensor* w, const uint16_t* A, const uint16_t* B, 
  * values already in those buffers (gradient accumulation, [QP] §6.4) instead
  * of overwriting them.  Requirements as for the forward, and
  * ws >= qlora_bwd_workspace_bytes(M, d_out, d_in, r).
+ * M = 0 (an empty batch): the gradients of an empty sum are zero, so dA and
+ * dB are set to zero (left as they are with accumulate_grads = 1) and nothing
+ * else happens; dY, X, T_saved and dX may then be NULL.
  */
 int qlora_linear_bwd(const nf4_tensor* w, const uint16_t* A, const uint16_t* B, int r,
                      float scaling, const uint16_t* X, const float* T_saved,

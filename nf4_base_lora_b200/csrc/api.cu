@@ -86,7 +86,7 @@ int check_layer_common(const nf4_tensor* w, const uint16_t* A, const uint16_t* B
     if (r < 1 || r > 256) return fail(NF4_ERR_INVALID_ARG, "r = %d outside [1, 256]", r);
     if (r % 8 != 0) return fail(NF4_ERR_UNSUPPORTED_SHAPE, "r = %d must be a multiple of 8", r);
     if (!std::isfinite(scaling)) return fail(NF4_ERR_INVALID_ARG, "scaling is not finite");
-    if (M < 1 || M >= (int64_t(1) << 31)) return fail(NF4_ERR_INVALID_ARG, "M = %lld outside [1, 2^31)", (long long)M);
+    if (M < 0 || M >= (int64_t(1) << 31)) return fail(NF4_ERR_INVALID_ARG, "M = %lld outside [0, 2^31)", (long long)M);
     if (!A || !B) return fail(NF4_ERR_INVALID_ARG, "A or B is NULL");
     if (!aligned16(A) || !aligned16(B)) return fail(NF4_ERR_MISALIGNED, "A or B not 16-byte aligned");
     return NF4_OK;
@@ -189,6 +189,7 @@ int qlora_linear_fwd(const nf4_tensor* w, const uint16_t* A, const uint16_t* B, 
                      void* stream) {
     int rc = check_layer_common(w, A, B, r, scaling, M);
     if (rc) return rc;
+    if (M == 0) return ok();  // an empty batch
     if (!X || !Y) return fail(NF4_ERR_INVALID_ARG, "X or Y is NULL");
     if (!aligned16(X) || !aligned16(Y) || (T_saved && !aligned16(T_saved)))
         return fail(NF4_ERR_MISALIGNED, "X, Y or T_saved not 16-byte aligned");
@@ -210,13 +211,25 @@ int qlora_linear_bwd(const nf4_tensor* w, const uint16_t* A, const uint16_t* B, 
                      uint16_t* dA, uint16_t* dB, int accumulate_grads, void* ws, size_t ws_bytes, void* stream) {
     int rc = check_layer_common(w, A, B, r, scaling, M);
     if (rc) return rc;
+    if (accumulate_grads != 0 && accumulate_grads != 1) return fail(NF4_ERR_INVALID_ARG, "accumulate_grads must be 0 or 1");
+    if (M == 0) {
+        // an empty batch: zero gradients for the adapters, nothing else
+        if (accumulate_grads || (!dA && !dB)) return ok();
+        if ((dA && !aligned16(dA)) || (dB && !aligned16(dB)))
+            return fail(NF4_ERR_MISALIGNED, "dA or dB not 16-byte aligned");
+        const cudaStream_t st = static_cast<cudaStream_t>(stream);
+        if (dA && cudaMemsetAsync(dA, 0, static_cast<size_t>(r) * w->d_in * 2, st) != cudaSuccess)
+            return fail(NF4_ERR_CUDA, "qlora_linear_bwd: clearing dA failed");
+        if (dB && cudaMemsetAsync(dB, 0, static_cast<size_t>(w->d_out) * r * 2, st) != cudaSuccess)
+            return fail(NF4_ERR_CUDA, "qlora_linear_bwd: clearing dB failed");
+        return ok();
+    }
     if (!dY) return fail(NF4_ERR_INVALID_ARG, "dY is NULL");
     const bool need_x = dA != nullptr || (dB != nullptr && T_saved == nullptr);
     if (need_x && !X) return fail(NF4_ERR_INVALID_ARG, "X is NULL but dA, or dB without T_saved, is requested");
     if (!aligned16(dY) || (X && !aligned16(X)) || (T_saved && !aligned16(T_saved)) || (dX && !aligned16(dX)) ||
         (dA && !aligned16(dA)) || (dB && !aligned16(dB)))
         return fail(NF4_ERR_MISALIGNED, "an array argument is not 16-byte aligned");
-    if (accumulate_grads != 0 && accumulate_grads != 1) return fail(NF4_ERR_INVALID_ARG, "accumulate_grads must be 0 or 1");
     if (!dX && !dA && !dB) return ok();
     rc = check_ws(ws, ws_bytes, bwd_workspace_bytes(M, w->d_out, w->d_in, r, kPlanSMs));
     if (rc) return rc;

@@ -96,8 +96,14 @@ def test_host_validation_without_device(nf):
     assert L.qlora_linear_fwd(ctypes.byref(s), A, B, 8, ctypes.c_float(float("inf")), X, 16, Y, None, ws,
                               1 << 30, None) == -1
     # M out of range
-    assert L.qlora_linear_fwd(ctypes.byref(s), A, B, 8, f, X, 0, Y, None, ws, 1 << 30, None) == -1
-    assert b"M = 0" in L.nf4lora_last_error_string()
+    assert L.qlora_linear_fwd(ctypes.byref(s), A, B, 8, f, X, -1, Y, None, ws, 1 << 30, None) == -1
+    assert b"M = -1" in L.nf4lora_last_error_string()
+    assert L.qlora_linear_fwd(ctypes.byref(s), A, B, 8, f, X, 1 << 31, Y, None, ws, 1 << 30, None) == -1
+    # an empty batch is a no-op (no device access: X, Y and the workspace may be NULL)
+    assert L.qlora_linear_fwd(ctypes.byref(s), A, B, 8, f, None, 0, None, None, None, 0, None) == 0
+    # ... and so is its backward when the gradients accumulate
+    assert L.qlora_linear_bwd(ctypes.byref(s), A, B, 8, f, None, None, None, 0, None, P(1 << 29), P(1 << 28), 1,
+                              None, 0, None) == 0
     # backward: dA needs X
     assert L.qlora_linear_bwd(ctypes.byref(s), A, B, 8, f, None, None, Y, 16, None, P(1 << 29), None, 0, ws,
                               1 << 30, None) == -1

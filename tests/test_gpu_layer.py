@@ -41,6 +41,8 @@ CASES = [
     (384, 1024, 200, 192),
     (4736, 4800, 2000, 16),   # enough tiles for the 256-row CTA tile; ragged tokens
     (9472, 1408, 5, 16),      # few tokens: two splits of 11 blocks (a ragged block quad)
+    (256, 256, 7, 256),       # largest rank, few tokens
+    (384, 256, 40, 256),      # largest rank, many tokens
 ]
 
 
@@ -117,3 +119,23 @@ def test_layer_is_deterministic(nf):
     for o in outs[1:]:
         for a, b in zip(outs[0], o):
             assert torch.equal(a, b)
+
+
+def test_empty_batch(nf):
+    """M = 0: the forward does nothing; the backward's adapter gradients are
+    zero (the gradient of an empty sum), or left as they are when accumulating."""
+    c, W_hat, w, dev = setup(nf, 256, 256, 1, 16)
+    X0 = dev["X"][:0]
+    Y0 = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
+    Y, T = nf.qlora_linear_fwd(w, dev["A"], dev["B"], c.scaling, X0, Y=Y0)
+    assert Y.shape == (0, 256) and T.shape == (0, 16)
+    dA = torch.full((16, 256), 3.0, dtype=torch.bfloat16, device="cuda")
+    dB = torch.full((256, 16), 3.0, dtype=torch.bfloat16, device="cuda")
+    dY0 = dev["dY"][:0]
+    nf.qlora_linear_bwd(w, dev["A"], dev["B"], c.scaling, X0, None, dY0, dA=dA, dB=dB, accumulate=True)
+    torch.cuda.synchronize()
+    assert torch.all(dA == 3.0) and torch.all(dB == 3.0)
+    nf.qlora_linear_bwd(w, dev["A"], dev["B"], c.scaling, X0, None, dY0, dA=dA, dB=dB, accumulate=False)
+    torch.cuda.synchronize()
+    nf.device_status()
+    assert torch.all(dA == 0) and torch.all(dB == 0)
