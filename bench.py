@@ -13,9 +13,12 @@ weight from HBM.  Steps are replayed from CUDA graphs; the library's own
 launch tracing times the dominant kernel on the stream it runs on.
 
 Rank 0 prints ONE JSON line.  With N > 1 (torchrun, one process per GPU)
-every rank runs the same per-GPU workload on its own data (weak scaling; the
-path has no exchange step for this workload) and the time is the max over
-ranks.  ``--impl reference`` times the CPU oracle (the plain fp64 statement
+every rank runs the same per-GPU workload on its own data (weak scaling) and
+the time is the max over ranks.  A forward + input-gradient workload has no
+exchange step (independent replicas); a full-backward workload is a
+data-parallel training step, so after each step the ranks sum their adapter
+gradients dA, dB with one all-reduce (``nf4_base_lora_b200.dp``), inside the
+timed region.  ``--impl reference`` times the CPU oracle (the plain fp64 statement
 of the method) on the host on a bounded sample of the same workload.
 """
 from __future__ import annotations
@@ -283,9 +286,12 @@ class GpuWorkload:
     def __init__(self, nf, wl, device, copies):
         self.nf, self.wl, self.device = nf, wl, device
         self.mods = []
+        self.fp32 = []  # the fp32 weights, kept where the workload times their encoding
         for i, mod in enumerate(wl.modules):
             W = torch.from_numpy(workloads.weight(mod.d_out, mod.d_in, wl.sigma, wl.outliers, i)).to(device)
             enc = nf.nf4_quantize(W)
+            if wl.quantize_timed:
+                self.fp32.append(W)
             del W
             encs = [enc] + [nf.NF4Tensor(mod.d_out, mod.d_in, device, buffer=enc.buffer.clone())
                             for _ in range(copies - 1)]
@@ -343,6 +349,74 @@ def dominant_kernel_stats(records, names):
     return dom, stats
 
 
+def quantize_bytes(d_out, d_in):
+    """Algorithmic bytes of one encoding: the fp32 weight read once, the
+    packed codes, int8 scale codes, fp32 group scales and mean written once."""
+    n = d_out * d_in
+    nb = n // 64
+    return 4 * n + n // 2 + nb + 4 * ((nb + 255) // 256) + 4
+
+
+def time_quantize(nf, gw, args, stream, device, world, hbm_peak, peak_src):
+    """Encoding of every module's fp32 weight through nf4_quantize, timed on
+    its own: K passes over all modules after W warm-up passes (the fp32
+    weights total more than 4x L2, so every pass reads them from HBM)."""
+    import torch.distributed as dist
+    wl = gw.wl
+    outs = [nf.NF4Tensor(m.d_out, m.d_in, device) for m in wl.modules]
+    ws = torch.empty(max(nf.nf4_quantize_workspace_bytes(m.d_out, m.d_in) for m in wl.modules),
+                     dtype=torch.uint8, device=device)
+    per_pass = sum(quantize_bytes(m.d_out, m.d_in) for m in wl.modules)
+    weights = sum(m.d_out * m.d_in for m in wl.modules)
+
+    def one_pass():
+        with torch.cuda.stream(stream):
+            for W, enc in zip(gw.fp32, outs):
+                nf.nf4_quantize(W, out=enc, workspace=ws)
+
+    for _ in range(args.warmup):
+        one_pass()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    passes = max(3, min(args.steps, 50))
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(passes):
+        one_pass()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / passes
+    if world > 1:
+        from nf4_base_lora_b200 import dp
+        ms = dp.max_over_ranks(ms, device)
+    # the encode kernel's own device time (library tracing, one more pass)
+    nf.trace_start(16 * len(wl.modules) + 64)
+    one_pass()
+    torch.cuda.synchronize()
+    records = nf.trace_records()
+    nf.trace_stop()
+    per_kernel = {}
+    for name, kms in records:
+        per_kernel.setdefault(name, []).append(kms)
+    enc_ms = sum(per_kernel.get("nf4_encode", [0.0]))
+    enc_bytes = sum(4 * m.d_out * m.d_in + m.d_out * m.d_in // 2 for m in wl.modules)
+    value = world * per_pass / (ms * 1e-3) / 1e9
+    out = {"ms_per_pass": ms, "passes": passes, "value": value, "unit": "GB/s",
+           "weights_per_pass": weights, "bytes_per_pass": per_pass,
+           "algorithmic": "per module 4n + n/2 + n/64 + 4*ceil(n/16384) + 4 bytes (n weights)",
+           "frac": value / world / hbm_peak,
+           "kernels": {k: {"launches": len(v), "avg_us": sum(v) / len(v) * 1e3} for k, v in sorted(per_kernel.items())}}
+    if enc_ms > 0:
+        achieved = enc_bytes / (enc_ms * 1e-3) / 1e9
+        out["roofline"] = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                           "frac": achieved / hbm_peak, "kernel": "nf4_encode",
+                           "algorithmic": "4n read + n/2 written per launch (fp32 weight in, packed codes out)",
+                           "peak_source": peak_src + " (hbm_gbs)"}
+    return out
+
+
 def run_ours(args, wl):
     import torch.distributed as dist
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -385,6 +459,12 @@ def run_ours(args, wl):
         launches_per_step = nf.trace_count() / cycle
         nf.trace_stop()
 
+    # data-parallel exchange of the adapter gradients (full backward, N > 1)
+    exchange = None
+    if world > 1 and wl.backward != "dx":
+        from nf4_base_lora_b200 import dp
+        exchange = dp.LoraGradExchange([t for d in gw.mods for t in (d["dA"], d["dB"])])
+
     def run_steps(k, base):
         with torch.cuda.stream(stream):
             for s in range(k):
@@ -392,11 +472,15 @@ def run_ours(args, wl):
                     graphs[(base + s) % cycle].replay()
                 else:
                     gw.step(((base + s) % cycle) * len(plan))
+                if exchange is not None:
+                    exchange()
 
     def run_steps_eager(k, base):
         with torch.cuda.stream(stream):
             for s in range(k):
                 gw.step(((base + s) % cycle) * len(plan))
+                if exchange is not None:
+                    exchange()
 
     if not graphs:
         nf.trace_start(len(plan) * 16 + 64)
@@ -426,9 +510,8 @@ def run_ours(args, wl):
     clocks = sampler.stop()
     ms = start.elapsed_time(stop)
     if world > 1:
-        t = torch.tensor([ms], device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+        from nf4_base_lora_b200 import dp
+        ms = dp.max_over_ranks(ms, device)
     ms_per_step = ms / args.steps
     value = world * step_bytes / (ms_per_step * 1e-3) / 1e9
     tflops = world * step_flops / (ms_per_step * 1e-3) / 1e12
@@ -476,6 +559,7 @@ def run_ours(args, wl):
                         "algorithmic": "2*M*K*N + 2*M*r*(K+N) flops per launch",
                         "peak_source": peak_src + " (bf16_tflops_sustained)"}
     kernel_table = {k: {"launches": v[0], "avg_us": v[1] / v[0] * 1e3} for k, v in sorted(kstats.items())}
+    quantize = time_quantize(nf, gw, args, stream, device, world, hbm_peak, peak_src) if gw.fp32 else None
 
     # end to end through the public API: pinned host inputs -> device -> layer -> host
     e2e_steps = max(3, min(args.steps, 200))
@@ -499,6 +583,8 @@ def run_ours(args, wl):
                 devX[i].copy_(hostX[i], non_blocking=True)
                 devdY[i].copy_(hostdY[i], non_blocking=True)
             gw.step((s % cycle) * len(plan), X=devX, dY=devdY, outs=outs)
+            if exchange is not None:
+                exchange()
             for i in range(len(gw.mods)):
                 for m in wl.tokens:
                     hostY[i][m].copy_(outs[i]["Y"][m], non_blocking=True)
@@ -518,9 +604,8 @@ def run_ours(args, wl):
     torch.cuda.synchronize()
     ems = e0.elapsed_time(e1)
     if world > 1:
-        t = torch.tensor([ems], device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ems = float(t.item())
+        from nf4_base_lora_b200 import dp
+        ems = dp.max_over_ranks(ems, device)
     e2e_value = world * step_bytes / (ems / e2e_steps * 1e-3) / 1e9
 
     cpu_baseline = None
@@ -542,7 +627,10 @@ def run_ours(args, wl):
             "data": "synthetic (seeded N(0, sigma) weights with 0.1% x10 outliers, N(0,1) activations)",
             "config": dict(workload_config(wl), l2_flush="rotating %d encoded weight copies (%.0f MB > 4x L2)"
                            % (copies, copies * wbytes / 1e6) if copies > 1 else "weights larger than 4x L2",
-                           graphs=bool(graphs)),
+                           graphs=bool(graphs),
+                           parallelism="dp%d%s" % (world, "" if world == 1 else
+                                                   " (all-reduce of dA, dB per step)" if exchange is not None
+                                                   else " (independent replicas: no exchange step)")),
             "tflops": tflops,
             "roofline": roofline,
             "cpu_baseline": cpu_baseline,
@@ -551,6 +639,8 @@ def run_ours(args, wl):
             "gpu_launches": int(round(launches_per_step * args.steps)) if launches_per_step else 0,
             "kernels": kernel_table,
             "clocks": clocks}
+    if quantize is not None:
+        line["quantize"] = quantize
     print(json.dumps(line), flush=True)
 
 

@@ -165,13 +165,16 @@ class NF4Tensor:
 
 
 # ---------------------------------------------------------------- entry points
-def nf4_quantize(W: torch.Tensor, out: Optional[NF4Tensor] = None) -> NF4Tensor:
-    """Encode fp32 W [d_out, d_in] (CUDA) to NF4 + double-quantised scales."""
+def nf4_quantize(W: torch.Tensor, out: Optional[NF4Tensor] = None,
+                 workspace: Optional[torch.Tensor] = None) -> NF4Tensor:
+    """Encode fp32 W [d_out, d_in] (CUDA) to NF4 + double-quantised scales.
+    `workspace` (uint8, >= nf4_quantize_workspace_bytes) is allocated when
+    not given."""
     if W.dtype != torch.float32 or not W.is_cuda or not W.is_contiguous() or W.dim() != 2:
         raise ValueError("W must be a contiguous 2-D float32 CUDA tensor")
     d_out, d_in = W.shape
     out = out if out is not None else NF4Tensor(d_out, d_in, W.device)
-    ws = _workspace(nf4_quantize_workspace_bytes(d_out, d_in), W.device)
+    ws = workspace if workspace is not None else _workspace(nf4_quantize_workspace_bytes(d_out, d_in), W.device)
     _check(lib.nf4_quantize(_ptr(W), d_out, d_in, ctypes.byref(out.struct), _ptr(ws),
                             0 if ws is None else ws.numel(), _stream()))
     return out

@@ -138,6 +138,26 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
+// Bulk prefetch of a global range into L2 (no data comes to the SM): address
+// 16-byte aligned, size a multiple of 16 bytes.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes)
+                 : "memory");
+}
+
+// ------------------------------------------------------------------ programmatic dependent launch
+// wait: block until the preceding kernel of the stream has completed and its
+// writes are visible (returns at once when the kernel was launched without
+// the programmatic-serialisation attribute).  launch_dependents: the next
+// kernel of the stream, if launched with that attribute, may start once every
+// CTA of this grid has executed it (or exited).
+__device__ __forceinline__ void pdl_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ tcgen05
 // Tensor memory: 128 lanes x 512 columns of 32-bit cells per SM.  An address
 // is (lane << 16) | column.

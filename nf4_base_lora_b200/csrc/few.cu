@@ -7,6 +7,14 @@
 // GEMM streams and decodes the weight while these run, and waits for them only
 // before its extension steps.  The contraction is split over a thread-block
 // cluster and summed through distributed shared memory in rank order.
+//
+// Both are themselves programmatic dependents of the kernel before them (the
+// previous fused GEMM releases its dependents when it starts): their CTAs
+// start early, stage the rows of the LoRA factor (a parameter, never written
+// by the preceding kernel), then wait for that kernel to finish before they
+// read the activations or gradients, which it may have produced.  They release
+// their own dependent only after that wait, so the fused GEMM that follows may
+// read the same activations before its own wait.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -23,11 +31,6 @@ namespace {
 
 constexpr int kMaxFewTokens = 16;
 
-__device__ __forceinline__ void allow_dependents() {
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
-
 __device__ __forceinline__ void store_split(uint16_t* dst_hi, uint16_t* dst_lo, float v) {
     const __nv_bfloat16 hi = __float2bfloat16_rn(v);
     const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
@@ -39,10 +42,11 @@ __device__ __forceinline__ void store_split(uint16_t* dst_hi, uint16_t* dst_lo, 
 // (m16n8k16: A operand = X, 16 tokens x 16 k; B operand = 8 rows of A).
 // CTA (x, z) computes columns 16x .. 16x + 15 of T over the z-th of up to 8
 // slices of K; the slices of one column group form a cluster.  A CTA copies
-// its part of X and its 16 rows of A (up to 512 k at a time) into shared
-// memory with asynchronous copies issued all at once, and releases the
-// dependent launch as soon as they are requested, so that these loads queue
-// ahead of the dependent kernel's.  The CTAs are small (four warps, 37 KB of
+// its 16 rows of A and its part of X (up to 512 k at a time) into shared
+// memory with asynchronous copies issued all at once (A before the wait for
+// the preceding kernel, X after it), and releases the dependent launch as
+// soon as they are requested, so that these loads queue ahead of the
+// dependent kernel's.  The CTAs are small (four warps, 37 KB of
 // shared memory) and many (one per SM for r = 64), so that the loads are
 // spread over SMs and the CTAs share SMs with the dependent kernel's.  Warp w
 // takes every fourth 16-wide chunk; partials are added in a fixed order: the
@@ -88,27 +92,27 @@ __global__ void __launch_bounds__(kDownThreads) k_few_down(const uint16_t* __res
     const int k_end = k_begin + 64 * (per + (rank < extra ? 1 : 0));
     float acc[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
 
-    bool released = false;
+    bool first = true;
     for (int k0 = k_begin; k0 < k_end; k0 += kDownBatch) {
         const int kn = min(kDownBatch, k_end - k0);  // a multiple of 64
         const int pieces = kn / 8;                   // 16-byte pieces per row
         __syncthreads();                             // the previous slice is no longer read
-        for (int i = tid; i < 2 * kMaxFewTokens * pieces; i += kDownThreads) {
-            const int row = i / pieces, pc = i - row * pieces;
-            if (row < kMaxFewTokens) {
-                uint16_t* dst = sX + row * kDownStride + pc * 8;
-                if (row < M) cp_async16(dst, X + static_cast<int64_t>(row) * K + k0 + pc * 8);
-                else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
-            } else {
-                const int j = j0 + row - kMaxFewTokens;
-                uint16_t* dst = sA + (row - kMaxFewTokens) * kDownStride + pc * 8;
-                if (j < r) cp_async16(dst, A + static_cast<int64_t>(j) * K + k0 + pc * 8);
-                else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
-            }
+        for (int i = tid; i < kMaxFewTokens * pieces; i += kDownThreads) {
+            const int row = i / pieces, pc = i - row * pieces, j = j0 + row;
+            uint16_t* dst = sA + row * kDownStride + pc * 8;
+            if (j < r) cp_async16(dst, A + static_cast<int64_t>(j) * K + k0 + pc * 8);
+            else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
         }
-        if (!released) {
-            allow_dependents();
-            released = true;
+        if (first) pdl_wait();  // X may be the preceding kernel's output
+        for (int i = tid; i < kMaxFewTokens * pieces; i += kDownThreads) {
+            const int row = i / pieces, pc = i - row * pieces;
+            uint16_t* dst = sX + row * kDownStride + pc * 8;
+            if (row < M) cp_async16(dst, X + static_cast<int64_t>(row) * K + k0 + pc * 8);
+            else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+        }
+        if (first) {
+            pdl_launch_dependents();
+            first = false;
         }
         cp_async_wait_all();
         __syncthreads();
@@ -127,7 +131,10 @@ __global__ void __launch_bounds__(kDownThreads) k_few_down(const uint16_t* __res
                          *reinterpret_cast<const uint32_t*>(ar1 + k + 8));
         }
     }
-    if (!released) allow_dependents();
+    if (first) {  // empty slice (not produced by the launcher): keep the ordering guarantees
+        pdl_wait();
+        pdl_launch_dependents();
+    }
 
     // acc[u]: tokens g (0, 1) and g + 8 (2, 3) at columns 8u + 2q + {0, 1}; the
     // four warps' partials added in order by warp 0 into s_w[0]
@@ -171,8 +178,9 @@ __global__ void __launch_bounds__(kDownThreads) k_few_down(const uint16_t* __res
 // transposed from shared memory with ldmatrix.trans).  The same layout as the
 // T kernel: CTA (x, z) computes columns 16x .. 16x + 15 of V over the z-th of
 // up to 8 slices of d_out, the slices of one column group form a cluster, the
-// slice of dY and of B (up to 512 rows at a time) comes in by asynchronous
-// copies issued at once, and the dependent launch is released right after.
+// slice of B and of dY (up to 256 rows at a time) comes in by asynchronous
+// copies issued at once (B before the wait for the preceding kernel, dY after
+// it), and the dependent launch is released right after.
 constexpr int kVBatch = 256;                    // rows of B per staged slice (small enough to share an SM with the dX kernel)
 constexpr int kVYStride = kVBatch + 8;          // dY staging row stride (elements)
 constexpr int kVBStride = 24;                   // B staging row stride (elements): 48 bytes, conflict-free ldmatrix
@@ -199,17 +207,10 @@ __global__ void __launch_bounds__(kDownThreads) k_few_v(const uint16_t* __restri
     const int n_end = n_begin + 16 * (per + (rank < extra ? 1 : 0));
     float acc[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
 
-    bool released = false;
+    bool first = true;
     for (int n0 = n_begin; n0 < n_end; n0 += kVBatch) {
         const int nn = min(kVBatch, n_end - n0);  // a multiple of 16
         __syncthreads();                          // the previous slice is no longer read
-        // dY[:, n0 : n0 + nn] in 16-byte pieces (N is a multiple of 8)
-        for (int i = tid; i < kMaxFewTokens * (nn / 8); i += kDownThreads) {
-            const int t = i / (nn / 8), pc = i - t * (nn / 8), n = n0 + 8 * pc;
-            uint16_t* dst = sY + t * kVYStride + 8 * pc;
-            if (t < M && n < N) cp_async16(dst, dY + static_cast<int64_t>(t) * N + n);
-            else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
-        }
         // B[n0 : n0 + nn, j0 : j0 + 16] in 16-byte pieces (r is a multiple of 8)
         for (int i = tid; i < nn * 2; i += kDownThreads) {
             const int row = i >> 1, h = i & 1, n = n0 + row, j = j0 + 8 * h;
@@ -217,9 +218,17 @@ __global__ void __launch_bounds__(kDownThreads) k_few_v(const uint16_t* __restri
             if (n < N && j < r) cp_async16(dst, B + static_cast<int64_t>(n) * r + j);
             else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
         }
-        if (!released) {
-            allow_dependents();
-            released = true;
+        if (first) pdl_wait();  // dY may be the preceding kernel's output
+        // dY[:, n0 : n0 + nn] in 16-byte pieces (N is a multiple of 8)
+        for (int i = tid; i < kMaxFewTokens * (nn / 8); i += kDownThreads) {
+            const int t = i / (nn / 8), pc = i - t * (nn / 8), n = n0 + 8 * pc;
+            uint16_t* dst = sY + t * kVYStride + 8 * pc;
+            if (t < M && n < N) cp_async16(dst, dY + static_cast<int64_t>(t) * N + n);
+            else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+        }
+        if (first) {
+            pdl_launch_dependents();
+            first = false;
         }
         cp_async_wait_all();
         __syncthreads();
@@ -239,7 +248,10 @@ __global__ void __launch_bounds__(kDownThreads) k_few_v(const uint16_t* __restri
             mma_m16n8k16(acc[1], a0, a1, a2, a3, c0, c1);
         }
     }
-    if (!released) allow_dependents();
+    if (first) {  // empty slice (not produced by the launcher): keep the ordering guarantees
+        pdl_wait();
+        pdl_launch_dependents();
+    }
 
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
@@ -298,13 +310,15 @@ cudaError_t launch_few_down(const uint16_t* X, const uint16_t* A, int M, int K, 
     cfg.blockDim = dim3(kDownThreads);
     cfg.dynamicSmemBytes = kDownSmem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 1;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = splits;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     TraceScope trace("few_lora_down", stream);
     return cudaLaunchKernelEx(&cfg, k_few_down, X, A, M, K, r, r64, s, T2, T_saved);
 }
@@ -331,13 +345,15 @@ cudaError_t launch_few_v(const uint16_t* dY, const uint16_t* B, int M, int N, in
     cfg.blockDim = dim3(kDownThreads);
     cfg.dynamicSmemBytes = kVSmem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 1;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = splits;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     TraceScope trace("few_lora_v", stream);
     return cudaLaunchKernelEx(&cfg, k_few_v, dY, B, M, N, r, r64, s, V2);
 }

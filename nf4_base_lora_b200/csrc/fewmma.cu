@@ -24,13 +24,18 @@
 // leaves the sums unchanged.
 //
 // Split-K: the CTAs that share one output tile form a thread-block cluster
-// along grid.z.  Inside a CTA the two warps of a row group add their fp32
-// partials through shared memory; every CTA of rank > 0 then pushes its
-// partial tile into a slot of rank 0 (distributed shared memory) and arrives
-// on an mbarrier there; rank 0 adds the slots in rank order and writes bf16.
-// The rank-r extension, once the kernel that produced T2 has finished
-// (programmatic dependent launch), is shared out among the ranks.  The
-// summation order is fixed, so the result is the same on every run.
+// along grid.z.  Inside a CTA every warp puts its fp32 partials into shared
+// memory and each thread adds up four outputs (the two warps of a row group,
+// in order); every CTA of rank > 0 then pushes its partial tile into a slot of
+// rank 0 (distributed shared memory) before a cluster barrier, after which
+// rank 0 adds the slots in rank order and writes bf16 rows.  The rank-r
+// extension, once the kernel that produced T2 has finished (programmatic
+// dependent launch), is shared out among the ranks.  The summation order is
+// fixed, so the result is the same on every run.
+//
+// Launch overlap: the kernel releases its own dependents as soon as it starts
+// (the next layer call's rank-r kernel may then stage its factor rows while
+// this one runs), and asks L2 for the rows of B its extension will read.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -65,10 +70,6 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ void wait_prerequisites() {
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-}
-
 // Even split of `total` units over `parts`; part p gets [begin, end).
 __device__ __forceinline__ void split_range(int total, int parts, int p, int& begin, int& end) {
     const int per = total / parts, extra = total % parts;
@@ -90,21 +91,32 @@ constexpr int kFwdBlockStride = 68;
 constexpr int kFwdTokStride = kFwdSegBlocks * kFwdBlockStride + 16;
 constexpr int kFwdQuadBytes = kTile * 128;  // codes of 4 blocks x 128 rows
 constexpr int kFwdMaxSplit = kMaxSplit;      // partial-tile slots of rank 0: kFwdMaxSplit - 1
-constexpr int kFwdSmemV2 =
-    1024 + 4 * kFwdQuadBytes + (kFwdMaxSplit - 1) * kPartFloats * 4 + 8 * 8 * 32 * 4 + kTok * kFwdTokStride * 2;
+constexpr int kFwdSmemV2 = 1024 + 4 * kFwdQuadBytes + (kFwdMaxSplit - 1) * kPartFloats * 4 + kTok * kFwdTokStride * 2;
+// row stride (floats) of the per-warp partial tiles [token][row] gathered for
+// the reduction: 132 puts the 8 x 4 (row, token) pairs of a fragment store in
+// distinct banks and keeps the rows 16-byte aligned
+constexpr int kSumStride = 132;
+static_assert(2 * kTok * kSumStride * 4 <= 4 * kFwdQuadBytes, "the forward's partial tiles reuse the code buffers");
+
+// Asks L2 for `bytes` (a multiple of 16) from a 16-byte aligned address.
+__device__ __forceinline__ void prefetch_l2_range(const void* src, uint32_t bytes) {
+    const uint8_t* p = static_cast<const uint8_t*>(src);
+    for (uint32_t off = 0; off < bytes; off += 32768u) prefetch_l2_bulk(p + off, min(32768u, bytes - off));
+}
 
 // Registers capped at 96 (48K of the SM's 64K) so that the CTAs of the kernel
 // producing T2, which this one overlaps, keep room on the same SM.
 __global__ void __maxnreg__(96) k_few_fwd(const __grid_constant__ CUtensorMap map_codes, const FewArgs a) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
-    __shared__ uint64_t bar_part, bar_q[4];
+    __shared__ uint64_t bar_q[4];
     __shared__ int s_abort;
-    // [codes: 4 quads x 128 rows x 128 B, 128-byte swizzle][partial slots][warp reduction][activations]
+    pdl_launch_dependents();
+    // [codes: 4 quads x 128 rows x 128 B, 128-byte swizzle; after the loop the
+    //  partial tiles][slots for the other ranks' partial tiles][activations]
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* s_codes = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-    float* s_part = reinterpret_cast<float*>(s_codes + 4 * kFwdQuadBytes);  // [kFwdMaxSplit - 1][8 values][256 threads]
-    float* s_red = s_part + (kFwdMaxSplit - 1) * kPartFloats;               // [8 row groups][8 values][32 lanes]
-    uint16_t* sX = reinterpret_cast<uint16_t*>(s_red + 8 * 8 * 32);          // [16][kFwdTokStride]
+    float* s_part = reinterpret_cast<float*>(s_codes + 4 * kFwdQuadBytes);  // [kFwdMaxSplit - 1][2048]
+    uint16_t* sX = reinterpret_cast<uint16_t*>(s_part + (kFwdMaxSplit - 1) * kPartFloats);  // [16][kFwdTokStride]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, q = lane & 3;
     const int rgp = warp & 7;  // 16-row group of the CTA's 128 rows
@@ -125,7 +137,6 @@ __global__ void __maxnreg__(96) k_few_fwd(const __grid_constant__ CUtensorMap ma
     };
     const int nq_first = (min(kb1 - kb0, kFwdSegBlocks) + 3) / 4;
     if (tid == 0) {
-        mbar_init(&bar_part, splits > 1 ? (splits - 1) * 256 : 1);
         for (int j = 0; j < 4; ++j) mbar_init(&bar_q[j], 1);
         s_abort = 0;
         fence_barrier_init();
@@ -133,6 +144,10 @@ __global__ void __maxnreg__(96) k_few_fwd(const __grid_constant__ CUtensorMap ma
             tma_prefetch_desc(&map_codes);
             issue_codes(kb0, nq_first);
         }
+    } else if (tid == 32 && a.ext_act != nullptr) {
+        // the CTA's rows of B (N is a multiple of 8, so the range is too)
+        const int rows = min(kTile, N - row0);
+        prefetch_l2_range(a.ext_w + static_cast<int64_t>(row0) * a.r, static_cast<uint32_t>(rows * a.r * 2));
     }
 
     const int lr = 16 * rgp + g;  // local row of nA (nB = nA + 8 is local row lr + 8)
@@ -158,15 +173,20 @@ __global__ void __maxnreg__(96) k_few_fwd(const __grid_constant__ CUtensorMap ma
             issued_seg = seg_i;
             issued_nq = nquads;
         }
-        // activations of the segment (L2 hits) and this thread's block scales
+        // activations of the segment (L2 hits) and this thread's block scales;
+        // a token row has `per` 16-byte pieces (128 in a full segment)
+        const int per = nbp * 8;
         uint4 xv[4];
+        int xt[4], xpc[4];
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
             const int i = tid + p * kThreads;
-            const int t = i / (nbp * 8), pc = i - t * (nbp * 8);
+            xt[p] = per == 128 ? (i >> 7) : i / per;
+            xpc[p] = i - xt[p] * per;
             xv[p] = make_uint4(0, 0, 0, 0);
-            if (t < M && pc < nb * 8)
-                xv[p] = __ldg(reinterpret_cast<const uint4*>(a.act + static_cast<int64_t>(t) * K + seg0 * 64) + pc);
+            if (xt[p] < M && xpc[p] < nb * 8)
+                xv[p] = __ldg(reinterpret_cast<const uint4*>(a.act + static_cast<int64_t>(xt[p]) * K + seg0 * 64) +
+                              xpc[p]);
         }
         int qA[2], qB[2];
         float aA[2], aB[2];
@@ -185,8 +205,7 @@ __global__ void __maxnreg__(96) k_few_fwd(const __grid_constant__ CUtensorMap ma
         }
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
-            const int i = tid + p * kThreads;
-            const int t = i / (nbp * 8), pc = i - t * (nbp * 8);
+            const int t = xt[p], pc = xpc[p];
             if (t < kTok) {
                 const int lb = pc >> 3, kk = (pc & 7) * 8;
                 uint2* dst = reinterpret_cast<uint2*>(sX + t * kFwdTokStride + lb * kFwdBlockStride + kk);
@@ -240,8 +259,8 @@ __global__ void __maxnreg__(96) k_few_fwd(const __grid_constant__ CUtensorMap ma
     // producing T2 has finished (programmatic dependent launch).  Its 16-wide
     // chunks are dealt round-robin to the ranks of the cluster (and to the two
     // warps of a row group), which add them to the partials they push.
+    if (a.pdl) pdl_wait();
     if (a.ext_act != nullptr) {
-        if (a.pdl) wait_prerequisites();
         const int nchunks = 2 * a.r64 / 16;
         const uint16_t* bA = a.ext_w + static_cast<int64_t>(nA) * a.r;
         const uint16_t* bB = a.ext_w + static_cast<int64_t>(nB) * a.r;
@@ -266,54 +285,59 @@ __global__ void __maxnreg__(96) k_few_fwd(const __grid_constant__ CUtensorMap ma
         }
     }
 
-    // the two warps of a row group add up (qs 1 into qs 0), then ranks > 0
-    // push to rank 0, which adds the ranks in order
-    float v[8] = {acc0[0], acc0[1], acc0[2], acc0[3], acc1[0], acc1[1], acc1[2], acc1[3]};
-    if (qs == 1) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) s_red[(rgp * 8 + i) * 32 + lane] = v[i];
+    // every warp's partials into shared memory (the code buffers are free:
+    // every copy has landed and been read), s_sum[qs][token][local row]; then
+    // thread tid adds up token tid / 32, rows 4 (tid % 32) .. + 3: the two
+    // warps of the row group in order
+    __syncthreads();
+    float* s_sum = reinterpret_cast<float*>(s_codes);
+    {
+        // acc0: tokens 2q, 2q + 1 of rows lr (0, 1) and lr + 8 (2, 3); acc1: tokens + 8
+        float* d0 = s_sum + qs * kTok * kSumStride + (2 * q) * kSumStride + lr;
+        float* d8 = d0 + 8 * kSumStride;
+        d0[0] = acc0[0];
+        d0[kSumStride] = acc0[1];
+        d0[8] = acc0[2];
+        d0[kSumStride + 8] = acc0[3];
+        d8[0] = acc1[0];
+        d8[kSumStride] = acc1[1];
+        d8[8] = acc1[2];
+        d8[kSumStride + 8] = acc1[3];
     }
     __syncthreads();
-    bool waited = false;
-    if (qs == 0) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] += s_red[(rgp * 8 + i) * 32 + lane];
-        const int slot = tid;  // 0..255
-        if (rank != 0) {
-            cluster_wait_acquire();
-            waited = true;
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-                st_cluster_f32(cluster_map(smem_u32(s_part + ((rank - 1) * 8 + i) * 256 + slot), 0), v[i]);
-            mbar_arrive_remote(cluster_map(smem_u32(&bar_part), 0));
-        } else {
-            const bool got = splits == 1 || mbar_wait_cluster(&bar_part, 0, &s_abort);
-            if (got) {
-                for (int rk = 1; rk < splits; ++rk)
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) v[i] += s_part[((rk - 1) * 8 + i) * 256 + slot];
-                // v[0..3]: tokens 2q, 2q+1 of rows nA (0, 1) and nB (2, 3); v[4..7]: tokens + 8
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int t0 = 2 * q + 8 * h;
-                    auto put = [&](int t, int n, float x) {
-                        if (t < M && n < N) {
-                            const __nv_bfloat16 b = __float2bfloat16_rn(x);
-                            a.out[static_cast<int64_t>(t) * N + n] = *reinterpret_cast<const uint16_t*>(&b);
-                        }
-                    };
-                    put(t0, nA, v[4 * h + 0]);
-                    put(t0 + 1, nA, v[4 * h + 1]);
-                    put(t0, nB, v[4 * h + 2]);
-                    put(t0 + 1, nB, v[4 * h + 3]);
-                }
-            }
-        }
+    const int ot = tid >> 5, orow = 4 * (tid & 31);
+    float4 o = *reinterpret_cast<const float4*>(s_sum + ot * kSumStride + orow);
+    {
+        const float4 o1 = *reinterpret_cast<const float4*>(s_sum + (kTok + ot) * kSumStride + orow);
+        o.x += o1.x;
+        o.y += o1.y;
+        o.z += o1.z;
+        o.w += o1.w;
     }
-    // no CTA leaves while another may still write into its shared memory
-    if (!waited) cluster_wait_acquire();
+    // ranks > 0 push into rank 0's slots; the cluster barrier (every CTA has
+    // started, then every push is visible) orders them before rank 0's sums,
+    // and no CTA touches another's shared memory after it
+    cluster_wait_acquire();
+    if (rank != 0)
+        st_cluster_f4(cluster_map(smem_u32(s_part + (rank - 1) * kPartFloats + 4 * tid), 0), o.x, o.y, o.z, o.w);
     cluster_arrive_release();
     cluster_wait_acquire();
+    if (rank == 0) {
+        for (int rk = 1; rk < splits; ++rk) {
+            const float4 v = *reinterpret_cast<const float4*>(s_part + (rk - 1) * kPartFloats + 4 * tid);
+            o.x += v.x;
+            o.y += v.y;
+            o.z += v.z;
+            o.w += v.w;
+        }
+        const int n = row0 + orow;  // N is a multiple of 8: rows n .. n + 3 all exist or none does
+        if (ot < M && n < N) {
+            uint2 packed;
+            packed.x = pack_bf16x2(o.x, o.y);
+            packed.y = pack_bf16x2(o.z, o.w);
+            *reinterpret_cast<uint2*>(a.out + static_cast<int64_t>(ot) * N + n) = packed;
+        }
+    }
 }
 
 // ---------------------------------------------------------------- input gradient
@@ -334,7 +358,7 @@ constexpr int kDxYStride = kDxRowsSeg + 8;         // dY staging, elements (2064
 constexpr int kDxMaxSplit = 4;
 constexpr int kDxSmem = 1024 + kDxRowsSeg * 64 + 16 * kDxTileBytes + kTok * kDxYStride * 2 +
                         (kDxMaxSplit - 1) * kPartFloats * 4;
-static_assert(7 * 2 * 32 * 32 * 4 <= 16 * kDxTileBytes, "warp reduction reuses the tiles");
+static_assert(8 * kTok * kSumStride * 4 <= 16 * kDxTileBytes, "the partial tiles reuse the decode tiles");
 static_assert(kTok * (2 * 256 + 8) <= kTok * kDxYStride, "V2 staging reuses the dY staging");
 
 __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
@@ -369,15 +393,16 @@ __device__ __forceinline__ void dx_chunk_mma(float (&acc)[4][2][4], uint32_t til
 
 __global__ void __maxnreg__(112) k_few_dx(const __grid_constant__ CUtensorMap map_codes, const FewArgs a) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
-    __shared__ uint64_t bar_part, bar_c[4];
+    __shared__ uint64_t bar_c[4];
     __shared__ int s_abort;
-    // [codes: kDxRowsSeg rows x 64 B, 64-byte swizzle][16 warp tiles][dY staging][partial slots]
+    pdl_launch_dependents();
+    // [codes: kDxRowsSeg rows x 64 B, 64-byte swizzle][16 warp tiles; after the
+    //  loop the partial tiles][dY staging][slots for the other ranks' partial tiles]
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* s_codes = smem_raw + (((raw + 1023u) & ~1023u) - raw);
     uint8_t* s_tiles = s_codes + kDxRowsSeg * 64;
     uint16_t* sY = reinterpret_cast<uint16_t*>(s_tiles + 16 * kDxTileBytes);
-    float* s_part = reinterpret_cast<float*>(sY + kTok * kDxYStride);  // [kDxMaxSplit - 1][32 values][64 threads]
-    float* s_red = reinterpret_cast<float*>(s_tiles);                   // [7][2][32 values][32 lanes], after the loop
+    float* s_part = reinterpret_cast<float*>(sY + kTok * kDxYStride);  // [kDxMaxSplit - 1][2048]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, q = lane & 3;
     const int cb = warp & 1, rw = warp >> 1;
@@ -396,7 +421,6 @@ __global__ void __maxnreg__(112) k_few_dx(const __grid_constant__ CUtensorMap ma
         }
     };
     if (tid == 0) {
-        mbar_init(&bar_part, splits > 1 ? (splits - 1) * 64 : 1);
         for (int b = 0; b < 4; ++b) mbar_init(&bar_c[b], 1);
         s_abort = 0;
         fence_barrier_init();
@@ -404,6 +428,11 @@ __global__ void __maxnreg__(112) k_few_dx(const __grid_constant__ CUtensorMap ma
             tma_prefetch_desc(&map_codes);
             issue_codes(ch0, min(ch1, ch0 + kDxRowsSeg / 32));
         }
+    } else if (tid >= 32 && tid < 32 + a.r && a.ext_act != nullptr) {
+        // row tid - 32 of A over the CTA's one or two 64-column blocks
+        const int j = tid - 32;
+        prefetch_l2_bulk(a.ext_w + static_cast<int64_t>(j) * K + 128 * blockIdx.x,
+                         2 * static_cast<int>(blockIdx.x) + 1 < bpr ? 256u : 128u);
     }
     const bool two_halves = M > 8;
     float acc[4][2][4];
@@ -432,10 +461,12 @@ __global__ void __maxnreg__(112) k_few_dx(const __grid_constant__ CUtensorMap ma
             issued_boxes = (sc1 - sc0 + 7) / 8;
         }
         // dY[:, 32 sc0 : 32 sc1] (rows >= N, tokens >= M as zeros) and this thread's scales
+        // a token row has `per` 8-byte pieces (256 in a full segment)
+        const int per = rows / 4;
         uint2 yv[8];
 #pragma unroll
         for (int p = 0; p < 8; ++p) {
-            const int i = tid + p * kThreads, t = i / (rows / 4), pc = i - t * (rows / 4);
+            const int i = tid + p * kThreads, t = per == 256 ? (i >> 8) : i / per, pc = i - t * per;
             const int n = 32 * sc0 + 4 * pc;
             yv[p] = make_uint2(0, 0);
             if (t < M && n < N) yv[p] = __ldg(reinterpret_cast<const uint2*>(a.act + static_cast<int64_t>(t) * N + n));
@@ -452,7 +483,7 @@ __global__ void __maxnreg__(112) k_few_dx(const __grid_constant__ CUtensorMap ma
         }
 #pragma unroll
         for (int p = 0; p < 8; ++p) {
-            const int i = tid + p * kThreads, t = i / (rows / 4), pc = i - t * (rows / 4);
+            const int i = tid + p * kThreads, t = per == 256 ? (i >> 8) : i / per, pc = i - t * per;
             if (t < kTok) *reinterpret_cast<uint2*>(sY + t * kDxYStride + 4 * pc) = yv[p];
         }
         __syncthreads();
@@ -489,8 +520,8 @@ __global__ void __maxnreg__(112) k_few_dx(const __grid_constant__ CUtensorMap ma
     // tiles, against V2 staged in place of dY, once the kernel producing V2
     // has finished; the chunks are dealt round-robin to the ranks, which add
     // them to the partials they push
+    if (a.pdl) pdl_wait();
     if (a.ext_act != nullptr) {
-        if (a.pdl) wait_prerequisites();
         const int vstride = 2 * a.r64 + 8;
         __syncthreads();  // dY staging and tiles are free
         for (int i = tid; i < kTok * (2 * a.r64 / 4); i += kThreads) {
@@ -512,72 +543,58 @@ __global__ void __maxnreg__(112) k_few_dx(const __grid_constant__ CUtensorMap ma
         }
     }
 
-    // the eight row warps of a block add up in order (into row warp 0), then
-    // ranks > 0 push to rank 0, which adds the ranks in order
-    __syncthreads();  // tiles are free for the reduction
-    if (rw > 0) {
+    // every warp's partials into shared memory (the tiles are free),
+    // s_sum[row warp][token][local column]; then thread tid adds up token
+    // tid / 32, columns 4 (tid % 32) .. + 3: the eight row warps in order
+    __syncthreads();
+    float* s_sum = reinterpret_cast<float*>(s_tiles);
+    {
+        float* dst = s_sum + rw * kTok * kSumStride;
+        // acc[m][h]: columns 64 cb + 16m + g (e = 0, 1) and + 8 (e = 2, 3), tokens 2q + 8h + (e & 1)
 #pragma unroll
         for (int m = 0; m < 4; ++m)
 #pragma unroll
             for (int h = 0; h < 2; ++h)
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
-                    s_red[(((rw - 1) * 2 + cb) * 32 + (m * 8 + h * 4 + e)) * 32 + lane] = acc[m][h][e];
+                    dst[(2 * q + 8 * h + (e & 1)) * kSumStride + 64 * cb + 16 * m + g + 8 * (e >> 1)] = acc[m][h][e];
     }
     __syncthreads();
-    bool waited = false;
-    if (rw == 0) {
-        for (int k = 0; k < 7; ++k)
+    const int ot = tid >> 5, ocol = 4 * (tid & 31);
+    float4 o = *reinterpret_cast<const float4*>(s_sum + ot * kSumStride + ocol);
 #pragma unroll
-            for (int m = 0; m < 4; ++m)
-#pragma unroll
-                for (int h = 0; h < 2; ++h)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) acc[m][h][e] += s_red[((k * 2 + cb) * 32 + (m * 8 + h * 4 + e)) * 32 + lane];
-        const int slot = cb * 32 + lane;  // 0..63
-        if (rank != 0) {
-            cluster_wait_acquire();
-            waited = true;
-#pragma unroll
-            for (int m = 0; m < 4; ++m)
-#pragma unroll
-                for (int h = 0; h < 2; ++h)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        st_cluster_f32(cluster_map(smem_u32(s_part + ((rank - 1) * 32 + (m * 8 + h * 4 + e)) * 64 + slot), 0),
-                                       acc[m][h][e]);
-            mbar_arrive_remote(cluster_map(smem_u32(&bar_part), 0));
-        } else {
-            const bool got = splits == 1 || mbar_wait_cluster(&bar_part, 0, &s_abort);
-            if (got && blk_ok) {
-                for (int rk = 1; rk < splits; ++rk)
-#pragma unroll
-                    for (int m = 0; m < 4; ++m)
-#pragma unroll
-                        for (int h = 0; h < 2; ++h)
-#pragma unroll
-                            for (int e = 0; e < 4; ++e)
-                                acc[m][h][e] += s_part[((rk - 1) * 32 + (m * 8 + h * 4 + e)) * 64 + slot];
-                // acc[m][h]: columns 16m + g (e = 0, 1) and + 8 (e = 2, 3), tokens 2q + 8h + (e & 1)
-#pragma unroll
-                for (int m = 0; m < 4; ++m)
-#pragma unroll
-                    for (int h = 0; h < 2; ++h)
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int t = 2 * q + 8 * h + (e & 1);
-                            const int col = 64 * blk + 16 * m + g + 8 * (e >> 1);
-                            if (t < M) {
-                                const __nv_bfloat16 b = __float2bfloat16_rn(acc[m][h][e]);
-                                a.out[static_cast<int64_t>(t) * K + col] = *reinterpret_cast<const uint16_t*>(&b);
-                            }
-                        }
-            }
-        }
+    for (int w = 1; w < 8; ++w) {
+        const float4 v = *reinterpret_cast<const float4*>(s_sum + (w * kTok + ot) * kSumStride + ocol);
+        o.x += v.x;
+        o.y += v.y;
+        o.z += v.z;
+        o.w += v.w;
     }
-    if (!waited) cluster_wait_acquire();
+    // ranks > 0 push into rank 0's slots; the cluster barrier (every CTA has
+    // started, then every push is visible) orders them before rank 0's sums,
+    // and no CTA touches another's shared memory after it
+    cluster_wait_acquire();
+    if (rank != 0)
+        st_cluster_f4(cluster_map(smem_u32(s_part + (rank - 1) * kPartFloats + 4 * tid), 0), o.x, o.y, o.z, o.w);
     cluster_arrive_release();
     cluster_wait_acquire();
+    if (rank == 0) {
+        for (int rk = 1; rk < splits; ++rk) {
+            const float4 v = *reinterpret_cast<const float4*>(s_part + (rk - 1) * kPartFloats + 4 * tid);
+            o.x += v.x;
+            o.y += v.y;
+            o.z += v.z;
+            o.w += v.w;
+        }
+        // columns 128 x + ocol .. + 3 lie in block 2x (ocol < 64) or 2x + 1
+        const bool col_ok = ocol < 64 || 2 * static_cast<int>(blockIdx.x) + 1 < bpr;
+        if (ot < M && col_ok) {
+            uint2 packed;
+            packed.x = pack_bf16x2(o.x, o.y);
+            packed.y = pack_bf16x2(o.z, o.w);
+            *reinterpret_cast<uint2*>(a.out + static_cast<int64_t>(ot) * K + 128 * blockIdx.x + ocol) = packed;
+        }
+    }
 }
 
 // `configured`: per-device flags of this kernel (both kernels have the same
