@@ -283,14 +283,14 @@ def workload_config(wl):
 
 
 class GpuWorkload:
-    def __init__(self, nf, wl, device, copies):
+    def __init__(self, nf, wl, device, copies, keep_fp32=False):
         self.nf, self.wl, self.device = nf, wl, device
         self.mods = []
         self.fp32 = []  # the fp32 weights, kept where the workload times their encoding
         for i, mod in enumerate(wl.modules):
             W = torch.from_numpy(workloads.weight(mod.d_out, mod.d_in, wl.sigma, wl.outliers, i)).to(device)
             enc = nf.nf4_quantize(W)
-            if wl.quantize_timed:
+            if wl.quantize_timed or keep_fp32:
                 self.fp32.append(W)
             del W
             encs = [enc] + [nf.NF4Tensor(mod.d_out, mod.d_in, device, buffer=enc.buffer.clone())
@@ -314,6 +314,7 @@ class GpuWorkload:
                          nf.qlora_bwd_workspace_bytes(m, mod.d_out, mod.d_in, wl.r))
         self.ws = torch.empty(ws, dtype=torch.uint8, device=device)
         self.plan = step_plan(wl)
+        self.sms = torch.cuda.get_device_properties(device).multi_processor_count
 
     def step(self, copy_base, X=None, dY=None, outs=None):
         """Enqueue one step; pass p uses encoded copy (copy_base + p)."""
@@ -417,6 +418,120 @@ def time_quantize(nf, gw, args, stream, device, world, hbm_peak, peak_src):
     return out
 
 
+def time_adamw(nf, gw, args, stream, device, world, hbm_peak, peak_src, l2):
+    """The step after the backward: one lora_adamw_step over every module's A
+    and B (fp32 master, bf16 copy, bf16 gradient from the backward, fp32
+    moments), timed on its own.  The optimizer state rotates over enough
+    copies to exceed 4x L2, as it would be cold after the layer's GEMMs."""
+    import torch.distributed as dist  # noqa: F401
+    grads = [t for d in gw.mods for t in (d["dA"], d["dB"])]
+    n_total = sum(g.numel() for g in grads)
+    per_copy = 26 * n_total  # fp32 master, m, v + bf16 copy and gradient
+    copies = max(1, int(math.ceil(4 * l2 / per_copy)))
+    states = []
+    for _ in range(copies):
+        st = []
+        for g, src in zip(grads, [t for d in gw.mods for t in (d["A"], d["B"])]):
+            st.append((src.float().reshape(-1).contiguous(), torch.empty_like(src).reshape(-1),
+                       g.reshape(-1), torch.zeros(g.numel(), dtype=torch.float32, device=device),
+                       torch.zeros(g.numel(), dtype=torch.float32, device=device)))
+        states.append(st)
+
+    def one_pass(k, t):
+        with torch.cuda.stream(stream):
+            nf.lora_adamw_step(states[k % copies], lr=2e-4, beta1=0.9, beta2=0.999, eps=1e-8,
+                               weight_decay=0.0, step=t)
+
+    for k in range(max(args.warmup, copies)):
+        one_pass(k, k + 1)
+    torch.cuda.synchronize()
+    passes = max(3, min(args.steps, 50))
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for k in range(passes):
+        one_pass(k, 100 + k)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / passes
+    if world > 1:
+        from nf4_base_lora_b200 import dp
+        ms = dp.max_over_ranks(ms, device)
+    nf.trace_start(64)
+    one_pass(0, 200)
+    torch.cuda.synchronize()
+    recs = nf.trace_records()
+    nf.trace_stop()
+    k_ms = [r[1] for r in recs if r[0] == "lora_adamw"]
+    step_bytes = 28 * n_total
+    value = world * step_bytes / (ms * 1e-3) / 1e9
+    out = {"ms_per_pass": ms, "passes": passes, "params": n_total, "bytes_per_pass": step_bytes,
+           "value": value, "unit": "GB/s", "frac": value / world / hbm_peak,
+           "algorithmic": "28 bytes per parameter: fp32 master, m, v read and written, bf16 gradient read, "
+                          "bf16 copy written",
+           "l2_flush": "rotating %d optimizer-state copies (%.0f MB)" % (copies, copies * per_copy / 1e6),
+           "peak_source": peak_src + " (hbm_gbs)"}
+    if k_ms:
+        out["kernels"] = {"lora_adamw": {"launches": len(k_ms), "avg_us": sum(k_ms) / len(k_ms) * 1e3}}
+    return out
+
+
+FP64_FMA_PER_CLK_PER_SM = 64  # B200: 148 SMs x 64 x 2 x 1.965 GHz = 37.2 TFLOP/s fp64, the published figure
+
+
+def time_merge(nf, gw, args, stream, device, world, clocks_mhz=1965.0):
+    """Deployment: the adapter folded into each module's base and the result
+    encoded again (nf4_merge_requantize), timed on its own over all modules.
+    The merge kernel is bound by its fp64 multiply-adds (n r per module);
+    its roofline is the fp64 FMA rate of the SMs at the maximum SM clock."""
+    wl = gw.wl
+    outs = [nf.NF4Tensor(m.d_out, m.d_in, device) for m in wl.modules]
+    ws = torch.empty(max(nf.nf4_merge_workspace_bytes(m.d_out, m.d_in) for m in wl.modules),
+                     dtype=torch.uint8, device=device)
+
+    def one_pass():
+        with torch.cuda.stream(stream):
+            for d, out in zip(gw.mods, outs):
+                nf.nf4_merge_requantize(d["encs"][0], d["A"], d["B"], wl.scaling, out=out, workspace=ws)
+
+    for _ in range(args.warmup):
+        one_pass()
+    torch.cuda.synchronize()
+    passes = max(3, min(args.steps, 20))
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(passes):
+        one_pass()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / passes
+    if world > 1:
+        from nf4_base_lora_b200 import dp
+        ms = dp.max_over_ranks(ms, device)
+    nf.trace_start(16 * len(wl.modules) + 64)
+    one_pass()
+    torch.cuda.synchronize()
+    per_kernel = {}
+    for name, kms in nf.trace_records():
+        per_kernel.setdefault(name, []).append(kms)
+    nf.trace_stop()
+    weights = sum(m.d_out * m.d_in for m in wl.modules)
+    flops = 2.0 * weights * wl.r
+    peak = gw.sms * FP64_FMA_PER_CLK_PER_SM * 2 * clocks_mhz * 1e6 / 1e12
+    out = {"ms_per_pass": ms, "passes": passes, "weights_per_pass": weights,
+           "kernels": {k: {"launches": len(v), "avg_us": sum(v) / len(v) * 1e3} for k, v in sorted(per_kernel.items())}}
+    mk = per_kernel.get("nf4_merge_lora")
+    if mk:
+        achieved = flops / (sum(mk) * 1e-3) / 1e12
+        out["roofline"] = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s (fp64)",
+                           "frac": achieved / peak, "kernel": "nf4_merge_lora",
+                           "algorithmic": "2 n r fp64 flops per module (the rank-r sum of each merged weight)",
+                           "peak_source": "derived: %d SMs x %d fp64 FMA/clk x 2 x %.0f MHz"
+                                          % (gw.sms, FP64_FMA_PER_CLK_PER_SM, clocks_mhz)}
+    return out
+
+
 def run_ours(args, wl):
     import torch.distributed as dist
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -431,6 +546,26 @@ def run_ours(args, wl):
     import nf4_base_lora_b200 as nf
     hbm_peak, tc_peak, peak_src = load_peaks()
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    if args.only:
+        # one phase of the workload on its own (a short command to profile):
+        # the encoding, the merge + re-encoding or the optimizer step
+        gw = GpuWorkload(nf, wl, device, 1, keep_fp32=args.only == "quantize")
+        stream = torch.cuda.Stream(device)
+        if args.only == "quantize":
+            obj = time_quantize(nf, gw, args, stream, device, world, hbm_peak, peak_src)
+        elif args.only == "merge":
+            obj = time_merge(nf, gw, args, stream, device, world)
+        else:
+            with torch.cuda.stream(stream):
+                gw.step(0)  # the backward fills dA, dB
+            obj = time_adamw(nf, gw, args, stream, device, world, hbm_peak, peak_src, l2)
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "phase": args.only, "n_gpus": world,
+                              "config": workload_config(wl), args.only: obj}), flush=True)
+        return
     plan = step_plan(wl)
     wbytes = sum(weight_bytes(mod.d_out, mod.d_in) for mod in wl.modules)
     # enough encoded copies that consecutive passes of one module never share L2
@@ -560,6 +695,9 @@ def run_ours(args, wl):
                         "peak_source": peak_src + " (bf16_tflops_sustained)"}
     kernel_table = {k: {"launches": v[0], "avg_us": v[1] / v[0] * 1e3} for k, v in sorted(kstats.items())}
     quantize = time_quantize(nf, gw, args, stream, device, world, hbm_peak, peak_src) if gw.fp32 else None
+    optimizer = (time_adamw(nf, gw, args, stream, device, world, hbm_peak, peak_src, l2)
+                 if wl.backward != "dx" else None)
+    merge = time_merge(nf, gw, args, stream, device, world) if wl.quantize_timed else None
 
     # end to end through the public API: pinned host inputs -> device -> layer -> host
     e2e_steps = max(3, min(args.steps, 200))
@@ -641,6 +779,10 @@ def run_ours(args, wl):
             "clocks": clocks}
     if quantize is not None:
         line["quantize"] = quantize
+    if optimizer is not None:
+        line["optimizer"] = optimizer
+    if merge is not None:
+        line["merge"] = merge
     print(json.dumps(line), flush=True)
 
 
@@ -654,6 +796,8 @@ def main():
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--only", choices=("quantize", "merge", "optimizer"),
+                    help="time one phase of the workload alone (encoding, merge + re-encoding, optimizer step)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -213,6 +213,87 @@ int qlora_linear_bwd(const nf4_tensor* w, const uint16_t* A, const uint16_t* B, 
                      uint16_t* dB, int accumulate_grads, void* ws, size_t ws_bytes,
                      void* stream);
 
+/* ---------------------------------------------------------------- adapter merge */
+
+/* Workspace (device bytes, 256-byte aligned) of nf4_merge_requantize: the
+ * fp32 merged weight plus the encoder's scratch.  0 for invalid shapes. */
+size_t nf4_merge_workspace_bytes(int64_t d_out, int64_t d_in);
+
+/*
+ * nf4_merge_lora -- the merged weight for deployment ([QP] §12.3: fold the
+ * adapter into the base, W + s B A; §12.4: the effective weight is the
+ * dequantised base plus the adapter):
+ *   W_merged[n, k] = fp32( W_hat[n, k] + s * sum_j B[n, j] A[j, k] )
+ * with W_hat the bf16 dequantisation of `w` (as nf4_dequantize), each
+ * product of two bf16 values exact in fp64, the rank sum in fp64 in
+ * ascending j (each addition rounded once), then one fp64 multiply by s, one
+ * fp64 add and one rounding to fp32 (to nearest even): bit-identical to that
+ * arithmetic on every run.  A [r, d_in], B [d_out, r] bf16; W_merged
+ * [d_out, d_in] fp32 (device).  Requirements: 1 <= r <= 256 (any r), s
+ * finite, the weight's shape rules.
+ */
+int nf4_merge_lora(const nf4_tensor* w, const uint16_t* A, const uint16_t* B, int r, float scaling,
+                   float* W_merged, void* stream);
+
+/*
+ * nf4_merge_requantize -- nf4_merge_lora followed by nf4_quantize of the
+ * merged weight into `out` ([QP] §12.3: the last step rounds again, so the
+ * merged 4-bit model is not exactly base + adapter).  `out` has the shape of
+ * `w` and may be `w` itself (the merged weight is complete before encoding
+ * starts).  ws >= nf4_merge_workspace_bytes(d_out, d_in).
+ */
+int nf4_merge_requantize(const nf4_tensor* w, const uint16_t* A, const uint16_t* B, int r,
+                         float scaling, const nf4_tensor* out, void* ws, size_t ws_bytes,
+                         void* stream);
+
+/* ---------------------------------------------------------------- optimizer */
+
+/*
+ * One trainable adapter tensor (A or B) for lora_adamw_step.  Device
+ * pointers, 16-byte aligned, n elements each, caller-owned:
+ *   master  fp32 parameters, updated in place;
+ *   param   the bf16 copy the layer reads, overwritten with bf16_rne(master),
+ *           or NULL;
+ *   grad    bf16 gradient (the dA or dB of qlora_linear_bwd), read only;
+ *   m, v    fp32 first and second moments, updated in place (zero before
+ *           the first step).
+ */
+typedef struct {
+    float* master;
+    uint16_t* param;
+    const uint16_t* grad;
+    float* m;
+    float* v;
+    int64_t n;
+} lora_adamw_tensor;
+
+typedef struct {
+    float lr;
+    float beta1;
+    float beta2;
+    float eps;
+    float weight_decay;
+    int64_t step; /* t, counted from 1 */
+} lora_adamw_hparams;
+
+/*
+ * lora_adamw_step -- one AdamW update of `count` adapter tensors, the step
+ * that follows the backward ([QP] §7.3: two fp32 moments per trainable
+ * parameter; §8.3: an fp32 master copy beside a bf16 adapter; the frozen
+ * base has no optimizer state).  The pages print no update rule; this is
+ * decoupled-weight-decay AdamW with bias-corrected moments:
+ *   p <- p (1 - lr wd);   m <- b1 m + (1 - b1) g;   v <- b2 v + (1 - b2) g^2;
+ *   p <- p - lr / (1 - b1^t) * m / (sqrt(v) / sqrt(1 - b2^t) + eps)
+ * computed per element in fp32; the constants 1 - lr wd, 1 - b1, 1 - b2,
+ * lr / (1 - b1^t) and 1 / sqrt(1 - b2^t) are formed on the host in fp64 and
+ * rounded once.  Requirements: 1 <= count <= 1024; n >= 0 (n = 0 tensors are
+ * skipped and may have NULL pointers); step >= 1; 0 <= beta1, beta2 < 1;
+ * eps > 0; lr >= 0; weight_decay >= 0; all finite.  Up to 8 tensors share
+ * one launch.  The tensors must not overlap one another.
+ */
+int lora_adamw_step(const lora_adamw_tensor* tensors, int count, const lora_adamw_hparams* h,
+                    void* stream);
+
 /* ---------------------------------------------------------------- status */
 
 /* Text of the last error returned to the calling host thread ("" if none). */

@@ -31,7 +31,8 @@ STATUS_NAMES = {0: "NF4_OK", -1: "NF4_ERR_INVALID_ARG", -2: "NF4_ERR_UNSUPPORTED
 ABI_SYMBOLS = ("nf4_packed_bytes", "nf4_tensor_from_buffer", "nf4_quantize_workspace_bytes",
                "qlora_fwd_workspace_bytes", "qlora_bwd_workspace_bytes", "nf4_quantize",
                "nf4_quantize_noalloc", "nf4_dequantize", "qlora_linear_fwd", "qlora_linear_bwd",
-               "nf4lora_last_error_string", "nf4lora_device_status", "nf4lora_trace_start",
+               "nf4_merge_workspace_bytes", "nf4_merge_lora", "nf4_merge_requantize",
+               "lora_adamw_step", "nf4lora_last_error_string", "nf4lora_device_status", "nf4lora_trace_start",
                "nf4lora_trace_stop", "nf4lora_trace_count", "nf4lora_trace_get", "nf4lora_version")
 
 
@@ -39,6 +40,16 @@ class Nf4TensorStruct(ctypes.Structure):
     _fields_ = [("d_out", ctypes.c_int64), ("d_in", ctypes.c_int64),
                 ("codes", ctypes.c_void_p), ("qscale", ctypes.c_void_p),
                 ("scale2", ctypes.c_void_p), ("scale_mean", ctypes.c_void_p)]
+
+
+class AdamwTensorStruct(ctypes.Structure):
+    _fields_ = [("master", ctypes.c_void_p), ("param", ctypes.c_void_p), ("grad", ctypes.c_void_p),
+                ("m", ctypes.c_void_p), ("v", ctypes.c_void_p), ("n", ctypes.c_int64)]
+
+
+class AdamwHparamsStruct(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float),
+                ("eps", ctypes.c_float), ("weight_decay", ctypes.c_float), ("step", ctypes.c_int64)]
 
 
 class Nf4Error(RuntimeError):
@@ -66,6 +77,10 @@ def _load() -> ctypes.CDLL:
         "nf4_dequantize": (I, [S, P, P]),
         "qlora_linear_fwd": (I, [S, P, P, I, F, P, I64, P, P, P, SZ, P]),
         "qlora_linear_bwd": (I, [S, P, P, I, F, P, P, P, I64, P, P, P, I, P, SZ, P]),
+        "nf4_merge_workspace_bytes": (SZ, [I64, I64]),
+        "nf4_merge_lora": (I, [S, P, P, I, F, P, P]),
+        "nf4_merge_requantize": (I, [S, P, P, I, F, S, P, SZ, P]),
+        "lora_adamw_step": (I, [ctypes.POINTER(AdamwTensorStruct), I, ctypes.POINTER(AdamwHparamsStruct), P]),
         "nf4lora_last_error_string": (ctypes.c_char_p, []),
         "nf4lora_device_status": (I, [P]),
         "nf4lora_trace_start": (I, [I]),
@@ -257,6 +272,60 @@ def qlora_linear_bwd(w: NF4Tensor, A: torch.Tensor, B: torch.Tensor, scaling: fl
                                 1 if accumulate else 0, _ptr(ws), 0 if ws is None else ws.numel(),
                                 _stream()))
     return dX, dA, dB
+
+
+def nf4_merge_workspace_bytes(d_out: int, d_in: int) -> int:
+    return int(lib.nf4_merge_workspace_bytes(d_out, d_in))
+
+
+def _adapter(w: NF4Tensor, A: torch.Tensor, B: torch.Tensor) -> int:
+    _bf16(A, "A")
+    _bf16(B, "B")
+    r = A.shape[0]
+    if A.dim() != 2 or B.dim() != 2 or A.shape[1] != w.d_in or tuple(B.shape) != (w.d_out, r):
+        raise ValueError("A must be [r, d_in] and B [d_out, r]")
+    return r
+
+
+def nf4_merge_lora(w: NF4Tensor, A: torch.Tensor, B: torch.Tensor, scaling: float,
+                   out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """fp32 W_hat + s B A [d_out, d_in] (the adapter folded into the base)."""
+    r = _adapter(w, A, B)
+    out = out if out is not None else torch.empty((w.d_out, w.d_in), dtype=torch.float32, device=A.device)
+    _check(lib.nf4_merge_lora(ctypes.byref(w.struct), _ptr(A), _ptr(B), r, scaling, _ptr(out), _stream()))
+    return out
+
+
+def nf4_merge_requantize(w: NF4Tensor, A: torch.Tensor, B: torch.Tensor, scaling: float,
+                         out: Optional[NF4Tensor] = None, workspace: Optional[torch.Tensor] = None) -> NF4Tensor:
+    """The merged weight encoded again (NF4 + double quantisation); `out` may be `w`."""
+    r = _adapter(w, A, B)
+    out = out if out is not None else NF4Tensor(w.d_out, w.d_in, A.device)
+    ws = workspace if workspace is not None else _workspace(nf4_merge_workspace_bytes(w.d_out, w.d_in), A.device)
+    _check(lib.nf4_merge_requantize(ctypes.byref(w.struct), _ptr(A), _ptr(B), r, scaling, ctypes.byref(out.struct),
+                                    _ptr(ws), 0 if ws is None else ws.numel(), _stream()))
+    return out
+
+
+def lora_adamw_step(tensors, lr: float, beta1: float = 0.9, beta2: float = 0.999, eps: float = 1e-8,
+                    weight_decay: float = 0.0, step: int = 1) -> None:
+    """One AdamW update, in place, of adapter tensors given as tuples
+    (master fp32, param bf16 or None, grad bf16, m fp32, v fp32), all
+    contiguous CUDA tensors of one size per tuple."""
+    arr = (AdamwTensorStruct * max(1, len(tensors)))()
+    for i, (master, param, grad, m, v) in enumerate(tensors):
+        n = master.numel()
+        for t, dt, name in ((master, torch.float32, "master"), (grad, torch.bfloat16, "grad"),
+                            (m, torch.float32, "m"), (v, torch.float32, "v"), (param, torch.bfloat16, "param")):
+            if t is None and name == "param":
+                continue
+            if t.dtype != dt or not t.is_cuda or not t.is_contiguous() or t.numel() != n:
+                raise ValueError("tensor %d: %s must be a contiguous %s CUDA tensor of %d elements"
+                                 % (i, name, dt, n))
+        arr[i] = AdamwTensorStruct(master.data_ptr(), None if param is None else param.data_ptr(),
+                                   grad.data_ptr(), m.data_ptr(), v.data_ptr(), n)
+    h = AdamwHparamsStruct(lr, beta1, beta2, eps, weight_decay, step)
+    _check(lib.lora_adamw_step(arr, len(tensors), ctypes.byref(h), _stream()))
 
 
 def device_status() -> None:

@@ -247,6 +247,115 @@ int qlora_linear_bwd(const nf4_tensor* w, const uint16_t* A, const uint16_t* B, 
 
 const char* nf4lora_last_error_string(void) { return t_last_error.c_str(); }
 
+size_t nf4_merge_workspace_bytes(int64_t d_out, int64_t d_in) {
+    if (!valid_weight_shape(d_out, d_in)) return 0;
+    return static_cast<size_t>(align256(d_out * d_in * 4) + quant_ws_bytes(d_out, d_in));
+}
+
+static int check_merge_args(const nf4_tensor* w, const uint16_t* A, const uint16_t* B, int r, float scaling) {
+    int rc = check_tensor(w);
+    if (rc) return rc;
+    if (r < 1 || r > 256) return fail(NF4_ERR_INVALID_ARG, "r = %d outside [1, 256]", r);
+    if (!std::isfinite(scaling)) return fail(NF4_ERR_INVALID_ARG, "scaling is not finite");
+    if (!A || !B) return fail(NF4_ERR_INVALID_ARG, "A or B is NULL");
+    if (!aligned16(A) || !aligned16(B)) return fail(NF4_ERR_MISALIGNED, "A or B not 16-byte aligned");
+    return NF4_OK;
+}
+
+int nf4_merge_lora(const nf4_tensor* w, const uint16_t* A, const uint16_t* B, int r, float scaling, float* W_merged,
+                   void* stream) {
+    int rc = check_merge_args(w, A, B, r, scaling);
+    if (rc) return rc;
+    if (W_merged == nullptr) return fail(NF4_ERR_INVALID_ARG, "W_merged is NULL");
+    if (!aligned16(W_merged)) return fail(NF4_ERR_MISALIGNED, "W_merged not 16-byte aligned");
+    int sms = 0;
+    rc = check_device(&sms);
+    if (rc) return rc;
+    const cudaError_t e = launch_merge_lora(w->codes, w->qscale, w->scale2, w->scale_mean, A, B, r, w->d_out, w->d_in,
+                                            scaling, W_merged, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(NF4_ERR_CUDA, "nf4_merge_lora launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+int nf4_merge_requantize(const nf4_tensor* w, const uint16_t* A, const uint16_t* B, int r, float scaling,
+                         const nf4_tensor* out, void* ws, size_t ws_bytes, void* stream) {
+    int rc = check_merge_args(w, A, B, r, scaling);
+    if (rc) return rc;
+    rc = check_tensor(out);
+    if (rc) return rc;
+    if (out->d_out != w->d_out || out->d_in != w->d_in)
+        return fail(NF4_ERR_INVALID_ARG, "out describes [%lld, %lld], the weight is [%lld, %lld]",
+                    (long long)out->d_out, (long long)out->d_in, (long long)w->d_out, (long long)w->d_in);
+    const int64_t n = w->d_out * w->d_in;
+    rc = check_ws(ws, ws_bytes, align256(n * 4) + quant_ws_bytes(w->d_out, w->d_in));
+    if (rc) return rc;
+    int sms = 0;
+    rc = check_device(&sms);
+    if (rc) return rc;
+    uint8_t* w8 = static_cast<uint8_t*>(ws);
+    float* merged = reinterpret_cast<float*>(w8);
+    float* absmax = reinterpret_cast<float*>(w8 + align256(n * 4));
+    double* tile_sums = reinterpret_cast<double*>(w8 + align256(n * 4) + align256(n / 64 * 4));
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = launch_merge_lora(w->codes, w->qscale, w->scale2, w->scale_mean, A, B, r, w->d_out, w->d_in,
+                                      scaling, merged, st);
+    if (e != cudaSuccess) return fail(NF4_ERR_CUDA, "nf4_merge_requantize launch: %s", cudaGetErrorString(e));
+    // the merged weight is complete before the encoder starts (an ordinary
+    // launch), so `out` may be `w` itself
+    e = launch_nf4_quantize(merged, n, out->codes, out->qscale, out->scale2, out->scale_mean, absmax, tile_sums, sms,
+                            st);
+    if (e != cudaSuccess) return fail(NF4_ERR_CUDA, "nf4_merge_requantize launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+int lora_adamw_step(const lora_adamw_tensor* tensors, int count, const lora_adamw_hparams* h, void* stream) {
+    if (tensors == nullptr || h == nullptr) return fail(NF4_ERR_INVALID_ARG, "tensors or hparams is NULL");
+    if (count < 1 || count > 1024) return fail(NF4_ERR_INVALID_ARG, "count %d outside [1, 1024]", count);
+    const double lr = h->lr, b1 = h->beta1, b2 = h->beta2, eps = h->eps, wd = h->weight_decay;
+    if (!(std::isfinite(lr) && lr >= 0.0) || !(b1 >= 0.0 && b1 < 1.0) || !(b2 >= 0.0 && b2 < 1.0) ||
+        !(std::isfinite(eps) && eps > 0.0) || !(std::isfinite(wd) && wd >= 0.0) || h->step < 1)
+        return fail(NF4_ERR_INVALID_ARG, "hyper-parameters out of range (lr >= 0, 0 <= beta < 1, eps > 0, "
+                                         "weight_decay >= 0, step >= 1)");
+    for (int i = 0; i < count; ++i) {
+        const lora_adamw_tensor& t = tensors[i];
+        if (t.n < 0) return fail(NF4_ERR_INVALID_ARG, "tensor %d: n < 0", i);
+        if (t.n == 0) continue;
+        if (!t.master || !t.grad || !t.m || !t.v) return fail(NF4_ERR_INVALID_ARG, "tensor %d: NULL pointer", i);
+        if (!aligned16(t.master) || !aligned16(t.grad) || !aligned16(t.m) || !aligned16(t.v) ||
+            (t.param && !aligned16(t.param)))
+            return fail(NF4_ERR_MISALIGNED, "tensor %d: pointer not 16-byte aligned", i);
+    }
+    int sms = 0;
+    int rc = check_device(&sms);
+    if (rc) return rc;
+    const double t = static_cast<double>(h->step);
+    AdamwConsts c;
+    c.decay = static_cast<float>(1.0 - lr * wd);
+    c.b1 = h->beta1;
+    c.omb1 = static_cast<float>(1.0 - b1);
+    c.b2 = h->beta2;
+    c.omb2 = static_cast<float>(1.0 - b2);
+    c.step_size = static_cast<float>(lr / (1.0 - std::pow(b1, t)));
+    c.inv_sqrt_bc2 = static_cast<float>(1.0 / std::sqrt(1.0 - std::pow(b2, t)));
+    c.eps = h->eps;
+    for (int i0 = 0; i0 < count; i0 += kAdamwMaxTensors) {
+        AdamwBatch b{};
+        for (int i = i0; i < count && b.count < kAdamwMaxTensors; ++i) {
+            const lora_adamw_tensor& src = tensors[i];
+            const int k = b.count++;
+            b.p[k] = src.master;
+            b.p16[k] = src.param;
+            b.g[k] = src.grad;
+            b.m[k] = src.m;
+            b.v[k] = src.v;
+            b.n[k] = src.n;
+        }
+        const cudaError_t e = launch_adamw(b, c, sms, static_cast<cudaStream_t>(stream));
+        if (e != cudaSuccess) return fail(NF4_ERR_CUDA, "lora_adamw_step launch: %s", cudaGetErrorString(e));
+    }
+    return ok();
+}
+
 int nf4lora_device_status(void* stream) {
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
         return fail(NF4_ERR_CUDA, "stream synchronisation failed: %s", cudaGetErrorString(cudaGetLastError()));

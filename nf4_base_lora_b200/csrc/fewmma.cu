@@ -35,7 +35,11 @@
 //
 // Launch overlap: the kernel releases its own dependents as soon as it starts
 // (the next layer call's rank-r kernel may then stage its factor rows while
-// this one runs), and asks L2 for the rows of B its extension will read.
+// this one runs), and asks L2 for the rows of B its extension will read.  It
+// reads the activations and the encoded weight before its own wait: the
+// rank-r kernel it depends on released it only after waiting for the kernel
+// before that, so every earlier write is complete; global loads go through
+// L2 (ld.global.cg), never a possibly stale L1 line.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -158,7 +162,7 @@ __global__ void __maxnreg__(96) k_few_fwd(const __grid_constant__ CUtensorMap ma
     float acc0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, acc1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     __syncthreads();
     cluster_arrive_relaxed();  // barriers initialised (made visible by the init fence)
-    const float mu = __ldg(a.scale_mean);
+    const float mu = __ldcg(a.scale_mean);
     volatile int* abort_flag = &s_abort;
 
     int seg_i = 0, issued_seg = 0, issued_nq = kb0 < kb1 ? nq_first : 0;
@@ -185,7 +189,7 @@ __global__ void __maxnreg__(96) k_few_fwd(const __grid_constant__ CUtensorMap ma
             xpc[p] = i - xt[p] * per;
             xv[p] = make_uint4(0, 0, 0, 0);
             if (xt[p] < M && xpc[p] < nb * 8)
-                xv[p] = __ldg(reinterpret_cast<const uint4*>(a.act + static_cast<int64_t>(xt[p]) * K + seg0 * 64) +
+                xv[p] = __ldcg(reinterpret_cast<const uint4*>(a.act + static_cast<int64_t>(xt[p]) * K + seg0 * 64) +
                               xpc[p]);
         }
         int qA[2], qB[2];
@@ -198,10 +202,10 @@ __global__ void __maxnreg__(96) k_few_fwd(const __grid_constant__ CUtensorMap ma
             const int64_t biA = static_cast<int64_t>(nA) * bpr + blk, biB = static_cast<int64_t>(nB) * bpr + blk;
             inA[it] = in && okA;
             inB[it] = in && okB;
-            qA[it] = inA[it] ? static_cast<int>(__ldg(a.qscale + biA)) : 0;
-            qB[it] = inB[it] ? static_cast<int>(__ldg(a.qscale + biB)) : 0;
-            aA[it] = inA[it] ? __ldg(a.scale2 + (biA >> 8)) : 0.0f;
-            aB[it] = inB[it] ? __ldg(a.scale2 + (biB >> 8)) : 0.0f;
+            qA[it] = inA[it] ? static_cast<int>(__ldcg(a.qscale + biA)) : 0;
+            qB[it] = inB[it] ? static_cast<int>(__ldcg(a.qscale + biB)) : 0;
+            aA[it] = inA[it] ? __ldcg(a.scale2 + (biA >> 8)) : 0.0f;
+            aB[it] = inB[it] ? __ldcg(a.scale2 + (biB >> 8)) : 0.0f;
         }
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
@@ -268,18 +272,18 @@ __global__ void __maxnreg__(96) k_few_fwd(const __grid_constant__ CUtensorMap ma
             const int j0 = ch * 16;
             const int jj = (j0 % a.r64) + 2 * q;  // column of B (same in both halves of T2)
             const bool lo_ok = jj < a.r, hi_ok = jj + 8 < a.r;
-            const uint32_t a0 = (okA && lo_ok) ? __ldg(reinterpret_cast<const uint32_t*>(bA + jj)) : 0u;
-            const uint32_t a1 = (okB && lo_ok) ? __ldg(reinterpret_cast<const uint32_t*>(bB + jj)) : 0u;
-            const uint32_t a2 = (okA && hi_ok) ? __ldg(reinterpret_cast<const uint32_t*>(bA + jj + 8)) : 0u;
-            const uint32_t a3 = (okB && hi_ok) ? __ldg(reinterpret_cast<const uint32_t*>(bB + jj + 8)) : 0u;
+            const uint32_t a0 = (okA && lo_ok) ? __ldcg(reinterpret_cast<const uint32_t*>(bA + jj)) : 0u;
+            const uint32_t a1 = (okB && lo_ok) ? __ldcg(reinterpret_cast<const uint32_t*>(bB + jj)) : 0u;
+            const uint32_t a2 = (okA && hi_ok) ? __ldcg(reinterpret_cast<const uint32_t*>(bA + jj + 8)) : 0u;
+            const uint32_t a3 = (okB && hi_ok) ? __ldcg(reinterpret_cast<const uint32_t*>(bB + jj + 8)) : 0u;
             const uint16_t* t0 = a.ext_act + static_cast<int64_t>(g) * 2 * a.r64 + j0 + 2 * q;
-            const uint32_t b0 = g < M ? __ldg(reinterpret_cast<const uint32_t*>(t0)) : 0u;
-            const uint32_t b1 = g < M ? __ldg(reinterpret_cast<const uint32_t*>(t0 + 8)) : 0u;
+            const uint32_t b0 = g < M ? __ldcg(reinterpret_cast<const uint32_t*>(t0)) : 0u;
+            const uint32_t b1 = g < M ? __ldcg(reinterpret_cast<const uint32_t*>(t0 + 8)) : 0u;
             mma_16816(acc0, a0, a1, a2, a3, b0, b1);
             if (two_halves) {
                 const uint16_t* t8 = t0 + 8 * 2 * a.r64;
-                const uint32_t c0 = g + 8 < M ? __ldg(reinterpret_cast<const uint32_t*>(t8)) : 0u;
-                const uint32_t c1 = g + 8 < M ? __ldg(reinterpret_cast<const uint32_t*>(t8 + 8)) : 0u;
+                const uint32_t c0 = g + 8 < M ? __ldcg(reinterpret_cast<const uint32_t*>(t8)) : 0u;
+                const uint32_t c1 = g + 8 < M ? __ldcg(reinterpret_cast<const uint32_t*>(t8 + 8)) : 0u;
                 mma_16816(acc1, a0, a1, a2, a3, c0, c1);
             }
         }
@@ -444,7 +448,7 @@ __global__ void __maxnreg__(112) k_few_dx(const __grid_constant__ CUtensorMap ma
             for (int e = 0; e < 4; ++e) acc[m][h][e] = 0.0f;
     __syncthreads();
     cluster_arrive_relaxed();  // barriers initialised (made visible by the init fence)
-    const float mu = __ldg(a.scale_mean);
+    const float mu = __ldcg(a.scale_mean);
     volatile int* abort_flag = &s_abort;
     uint8_t* my_tile = s_tiles + warp * kDxTileBytes;
     const uint32_t my_tile_u32 = smem_u32(my_tile);
@@ -469,7 +473,7 @@ __global__ void __maxnreg__(112) k_few_dx(const __grid_constant__ CUtensorMap ma
             const int i = tid + p * kThreads, t = per == 256 ? (i >> 8) : i / per, pc = i - t * per;
             const int n = 32 * sc0 + 4 * pc;
             yv[p] = make_uint2(0, 0);
-            if (t < M && n < N) yv[p] = __ldg(reinterpret_cast<const uint2*>(a.act + static_cast<int64_t>(t) * N + n));
+            if (t < M && n < N) yv[p] = __ldcg(reinterpret_cast<const uint2*>(a.act + static_cast<int64_t>(t) * N + n));
         }
         int qv[4];
         float a2v[4];
@@ -478,8 +482,8 @@ __global__ void __maxnreg__(112) k_few_dx(const __grid_constant__ CUtensorMap ma
             const int c = sc0 + rw + 8 * it, n = 32 * c + lane;
             const bool ok = c < sc1 && n < N && blk_ok;
             const int64_t bi = static_cast<int64_t>(n) * bpr + blk;
-            qv[it] = ok ? static_cast<int>(__ldg(a.qscale + bi)) : 0;
-            a2v[it] = ok ? __ldg(a.scale2 + (bi >> 8)) : 0.0f;
+            qv[it] = ok ? static_cast<int>(__ldcg(a.qscale + bi)) : 0;
+            a2v[it] = ok ? __ldcg(a.scale2 + (bi >> 8)) : 0.0f;
         }
 #pragma unroll
         for (int p = 0; p < 8; ++p) {
@@ -527,7 +531,7 @@ __global__ void __maxnreg__(112) k_few_dx(const __grid_constant__ CUtensorMap ma
         for (int i = tid; i < kTok * (2 * a.r64 / 4); i += kThreads) {
             const int t = i / (2 * a.r64 / 4), pc = i - t * (2 * a.r64 / 4);
             uint2 v = make_uint2(0, 0);
-            if (t < M) v = __ldg(reinterpret_cast<const uint2*>(a.ext_act + static_cast<int64_t>(t) * 2 * a.r64) + pc);
+            if (t < M) v = __ldcg(reinterpret_cast<const uint2*>(a.ext_act + static_cast<int64_t>(t) * 2 * a.r64) + pc);
             *reinterpret_cast<uint2*>(sY + t * vstride + 4 * pc) = v;
         }
         __syncthreads();
@@ -536,7 +540,7 @@ __global__ void __maxnreg__(112) k_few_dx(const __grid_constant__ CUtensorMap ma
             uint4* trow = reinterpret_cast<uint4*>(my_tile + lane * kDxTileStride);
             const uint4* arow = reinterpret_cast<const uint4*>(a.ext_w + static_cast<int64_t>(j) * K + 64 * blk);
 #pragma unroll
-            for (int k = 0; k < 8; ++k) trow[k] = (j < a.r && blk_ok) ? __ldg(arow + k) : make_uint4(0, 0, 0, 0);
+            for (int k = 0; k < 8; ++k) trow[k] = (j < a.r && blk_ok) ? __ldcg(arow + k) : make_uint4(0, 0, 0, 0);
             __syncwarp();
             dx_chunk_mma(acc, my_tile_u32, sY, vstride, 32 * c, lane, two_halves);
             __syncwarp();

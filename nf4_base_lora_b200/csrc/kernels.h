@@ -15,8 +15,35 @@ cudaError_t launch_nf4_dequantize(const uint8_t* codes, const int8_t* qscale, co
                                   const float* scale_mean, int64_t n, uint16_t* out, int num_sms,
                                   cudaStream_t stream);
 
-// Few-token (M <= 16) rank-r intermediates as bf16 hi | lo pairs; each
-// releases its dependent launch as soon as it starts.
+// AdamW step of up to kAdamwMaxTensors adapter tensors per launch (fp32
+// master p, bf16 copy p16 or NULL, bf16 gradient g, fp32 moments m, v; n
+// elements each; pointers 16-byte aligned).
+constexpr int kAdamwMaxTensors = 8;
+struct AdamwBatch {
+    float* p[kAdamwMaxTensors];
+    uint16_t* p16[kAdamwMaxTensors];
+    const uint16_t* g[kAdamwMaxTensors];
+    float* m[kAdamwMaxTensors];
+    float* v[kAdamwMaxTensors];
+    int64_t n[kAdamwMaxTensors];
+    int count;
+};
+// decay = 1 - lr wd; b1, omb1 = 1 - b1, b2, omb2 = 1 - b2;
+// step_size = lr / (1 - b1^t); inv_sqrt_bc2 = 1 / sqrt(1 - b2^t); eps.
+struct AdamwConsts {
+    float decay, b1, omb1, b2, omb2, step_size, inv_sqrt_bc2, eps;
+};
+cudaError_t launch_adamw(const AdamwBatch& b, const AdamwConsts& c, int num_sms, cudaStream_t stream);
+
+// W'[N, K] fp32 = fp32(W_hat + s B A) from an encoded weight and the adapter
+// (rank sum in fp64, ascending j).
+cudaError_t launch_merge_lora(const uint8_t* codes, const int8_t* qscale, const float* scale2,
+                              const float* scale_mean, const uint16_t* A, const uint16_t* B, int r, int64_t N,
+                              int64_t K, float s, float* out, cudaStream_t stream);
+
+// Few-token (M <= 16) rank-r intermediates as bf16 hi | lo pairs; each is a
+// programmatic dependent of the kernel before it and releases its own
+// dependent once it has waited for that kernel.
 cudaError_t launch_few_down(const uint16_t* X, const uint16_t* A, int M, int K, int r, int r64, float s,
                             uint16_t* T2, float* T_saved, cudaStream_t stream);
 cudaError_t launch_few_v(const uint16_t* dY, const uint16_t* B, int M, int N, int r, int r64, float s,

@@ -21,110 +21,185 @@ namespace {
 
 constexpr int kTileBlocks = 256;  // = one double-quantisation group
 
-// Code of x: the number of thresholds m_j (ascending, j = 0..14) strictly
-// below x, by a 4-step binary search over the thresholds held in shared memory
-// (m[15] = +inf pads the table).
-__device__ __forceinline__ uint32_t nf4_code(float x, const float* m) {
-    uint32_t i = (x > m[7]) ? 8u : 0u;
-    i += (x > m[i + 3]) ? 4u : 0u;
-    i += (x > m[i + 1]) ? 2u : 0u;
-    i += (x > m[i]) ? 1u : 0u;
-    return i;
+// The pairwise tree over the 32 lanes' values (level l adds lane pairs
+// 2^l apart within aligned runs): lane 0 returns the sum of the run.
+__device__ __forceinline__ double pairwise_warp(double v) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const double u = __shfl_down_sync(0xffffffffu, v, o);
+        if ((threadIdx.x & (2 * o - 1)) == 0) v = __dadd_rn(v, u);
+    }
+    return v;
 }
 
-__global__ void __launch_bounds__(256) k_nf4_encode(const float* __restrict__ W, int64_t n_blocks,
+// Code of x = w / a (IEEE fp32 division): the number of thresholds m_j
+// (ascending, j = 0..14, m_j = (level_j + level_j+1) / 2) strictly below x.
+__device__ __noinline__ uint32_t nf4_code_exact(float w, float a, const float* m) {
+    const float x = __fdiv_rn(w, a);
+    uint32_t c = 0;
+#pragma unroll
+    for (int j = 0; j < 15; ++j) c += x > m[j] ? 1u : 0u;
+    return c;
+}
+
+// The same code without the division, for a normal absmax a: x' = w * fl(1/a)
+// lies within 2 ulp of fl(w / a).  Bucket b (0..31) covers [-1 + b/16,
+// -1 + (b+1)/16): the thresholds are more than 1/16 apart and none lies within
+// 1e-3 of a bucket edge, so each bucket holds at most one threshold (thr, else
+// +inf) above `base` others, and base + (x > thr) is the code of every x in the
+// bucket or within rounding distance of it.  The bucket index is
+// floor(16 x' + 16): one fused multiply-add adds 1.5 * 2^23 + 16 (an integer,
+// exact in fp32, where the fp32 spacing is 1) and rounds toward -inf, so the
+// low bits of the result are exactly that floor; -1 and 32, reachable only by
+// rounding at x' = -1 and +1, index copies of buckets 0 and 31 (table entries
+// 63 and 32).
+// Where x' falls within 1e-6 of the bucket's threshold the exact division
+// decides, so the result is always the code of fl(w / a).
+struct Bucket {
+    float thr;
+    uint32_t base;
+};
+
+__device__ __forceinline__ uint32_t nf4_code_fast(float w, float rinv, const Bucket* bkt, bool& unsure) {
+    const float xa = __fmul_rn(w, rinv);
+    static_assert(12582928.0f == 12582928.0, "1.5 * 2^23 + 16 is exact in fp32");
+    const int b = __float_as_int(__fmaf_rd(xa, 16.0f, 12582928.0f)) & 63;
+    const Bucket e = bkt[b];
+    unsure |= fabsf(__fsub_rn(xa, e.thr)) <= 1.0e-6f;
+    return e.base + (xa > e.thr ? 1u : 0u);
+}
+
+// Four lanes per 64-block: lane s of the group holds the 16-byte pieces
+// s, s + 4, s + 8, s + 12 (elements 4 (s + 4k) .. + 3), so each load
+// instruction of a warp reads eight whole 64-byte runs, and the absmax needs
+// two shuffle levels.  A warp takes eight blocks per step, a CTA of 8 warps
+// one tile of 256 blocks in four steps.
+__global__ void __launch_bounds__(256, 3) k_nf4_encode(const float* __restrict__ W, int64_t n_blocks,
                                                    uint8_t* __restrict__ codes,
                                                    float* __restrict__ absmax,
                                                    double* __restrict__ tile_sums) {
     __shared__ float s_mid[16];
+    __shared__ Bucket s_bkt[64];
     __shared__ double s_sum[kTileBlocks];
     const int tid = threadIdx.x;
+    pdl_launch_dependents();  // the mean kernel may take an SM as soon as one frees; it waits for this grid
     if (tid < 15) {
         s_mid[tid] = __fmul_rn(__fadd_rn(nf4_level(tid), nf4_level(tid + 1)), 0.5f);
-    } else if (tid == 15) {
-        s_mid[15] = __int_as_float(0x7f800000);
+    } else if (tid >= 64 && tid < 128) {
+        const int idx = tid - 64;
+        const int bi = idx < 32 ? idx : (idx == 32 ? 31 : 0);  // 32: rounding above +1; 63: below -1
+        const float lo = -1.0f + 0.0625f * static_cast<float>(bi), hi = lo + 0.0625f;
+        Bucket e{__int_as_float(0x7f800000), 0u};
+        for (int j = 0; j < 15; ++j) {
+            const float m = __fmul_rn(__fadd_rn(nf4_level(j), nf4_level(j + 1)), 0.5f);
+            if (m < lo) ++e.base;
+            else if (m < hi) e.thr = m;
+        }
+        s_bkt[idx] = e;
     }
     __syncthreads();
     const int lane = tid & 31, warp = tid >> 5;
-    const int half = lane >> 4, sub = lane & 15;
+    const int grp = lane >> 2, sub = lane & 3;
     const int64_t n_tiles = (n_blocks + kTileBlocks - 1) / kTileBlocks;
 
     for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
-        // warp w owns blocks [32w, 32w + 32) of the tile, two per step
-#pragma unroll 4
-        for (int it = 0; it < 16; ++it) {
-            const int local = warp * 32 + it * 2 + half;
+#pragma unroll 2
+        for (int it = 0; it < 4; ++it) {
+            const int local = warp * 32 + it * 8 + grp;
             const int64_t b = tile * kTileBlocks + local;
-            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
             const bool valid = b < n_blocks;
-            if (valid) v = __ldcs(reinterpret_cast<const float4*>(W + b * 64) + sub);
-            float a = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+            float v[16];
 #pragma unroll
-            for (int o = 8; o >= 1; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-            uint32_t c0 = 7, c1 = 7, c2 = 7, c3 = 7;
+            for (int k = 0; k < 4; ++k) {
+                float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (valid) q = __ldcs(reinterpret_cast<const float4*>(W + b * 64) + sub + 4 * k);
+                v[4 * k] = q.x;
+                v[4 * k + 1] = q.y;
+                v[4 * k + 2] = q.z;
+                v[4 * k + 3] = q.w;
+            }
+            float a = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(v[i]));
+            a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+            a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+            uint32_t c[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) c[i] = 7;
             if (a != 0.0f) {
-                c0 = nf4_code(__fdiv_rn(v.x, a), s_mid);
-                c1 = nf4_code(__fdiv_rn(v.y, a), s_mid);
-                c2 = nf4_code(__fdiv_rn(v.z, a), s_mid);
-                c3 = nf4_code(__fdiv_rn(v.w, a), s_mid);
+                bool unsure = !(a >= 1.0e-37f);  // fl(1/a) not finite or not normal: exact division
+                if (!unsure) {
+                    const float rinv = __frcp_rn(a);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) c[i] = nf4_code_fast(v[i], rinv, s_bkt, unsure);
+                }
+                if (unsure) {  // rare: near a threshold, or a tiny absmax
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) c[i] = nf4_code_exact(v[i], a, s_mid);
+                }
             }
             if (valid) {
-                // byte k holds (even element << 4) | odd element
-                const uint16_t packed =
-                    static_cast<uint16_t>(((c0 << 4) | c1) | (((c2 << 4) | c3) << 8));
-                reinterpret_cast<uint16_t*>(codes + b * 32)[sub] = packed;
+                // piece p = sub + 4k holds elements 4p .. 4p + 3: code bytes 2p, 2p + 1
+                // (byte = (even element << 4) | odd element)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint32_t packed = (c[4 * k] << 4) | c[4 * k + 1] | (((c[4 * k + 2] << 4) | c[4 * k + 3]) << 8);
+                    reinterpret_cast<uint16_t*>(codes + b * 32)[sub + 4 * k] = static_cast<uint16_t>(packed);
+                }
                 if (sub == 0) absmax[b] = a;
             }
             if (sub == 0) s_sum[local] = valid ? static_cast<double>(a) : 0.0;
         }
         __syncthreads();
         // fp64 pairwise tree over the tile's 256 scales (zero-padded: x + 0 == x
-        // keeps the carried-up elements of a short tail unchanged)
-        for (int stride = 1; stride < kTileBlocks; stride <<= 1) {
-            const int idx = tid * 2 * stride;
-            if (idx < kTileBlocks) s_sum[idx] = __dadd_rn(s_sum[idx], s_sum[idx + stride]);
-            __syncthreads();
+        // keeps the carried-up elements of a short tail unchanged): five levels
+        // inside each warp's aligned run of 32, three over the eight warp sums
+        double t = pairwise_warp(s_sum[tid]);
+        __syncthreads();  // every s_sum read before warp 0's lanes reuse it
+        if (lane == 0) s_sum[warp] = t;
+        __syncthreads();
+        if (warp == 0) {
+            t = pairwise_warp(lane < 8 ? s_sum[lane] : 0.0);
+            if (lane == 0) tile_sums[tile] = t;
         }
-        if (tid == 0) tile_sums[tile] = s_sum[0];
         __syncthreads();
     }
 }
 
-// One CTA: pairwise tree over the tile sums (zero-padded to a power of two,
-// processed in aligned segments of 2048), then mean = fp32(sum / n_b).
+// The pairwise tree over src[0 .. 2048) (entries at or beyond `count` read as
+// zero) by 1024 threads: level 1 in each thread, five in each warp, five in
+// warp 0 over the 32 warp sums.  Returns the sum in thread 0.
+__device__ __forceinline__ double pairwise_2048(const double* src, int64_t count, double* s_w) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const double x0 = 2 * tid < count ? src[2 * tid] : 0.0;
+    const double x1 = 2 * tid + 1 < count ? src[2 * tid + 1] : 0.0;
+    double v = pairwise_warp(__dadd_rn(x0, x1));
+    if (lane == 0) s_w[warp] = v;
+    __syncthreads();
+    if (warp == 0) v = pairwise_warp(s_w[lane]);
+    __syncthreads();  // s_w is free again
+    return v;
+}
+
+// One CTA of 1024 threads: the pairwise tree over the tile sums (zero-padded
+// to a power of two, in aligned segments of 2048, then over the segment sums),
+// then mean = fp32(sum / n_b).
 __global__ void __launch_bounds__(1024) k_dq_mean(const double* __restrict__ tile_sums,
                                                   int64_t n_tiles, int64_t n_blocks,
                                                   float* __restrict__ mean_out) {
     constexpr int kSeg = 2048;
-    __shared__ double s[kSeg];
+    __shared__ double s_w[32];
     __shared__ double s_segs[kSeg];
-    const int tid = threadIdx.x;
     const int64_t n_segs = (n_tiles + kSeg - 1) / kSeg;  // <= kSeg for any supported size
+    pdl_wait();                // the encoder's tile sums (and absmax) are complete and visible
+    pdl_launch_dependents();   // so the scale quantiser may start and load the absmax values
     for (int64_t seg = 0; seg < n_segs; ++seg) {
-        for (int i = tid; i < kSeg; i += blockDim.x) {
-            const int64_t g = seg * kSeg + i;
-            s[i] = g < n_tiles ? tile_sums[g] : 0.0;
-        }
-        __syncthreads();
-        for (int stride = 1; stride < kSeg; stride <<= 1) {
-            for (int idx = tid * 2 * stride; idx < kSeg; idx += blockDim.x * 2 * stride)
-                s[idx] = __dadd_rn(s[idx], s[idx + stride]);
-            __syncthreads();
-        }
-        if (tid == 0) s_segs[seg] = s[0];
-        __syncthreads();
+        const double v = pairwise_2048(tile_sums + seg * kSeg, n_tiles - seg * kSeg, s_w);
+        if (threadIdx.x == 0) s_segs[seg] = v;
     }
-    for (int i = tid; i < kSeg; i += blockDim.x)
-        if (i >= n_segs) s_segs[i] = 0.0;
     __syncthreads();
-    int width = 1;
-    while (width < n_segs) width <<= 1;
-    for (int stride = 1; stride < width; stride <<= 1) {
-        for (int idx = tid * 2 * stride; idx < width; idx += blockDim.x * 2 * stride)
-            s_segs[idx] = __dadd_rn(s_segs[idx], s_segs[idx + stride]);
-        __syncthreads();
-    }
-    if (tid == 0) *mean_out = __double2float_rn(__ddiv_rn(s_segs[0], static_cast<double>(n_blocks)));
+    const double total = pairwise_2048(s_segs, n_segs, s_w);
+    if (threadIdx.x == 0) *mean_out = __double2float_rn(__ddiv_rn(total, static_cast<double>(n_blocks)));
 }
 
 // One warp per group of 256 first-level scales; lane l owns scales
@@ -138,16 +213,27 @@ __global__ void __launch_bounds__(256) k_dq_quantize(const float* __restrict__ a
     const int64_t g = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int64_t n_groups = (n_blocks + kTileBlocks - 1) / kTileBlocks;
     if (g >= n_groups) return;
-    const float mu = *mean_ptr;
     const int64_t b0 = g * kTileBlocks + lane * 8;
+    // the absmax values were written by the encoder, which had finished before
+    // the mean kernel released this one; the mean itself needs the wait
+    float x[8];
+    if (b0 + 8 <= n_blocks) {
+        const float4 u0 = __ldcg(reinterpret_cast<const float4*>(absmax + b0));
+        const float4 u1 = __ldcg(reinterpret_cast<const float4*>(absmax + b0) + 1);
+        x[0] = u0.x; x[1] = u0.y; x[2] = u0.z; x[3] = u0.w;
+        x[4] = u1.x; x[5] = u1.y; x[6] = u1.z; x[7] = u1.w;
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[i] = b0 + i < n_blocks ? __ldcg(absmax + b0 + i) : 0.0f;
+    }
+    pdl_wait();
+    const float mu = *mean_ptr;
     float d[8];
     float m = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int64_t b = b0 + i;
-        d[i] = b < n_blocks ? __fsub_rn(absmax[b], mu) : 0.0f;
-        m = fmaxf(m, fabsf(d[i]));
-    }
+    for (int i = 0; i < 8; ++i) d[i] = b0 + i < n_blocks ? __fsub_rn(x[i], mu) : 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(d[i]));
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     if (lane == 0) scale2[g] = m;
@@ -217,12 +303,22 @@ static cudaLaunchConfig_t config(int64_t grid, int block, cudaStream_t stream) {
     return cfg;
 }
 
+// A programmatic dependent of the kernel before it on the stream (it waits
+// for that kernel with griddepcontrol.wait before reading its results).
+static cudaLaunchAttribute g_pdl_attr = [] {
+    cudaLaunchAttribute a{};
+    a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    a.val.programmaticStreamSerializationAllowed = 1;
+    return a;
+}();
+
 cudaError_t launch_nf4_quantize(const float* W, int64_t n, uint8_t* codes, int8_t* qscale,
                                 float* scale2, float* scale_mean, float* ws_absmax,
                                 double* ws_tile_sums, int num_sms, cudaStream_t stream) {
     const int64_t n_blocks = n / 64;
     const int64_t n_tiles = (n_blocks + kTileBlocks - 1) / kTileBlocks;
-    const int64_t grid1 = n_tiles < int64_t(num_sms) * 8 ? n_tiles : int64_t(num_sms) * 8;
+    // three CTAs per SM (at most 85 registers a thread): every CTA resident at once
+    const int64_t grid1 = n_tiles < int64_t(num_sms) * 3 ? n_tiles : int64_t(num_sms) * 3;
     cudaError_t e;
     {
         TraceScope trace("nf4_encode", stream);
@@ -233,6 +329,8 @@ cudaError_t launch_nf4_quantize(const float* W, int64_t n, uint8_t* codes, int8_
     {
         TraceScope trace("dq_mean", stream);
         cudaLaunchConfig_t cfg = config(1, 1024, stream);
+        cfg.attrs = &g_pdl_attr;
+        cfg.numAttrs = 1;
         e = cudaLaunchKernelEx(&cfg, k_dq_mean, static_cast<const double*>(ws_tile_sums), n_tiles, n_blocks,
                                scale_mean);
         if (e != cudaSuccess) return e;
@@ -240,6 +338,8 @@ cudaError_t launch_nf4_quantize(const float* W, int64_t n, uint8_t* codes, int8_
     {
         TraceScope trace("dq_quantize", stream);
         cudaLaunchConfig_t cfg = config((n_tiles + 7) / 8, 256, stream);
+        cfg.attrs = &g_pdl_attr;
+        cfg.numAttrs = 1;
         e = cudaLaunchKernelEx(&cfg, k_dq_quantize, static_cast<const float*>(ws_absmax), n_blocks,
                                static_cast<const float*>(scale_mean), qscale, scale2);
     }

@@ -276,3 +276,57 @@ def lora_grads(A, B, X, dY, scaling: float):
 def trainable_parameters(d_in: int, d_out: int, r: int) -> int:
     """Entries of A and B, the only trainable tensors of the layer."""
     return r * d_in + d_out * r
+
+
+# ---------------------------------------------------------------- the adapter's optimizer step
+def adamw_step(p, g, m, v, step: int, lr: float, beta1: float = 0.9, beta2: float = 0.999,
+               eps: float = 1e-8, weight_decay: float = 0.0):
+    """One AdamW update of a trainable tensor (the adapter A or B), in fp64.
+
+    "第 04 篇：QLoRA 原理" §7.3 and §8.3 keep two fp32 moments per trainable
+    parameter (first m, second v) and optionally a separate master copy of
+    the parameter; the pages print no update rule, so this is the decoupled
+    weight-decay AdamW of Loshchilov and Hutter with bias-corrected moments
+    (t = step, counted from 1):
+
+        p <- p (1 - lr wd)
+        m <- b1 m + (1 - b1) g
+        v <- b2 v + (1 - b2) g^2
+        p <- p - lr / (1 - b1^t) * m / (sqrt(v) / sqrt(1 - b2^t) + eps)
+
+    Returns the new (p, m, v) as fp64 arrays."""
+    p, g, m, v = map(_f64, (p, g, m, v))
+    if step < 1:
+        raise ValueError("step counts from 1")
+    p = p * (1.0 - lr * weight_decay)
+    m = beta1 * m + (1.0 - beta1) * g
+    v = beta2 * v + (1.0 - beta2) * g * g
+    bc1 = 1.0 - beta1 ** step
+    bc2 = 1.0 - beta2 ** step
+    p = p - (lr / bc1) * m / (np.sqrt(v) / np.sqrt(bc2) + eps)
+    return p, m, v
+
+
+# ---------------------------------------------------------------- adapter merge
+def merge_lora(W_hat, A, B, scaling: float) -> np.ndarray:
+    """The merged weight fp32(W_hat + s B A) ("第 04 篇：QLoRA 原理" §12.3: merge
+    the adapter into the base, W + s B A, for deployment; §12.4: the effective
+    weight of QLoRA is the dequantised base plus the adapter).
+
+    W_hat is the bf16 dequantised base ([d_out, d_in]; the fp32 original is
+    not kept), A [r, d_in], B [d_out, r] bf16.  Each product B[n, j] A[j, k]
+    of two bf16 values is exact in fp64; the rank-r sum is taken in fp64 in
+    ascending j, then multiplied by s (fp32) and added to W_hat, each in fp64
+    and rounded once, and the result is rounded to fp32 (to nearest even)."""
+    W_hat, A, B = map(_f64, (W_hat, A, B))
+    acc = np.zeros(W_hat.shape, np.float64)
+    for j in range(A.shape[0]):
+        acc = acc + B[:, j:j + 1] * A[j:j + 1, :]
+    s = np.float64(np.float32(scaling))
+    return (W_hat + s * acc).astype(np.float32)
+
+
+def merge_requantize(qt: Dict[str, np.ndarray], shape, A, B, scaling: float) -> Dict[str, np.ndarray]:
+    """§12.3's deployment path: the merged weight encoded again with the same
+    NF4 + double quantisation (a second rounding of the weight)."""
+    return quantize(merge_lora(dequantize(qt, shape), A, B, scaling))

@@ -118,6 +118,28 @@ def test_host_validation_without_device(nf):
     assert L.nf4_dequantize(None, Y, None) == -1
 
 
+def test_adamw_host_validation_without_device(nf):
+    L = nf.lib
+    T = nf.AdamwTensorStruct
+    h = nf.AdamwHparamsStruct(1e-3, 0.9, 0.999, 1e-8, 0.0, 1)
+    good = (T * 1)(T(1 << 24, None, 1 << 25, 1 << 26, 1 << 27, 64))
+    assert L.lora_adamw_step(good, 0, ctypes.byref(h), None) == -1          # count
+    assert L.lora_adamw_step(None, 1, ctypes.byref(h), None) == -1          # no tensors
+    assert L.lora_adamw_step(good, 1, None, None) == -1                     # no hyper-parameters
+    bad = (T * 1)(T(1 << 24, None, None, 1 << 26, 1 << 27, 64))
+    assert L.lora_adamw_step(bad, 1, ctypes.byref(h), None) == -1           # NULL gradient
+    mis = (T * 1)(T((1 << 24) + 4, None, 1 << 25, 1 << 26, 1 << 27, 64))
+    assert L.lora_adamw_step(mis, 1, ctypes.byref(h), None) == -3           # misaligned master
+    neg = (T * 1)(T(1 << 24, None, 1 << 25, 1 << 26, 1 << 27, -1))
+    assert L.lora_adamw_step(neg, 1, ctypes.byref(h), None) == -1           # n < 0
+    for hp in [(1e-3, 1.0, 0.999, 1e-8, 0.0, 1), (1e-3, 0.9, 0.999, 0.0, 0.0, 1),
+               (-1e-3, 0.9, 0.999, 1e-8, 0.0, 1), (1e-3, 0.9, 0.999, 1e-8, 0.0, 0),
+               (float("nan"), 0.9, 0.999, 1e-8, 0.0, 1), (1e-3, 0.9, 0.999, 1e-8, -0.1, 1)]:
+        bh = nf.AdamwHparamsStruct(*hp)
+        assert L.lora_adamw_step(good, 1, ctypes.byref(bh), None) == -1, hp
+    assert b"hyper-parameters" in L.nf4lora_last_error_string()
+
+
 def test_workspace_grows_with_tokens(nf):
     a = nf.qlora_fwd_workspace_bytes(16, 4096, 4096, 64)
     b = nf.qlora_fwd_workspace_bytes(4096, 4096, 4096, 64)

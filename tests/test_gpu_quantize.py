@@ -53,6 +53,39 @@ def test_quantize_constant_weight(nf):
     assert np.all(dev.qscale.cpu().numpy() == 0)
 
 
+def near_threshold_blocks(n_blocks: int = 256, seed: int = 11) -> np.ndarray:
+    """[n_blocks / 4, 256] fp32: each 64-block attains its absmax a (random,
+    some powers of two) at element 0 and puts w = fl(m_j a) moved by -2..+1
+    ulp for every threshold m_j (j = 0..14) in the rest, half the blocks
+    negated: fl(w / a) then lands on or within a few ulp of the thresholds,
+    where the encoder's division-free test hands over to the exact division."""
+    rng = np.random.default_rng(seed)
+    m = oracle.midpoints().astype(np.float32)
+    out = np.zeros((n_blocks, 64), np.float32)
+    for b in range(n_blocks):
+        a = np.float32(2.0 ** rng.integers(-8, 3)) if b % 4 == 0 else np.float32(rng.uniform(0.003, 4.0))
+        blk = [a]
+        for j in range(15):
+            w = np.float32(m[j] * a)
+            for step in (-2, -1, 0, 1):
+                v = w
+                for _ in range(abs(step)):
+                    v = np.nextafter(v, np.float32(np.copysign(np.inf, step)))
+                blk.append(np.float32(v))
+        blk += list(rng.uniform(-1, 1, 64 - len(blk)).astype(np.float32) * a)
+        out[b] = np.array(blk, np.float32)
+        assert np.max(np.abs(out[b])) == a
+        if b % 2:
+            out[b] = -out[b]
+    return out.reshape(n_blocks // 4, 256)
+
+
+def test_quantize_near_thresholds_bit_exact(nf):
+    w = near_threshold_blocks()
+    qt, dev = encode_both(nf, w)
+    assert_encoding_equal(qt, dev)
+
+
 @pytest.mark.parametrize("d_out,d_in", [(4096, 4096), (11008, 4096)])
 def test_quantize_llama_shapes_bit_exact(nf, d_out, d_in):
     w = workloads.weight(d_out, d_in, outliers=True, index=1)

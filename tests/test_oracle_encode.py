@@ -117,3 +117,15 @@ def test_pack_order_and_unpack():
     packed = oracle.pack(codes)
     assert list(packed) == [0x12, 0x3F, 0x07, 0x90]
     assert np.array_equal(oracle.unpack(packed, 7), codes)
+
+
+def test_thresholds_fit_sixteenth_buckets():
+    """The spacing the GPU encoder's division-free code search relies on:
+    consecutive thresholds are more than 1/16 apart (so a bucket
+    [-1 + b/16, -1 + (b+1)/16) holds at most one) and none lies within 1e-3 of
+    a bucket edge (so rounding x by a few ulp never moves it past a threshold
+    when it moves it to the next bucket)."""
+    m = oracle.midpoints().astype(np.float64)
+    assert np.all(np.diff(m) > 1.0 / 16)
+    edges = -1.0 + np.arange(33) / 16.0
+    assert np.min(np.abs(m[:, None] - edges[None, :])) >= 1e-3
