@@ -126,6 +126,21 @@ def load_traffic(kernel, workload):
     return None
 
 
+def load_traffic_per_weight(kernel):
+    """DRAM bytes per weight of a kernel whose traffic grows in proportion to
+    the weights it processes (the encoder, the merge), from a capture of a
+    smaller case, under the same source-hash rule."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            e = json.load(f).get("per_weight", {}).get(kernel)
+        if e and e.get("source_hash") == kernel_source_hash():
+            return float(e["bytes_per_weight"])
+    except Exception:
+        pass
+    return None
+
+
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -411,8 +426,10 @@ def time_quantize(nf, gw, args, stream, device, world, hbm_peak, peak_src):
            "kernels": {k: {"launches": len(v), "avg_us": sum(v) / len(v) * 1e3} for k, v in sorted(per_kernel.items())}}
     if enc_ms > 0:
         achieved = enc_bytes / (enc_ms * 1e-3) / 1e9
+        bpw = load_traffic_per_weight("nf4_encode")
         out["roofline"] = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                            "frac": achieved / hbm_peak, "kernel": "nf4_encode",
+                           "traffic": None if bpw is None else bpw * weights / len(wl.modules),
                            "algorithmic": "4n read + n/2 written per launch (fp32 weight in, packed codes out)",
                            "peak_source": peak_src + " (hbm_gbs)"}
     return out
@@ -524,8 +541,10 @@ def time_merge(nf, gw, args, stream, device, world, clocks_mhz=1965.0):
     mk = per_kernel.get("nf4_merge_lora")
     if mk:
         achieved = flops / (sum(mk) * 1e-3) / 1e12
+        bpw = load_traffic_per_weight("nf4_merge_lora")
         out["roofline"] = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s (fp64)",
                            "frac": achieved / peak, "kernel": "nf4_merge_lora",
+                           "traffic": None if bpw is None else bpw * weights / len(wl.modules),
                            "algorithmic": "2 n r fp64 flops per module (the rank-r sum of each merged weight)",
                            "peak_source": "derived: %d SMs x %d fp64 FMA/clk x 2 x %.0f MHz"
                                           % (gw.sms, FP64_FMA_PER_CLK_PER_SM, clocks_mhz)}
