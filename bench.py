@@ -98,12 +98,14 @@ def load_peaks():
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
 
 
-def kernel_source_hash():
-    """Hash of every CUDA source of the library (a traffic figure is used only
-    while the kernels are the ones it was measured on)."""
+def kernel_source_hash(files=None):
+    """Hash of the CUDA sources a kernel is built from (all of the library's
+    when `files` is None): a traffic figure is used only while the kernel is
+    the one it was measured on."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "nf4_base_lora_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    names = sorted(files) if files else sorted(os.listdir(csrc))
+    for name in names:
         if name.endswith((".cu", ".cuh", ".h")):
             with open(os.path.join(csrc, name), "rb") as f:
                 h.update(name.encode())
@@ -119,7 +121,7 @@ def load_traffic(kernel, workload):
         with open(path) as f:
             t = json.load(f)
         e = t.get(workload, {}).get(kernel)
-        if e and e.get("source_hash") == kernel_source_hash():
+        if e and e.get("source_hash") == kernel_source_hash(e.get("sources")):
             return float(e["bytes_per_launch"])
     except Exception:
         pass
@@ -134,7 +136,7 @@ def load_traffic_per_weight(kernel):
     try:
         with open(path) as f:
             e = json.load(f).get("per_weight", {}).get(kernel)
-        if e and e.get("source_hash") == kernel_source_hash():
+        if e and e.get("source_hash") == kernel_source_hash(e.get("sources")):
             return float(e["bytes_per_weight"])
     except Exception:
         pass
