@@ -12,6 +12,14 @@ enough encoded copies to exceed 4x the L2 cache, so every pass streams its
 weight from HBM.  Steps are replayed from CUDA graphs; the library's own
 launch tracing times the dominant kernel on the stream it runs on.
 
+Besides the step, the line carries the phases around it where the workload
+has them, each timed on its own with CUDA events: ``quantize`` (encoding of
+the fp32 weights, the LLaMA-65B workload), ``optimizer`` (the AdamW step of
+A and B after a full backward) and ``merge`` (the adapter folded into the
+base and re-encoded, the LLaMA-65B workload), each with its roofline.
+``--only quantize|merge|optimizer`` times one phase alone (a short command to
+profile).
+
 Rank 0 prints ONE JSON line.  With N > 1 (torchrun, one process per GPU)
 every rank runs the same per-GPU workload on its own data (weak scaling) and
 the time is the max over ranks.  A forward + input-gradient workload has no

@@ -14,7 +14,7 @@
 // The fp64 multiply-adds bound the kernel (n * r of them against 4.5 bytes
 // of memory traffic per weight).  A CTA computes a 128 x 64 tile of W': the
 // factor slices of 16 ranks at a time are staged in shared memory as fp64
-// (B transposed), and each thread keeps an 8 x 4 block of fp64 sums; the
+// (B transposed), and each thread keeps 8 rows x 4 columns of fp64 sums; the
 // epilogue decodes the tile's codes (one 64-block per row) and writes fp32
 // rows.
 #include <cuda_bf16.h>
@@ -51,7 +51,9 @@ __global__ void __launch_bounds__(256) k_merge_lora(const uint8_t* __restrict__ 
     const int64_t n0 = static_cast<int64_t>(blockIdx.y) * kMergeRows;
     const int64_t k0 = static_cast<int64_t>(blockIdx.x) * kMergeCols;
     const int rb = 16 * warp + 8 * ty;  // this thread's first row in the tile (8 rows)
-    const int cb = 4 * tx;              // this thread's first column (4 columns)
+    // this thread's columns: 2 tx, 2 tx + 1 and 32 + 2 tx, 33 + 2 tx, so that the
+    // 16-byte reads of eight consecutive lanes cover 128 contiguous bytes
+    const int cb = 2 * tx;
 
     double acc[8][4];
 #pragma unroll
@@ -68,14 +70,14 @@ __global__ void __launch_bounds__(256) k_merge_lora(const uint8_t* __restrict__ 
                                 : 0.0;
         }
         for (int i = tid; i < kMergeRanks * kMergeRows; i += 256) {
-            const int rr = i / kMergeRanks, jj = i % kMergeRanks;
+            const int jj = i / kMergeRows, rr = i % kMergeRows;  // consecutive lanes: consecutive rows (no conflicts)
             const int64_t n = n0 + rr;
             sB[jj][rr] = (jj < nj && n < N) ? static_cast<double>(bf16_bits_to_float(B[n * r + j0 + jj])) : 0.0;
         }
         __syncthreads();
         for (int jj = 0; jj < nj; ++jj) {
             const double2 a01 = *reinterpret_cast<const double2*>(&sA[jj][cb]);
-            const double2 a23 = *reinterpret_cast<const double2*>(&sA[jj][cb + 2]);
+            const double2 a23 = *reinterpret_cast<const double2*>(&sA[jj][32 + cb]);
             const double a[4] = {a01.x, a01.y, a23.x, a23.y};
             double b[8];
 #pragma unroll
@@ -101,16 +103,19 @@ __global__ void __launch_bounds__(256) k_merge_lora(const uint8_t* __restrict__ 
         if (n >= N) break;
         const int64_t bi = n * bpr + blk;
         const float sc = nf4_block_scale(qscale[bi], scale2[bi >> 8], mu);
-        // four codes: elements k0 + cb .. + 3 of row n, two bytes, the even element in the high nibble
-        const uint16_t two = *reinterpret_cast<const uint16_t*>(codes + (n * K + k0 + cb) / 2);
-        const uint32_t code[4] = {(two >> 4) & 15u, two & 15u, (two >> 12) & 15u, (two >> 8) & 15u};
+        // codes of elements k0 + cb, + 1 and k0 + 32 + cb, + 1 of row n: one byte
+        // each, the even element in the high nibble
+        const uint8_t* row = codes + (n * K + k0) / 2;
+        const uint32_t b0 = row[cb / 2], b1 = row[16 + cb / 2];
+        const uint32_t code[4] = {b0 >> 4, b0 & 15u, b1 >> 4, b1 & 15u};
         float o[4];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
             const float w_hat = __bfloat162float(__float2bfloat16_rn(__fmul_rn(s_lvl[code[c]], sc)));
             o[c] = __double2float_rn(__dadd_rn(static_cast<double>(w_hat), __dmul_rn(sd, acc[i][c])));
         }
-        *reinterpret_cast<float4*>(out + n * K + k0 + cb) = make_float4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<float2*>(out + n * K + k0 + cb) = make_float2(o[0], o[1]);
+        *reinterpret_cast<float2*>(out + n * K + k0 + 32 + cb) = make_float2(o[2], o[3]);
     }
 }
 

@@ -45,28 +45,29 @@ __device__ __noinline__ uint32_t nf4_code_exact(float w, float a, const float* m
 // The same code without the division, for a normal absmax a: x' = w * fl(1/a)
 // lies within 2 ulp of fl(w / a).  Bucket b (0..31) covers [-1 + b/16,
 // -1 + (b+1)/16): the thresholds are more than 1/16 apart and none lies within
-// 1e-3 of a bucket edge, so each bucket holds at most one threshold (thr, else
-// +inf) above `base` others, and base + (x > thr) is the code of every x in the
-// bucket or within rounding distance of it.  The bucket index is
+// 1e-3 of a bucket edge, so each bucket holds at most one threshold thr (if
+// none, take any value above 1) above `base` others, and base + (x > thr) is
+// the code of every x in the bucket or within rounding distance of it.  The bucket index is
 // floor(16 x' + 16): one fused multiply-add adds 1.5 * 2^23 + 16 (an integer,
 // exact in fp32, where the fp32 spacing is 1) and rounds toward -inf, so the
 // low bits of the result are exactly that floor; -1 and 32, reachable only by
 // rounding at x' = -1 and +1, index copies of buckets 0 and 31 (table entries
 // 63 and 32).
-// Where x' falls within 1e-6 of the bucket's threshold the exact division
-// decides, so the result is always the code of fl(w / a).
-struct Bucket {
-    float thr;
-    uint32_t base;
-};
-
-__device__ __forceinline__ uint32_t nf4_code_fast(float w, float rinv, const Bucket* bkt, bool& unsure) {
+// A table entry is one 32-bit word, so the 32 lanes of a warp never meet on a
+// bank unless they read the same entry: the fp32 threshold with its low four
+// mantissa bits replaced by `base` (a change of less than 16 ulp, under 1e-6
+// for |thr| < 1), or 2.0 with `base` in those bits for a bucket without one.
+// Where x' falls within 2e-6 of that value the exact division decides (the
+// true threshold is within 1e-6 of it and x' within 2.4e-7 of fl(w / a)), so
+// the result is always the code of fl(w / a).
+__device__ __forceinline__ uint32_t nf4_code_fast(float w, float rinv, const uint32_t* bkt, bool& unsure) {
     const float xa = __fmul_rn(w, rinv);
     static_assert(12582928.0f == 12582928.0, "1.5 * 2^23 + 16 is exact in fp32");
     const int b = __float_as_int(__fmaf_rd(xa, 16.0f, 12582928.0f)) & 63;
-    const Bucket e = bkt[b];
-    unsure |= fabsf(__fsub_rn(xa, e.thr)) <= 1.0e-6f;
-    return e.base + (xa > e.thr ? 1u : 0u);
+    const uint32_t e = bkt[b];
+    const float thr = __uint_as_float(e);
+    unsure |= fabsf(__fsub_rn(xa, thr)) <= 2.0e-6f;
+    return (e & 15u) + (xa > thr ? 1u : 0u);
 }
 
 // Four lanes per 64-block: lane s of the group holds the 16-byte pieces
@@ -79,7 +80,7 @@ __global__ void __launch_bounds__(256, 3) k_nf4_encode(const float* __restrict__
                                                    float* __restrict__ absmax,
                                                    double* __restrict__ tile_sums) {
     __shared__ float s_mid[16];
-    __shared__ Bucket s_bkt[64];
+    __shared__ uint32_t s_bkt[64];
     __shared__ double s_sum[kTileBlocks];
     const int tid = threadIdx.x;
     pdl_launch_dependents();  // the mean kernel may take an SM as soon as one frees; it waits for this grid
@@ -89,13 +90,14 @@ __global__ void __launch_bounds__(256, 3) k_nf4_encode(const float* __restrict__
         const int idx = tid - 64;
         const int bi = idx < 32 ? idx : (idx == 32 ? 31 : 0);  // 32: rounding above +1; 63: below -1
         const float lo = -1.0f + 0.0625f * static_cast<float>(bi), hi = lo + 0.0625f;
-        Bucket e{__int_as_float(0x7f800000), 0u};
+        float thr = 2.0f;
+        uint32_t base = 0;
         for (int j = 0; j < 15; ++j) {
             const float m = __fmul_rn(__fadd_rn(nf4_level(j), nf4_level(j + 1)), 0.5f);
-            if (m < lo) ++e.base;
-            else if (m < hi) e.thr = m;
+            if (m < lo) ++base;
+            else if (m < hi) thr = m;
         }
-        s_bkt[idx] = e;
+        s_bkt[idx] = (__float_as_uint(thr) & ~15u) | base;
     }
     __syncthreads();
     const int lane = tid & 31, warp = tid >> 5;
