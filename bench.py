@@ -44,6 +44,7 @@ import time
 
 import numpy as np
 import torch
+import torch.distributed as dist
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
@@ -387,7 +388,6 @@ def time_quantize(nf, gw, args, stream, device, world, hbm_peak, peak_src):
     """Encoding of every module's fp32 weight through nf4_quantize, timed on
     its own: K passes over all modules after W warm-up passes (the fp32
     weights total more than 4x L2, so every pass reads them from HBM)."""
-    import torch.distributed as dist
     wl = gw.wl
     outs = [nf.NF4Tensor(m.d_out, m.d_in, device) for m in wl.modules]
     ws = torch.empty(max(nf.nf4_quantize_workspace_bytes(m.d_out, m.d_in) for m in wl.modules),
@@ -450,7 +450,6 @@ def time_adamw(nf, gw, args, stream, device, world, hbm_peak, peak_src, l2):
     and B (fp32 master, bf16 copy, bf16 gradient from the backward, fp32
     moments), timed on its own.  The optimizer state rotates over enough
     copies to exceed 4x L2, as it would be cold after the layer's GEMMs."""
-    import torch.distributed as dist  # noqa: F401
     grads = [t for d in gw.mods for t in (d["dA"], d["dB"])]
     n_total = sum(g.numel() for g in grads)
     per_copy = 26 * n_total  # fp32 master, m, v + bf16 copy and gradient
@@ -472,6 +471,8 @@ def time_adamw(nf, gw, args, stream, device, world, hbm_peak, peak_src, l2):
     for k in range(max(args.warmup, copies)):
         one_pass(k, k + 1)
     torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
     passes = max(3, min(args.steps, 50))
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
@@ -524,6 +525,8 @@ def time_merge(nf, gw, args, stream, device, world, clocks_mhz=1965.0):
     for _ in range(args.warmup):
         one_pass()
     torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
     passes = max(3, min(args.steps, 20))
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
@@ -562,7 +565,6 @@ def time_merge(nf, gw, args, stream, device, world, clocks_mhz=1965.0):
 
 
 def run_ours(args, wl):
-    import torch.distributed as dist
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))

@@ -118,6 +118,25 @@ def test_host_validation_without_device(nf):
     assert L.nf4_dequantize(None, Y, None) == -1
 
 
+def test_merge_host_validation_without_device(nf):
+    L = nf.lib
+    s = fake_tensor(nf)
+    A = P(1 << 24); B = P(1 << 25); out = P(1 << 26); ws = P(1 << 28)
+    f = ctypes.c_float(0.5)
+    assert nf.nf4_merge_workspace_bytes(128, 256) >= 128 * 256 * 4
+    assert nf.nf4_merge_workspace_bytes(128, 100) == 0                       # d_in % 64 != 0
+    assert L.nf4_merge_lora(ctypes.byref(s), A, B, 8, f, None, None) == -1    # no output
+    assert L.nf4_merge_lora(ctypes.byref(s), A, B, 8, f, P((1 << 26) + 4), None) == -3
+    assert L.nf4_merge_lora(ctypes.byref(s), A, B, 0, f, out, None) == -1     # r out of range
+    assert L.nf4_merge_lora(ctypes.byref(s), A, B, 257, f, out, None) == -1
+    assert L.nf4_merge_lora(ctypes.byref(s), None, B, 8, f, out, None) == -1
+    assert L.nf4_merge_lora(ctypes.byref(s), A, B, 8, ctypes.c_float(float("nan")), out, None) == -1
+    other = fake_tensor(nf, 64, 256)
+    assert L.nf4_merge_requantize(ctypes.byref(s), A, B, 8, f, ctypes.byref(other), ws, 1 << 30, None) == -1
+    assert L.nf4_merge_requantize(ctypes.byref(s), A, B, 8, f, ctypes.byref(s), ws, 1024, None) == -4
+    assert L.nf4_merge_requantize(ctypes.byref(s), A, B, 8, f, ctypes.byref(s), None, 0, None) == -4
+
+
 def test_adamw_host_validation_without_device(nf):
     L = nf.lib
     T = nf.AdamwTensorStruct
