@@ -10,11 +10,12 @@
 //
 // Both are themselves programmatic dependents of the kernel before them (the
 // previous fused GEMM releases its dependents when it starts): their CTAs
-// start early, stage the rows of the LoRA factor (a parameter, never written
-// by the preceding kernel), then wait for that kernel to finish before they
-// read the activations or gradients, which it may have produced.  They release
-// their own dependent only after that wait, so the fused GEMM that follows may
-// read the same activations before its own wait.
+// start early and ask L2 for their rows of the LoRA factor (a prefetch only:
+// the factor may have been written by that very kernel, an optimizer step for
+// instance), then wait for the preceding kernel to finish before they read
+// anything.  They release their own dependent right after that wait, so the
+// fused GEMM that follows may read the activations and the encoded weight
+// before its own wait.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -31,6 +32,13 @@ namespace {
 
 constexpr int kMaxFewTokens = 16;
 
+// Asks L2 for `bytes` (a multiple of 16) from a 16-byte aligned address, in
+// pieces of at most 32 KB.
+__device__ __forceinline__ void prefetch_l2_pieces(const void* src, uint32_t bytes) {
+    const uint8_t* p = static_cast<const uint8_t*>(src);
+    for (uint32_t off = 0; off < bytes; off += 32768u) prefetch_l2_bulk(p + off, min(32768u, bytes - off));
+}
+
 __device__ __forceinline__ void store_split(uint16_t* dst_hi, uint16_t* dst_lo, float v) {
     const __nv_bfloat16 hi = __float2bfloat16_rn(v);
     const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
@@ -43,10 +51,9 @@ __device__ __forceinline__ void store_split(uint16_t* dst_hi, uint16_t* dst_lo, 
 // CTA (x, z) computes columns 16x .. 16x + 15 of T over the z-th of up to 8
 // slices of K; the slices of one column group form a cluster.  A CTA copies
 // its 16 rows of A and its part of X (up to 512 k at a time) into shared
-// memory with asynchronous copies issued all at once (A before the wait for
-// the preceding kernel, X after it), and releases the dependent launch as
-// soon as they are requested, so that these loads queue ahead of the
-// dependent kernel's.  The CTAs are small (four warps, 37 KB of
+// memory with asynchronous copies issued all at once, after the wait for the
+// preceding kernel (the rows of A were asked into L2 before it), and the
+// dependent launch is released right after that wait.  The CTAs are small (four warps, 37 KB of
 // shared memory) and many (one per SM for r = 64), so that the loads are
 // spread over SMs and the CTAs share SMs with the dependent kernel's.  Warp w
 // takes every fourth 16-wide chunk; partials are added in a fixed order: the
@@ -92,7 +99,12 @@ __global__ void __launch_bounds__(kDownThreads) k_few_down(const uint16_t* __res
     const int k_end = k_begin + 64 * (per + (rank < extra ? 1 : 0));
     float acc[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
 
-    bool first = true;
+    // this CTA's rows of A over its K slice, into L2 while the preceding kernel runs
+    if (tid < 16 && j0 + tid < r && k_begin < k_end)
+        prefetch_l2_pieces(A + static_cast<int64_t>(j0 + tid) * K + k_begin,
+                           static_cast<uint32_t>(2 * (k_end - k_begin)));
+    pdl_wait();                // the preceding kernel's writes (X, or A itself) are complete and visible
+    pdl_launch_dependents();   // the fused GEMM may start: everything before it is complete
     for (int k0 = k_begin; k0 < k_end; k0 += kDownBatch) {
         const int kn = min(kDownBatch, k_end - k0);  // a multiple of 64
         const int pieces = kn / 8;                   // 16-byte pieces per row
@@ -103,16 +115,11 @@ __global__ void __launch_bounds__(kDownThreads) k_few_down(const uint16_t* __res
             if (j < r) cp_async16(dst, A + static_cast<int64_t>(j) * K + k0 + pc * 8);
             else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
         }
-        if (first) pdl_wait();  // X may be the preceding kernel's output
         for (int i = tid; i < kMaxFewTokens * pieces; i += kDownThreads) {
             const int row = i / pieces, pc = i - row * pieces;
             uint16_t* dst = sX + row * kDownStride + pc * 8;
             if (row < M) cp_async16(dst, X + static_cast<int64_t>(row) * K + k0 + pc * 8);
             else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
-        }
-        if (first) {
-            pdl_launch_dependents();
-            first = false;
         }
         cp_async_wait_all();
         __syncthreads();
@@ -130,10 +137,6 @@ __global__ void __launch_bounds__(kDownThreads) k_few_down(const uint16_t* __res
             mma_m16n8k16(acc[1], a0, a1, a2, a3, *reinterpret_cast<const uint32_t*>(ar1 + k),
                          *reinterpret_cast<const uint32_t*>(ar1 + k + 8));
         }
-    }
-    if (first) {  // empty slice (not produced by the launcher): keep the ordering guarantees
-        pdl_wait();
-        pdl_launch_dependents();
     }
 
     // acc[u]: tokens g (0, 1) and g + 8 (2, 3) at columns 8u + 2q + {0, 1}; the
@@ -179,8 +182,9 @@ __global__ void __launch_bounds__(kDownThreads) k_few_down(const uint16_t* __res
 // T kernel: CTA (x, z) computes columns 16x .. 16x + 15 of V over the z-th of
 // up to 8 slices of d_out, the slices of one column group form a cluster, the
 // slice of B and of dY (up to 256 rows at a time) comes in by asynchronous
-// copies issued at once (B before the wait for the preceding kernel, dY after
-// it), and the dependent launch is released right after.
+// copies issued at once after the wait for the preceding kernel (the rows of B
+// were asked into L2 before it), and the dependent launch is released right
+// after that wait.
 constexpr int kVBatch = 256;                    // rows of B per staged slice (small enough to share an SM with the dX kernel)
 constexpr int kVYStride = kVBatch + 8;          // dY staging row stride (elements)
 constexpr int kVBStride = 24;                   // B staging row stride (elements): 48 bytes, conflict-free ldmatrix
@@ -207,7 +211,14 @@ __global__ void __launch_bounds__(kDownThreads) k_few_v(const uint16_t* __restri
     const int n_end = n_begin + 16 * (per + (rank < extra ? 1 : 0));
     float acc[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
 
-    bool first = true;
+    // this CTA's rows of B (all r columns of each, contiguous), into L2 while the preceding kernel runs
+    if (tid == 0 && n_begin < n_end && j0 < r) {
+        const int rows = min(n_end, N) - n_begin;
+        if (rows > 0)
+            prefetch_l2_pieces(B + static_cast<int64_t>(n_begin) * r, static_cast<uint32_t>(2 * rows * r));
+    }
+    pdl_wait();                // the preceding kernel's writes (dY, or B itself) are complete and visible
+    pdl_launch_dependents();   // the fused GEMM may start: everything before it is complete
     for (int n0 = n_begin; n0 < n_end; n0 += kVBatch) {
         const int nn = min(kVBatch, n_end - n0);  // a multiple of 16
         __syncthreads();                          // the previous slice is no longer read
@@ -218,17 +229,12 @@ __global__ void __launch_bounds__(kDownThreads) k_few_v(const uint16_t* __restri
             if (n < N && j < r) cp_async16(dst, B + static_cast<int64_t>(n) * r + j);
             else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
         }
-        if (first) pdl_wait();  // dY may be the preceding kernel's output
         // dY[:, n0 : n0 + nn] in 16-byte pieces (N is a multiple of 8)
         for (int i = tid; i < kMaxFewTokens * (nn / 8); i += kDownThreads) {
             const int t = i / (nn / 8), pc = i - t * (nn / 8), n = n0 + 8 * pc;
             uint16_t* dst = sY + t * kVYStride + 8 * pc;
             if (t < M && n < N) cp_async16(dst, dY + static_cast<int64_t>(t) * N + n);
             else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
-        }
-        if (first) {
-            pdl_launch_dependents();
-            first = false;
         }
         cp_async_wait_all();
         __syncthreads();
@@ -247,10 +253,6 @@ __global__ void __launch_bounds__(kDownThreads) k_few_v(const uint16_t* __restri
             mma_m16n8k16(acc[0], a0, a1, a2, a3, b0, b1);
             mma_m16n8k16(acc[1], a0, a1, a2, a3, c0, c1);
         }
-    }
-    if (first) {  // empty slice (not produced by the launcher): keep the ordering guarantees
-        pdl_wait();
-        pdl_launch_dependents();
     }
 
 #pragma unroll

@@ -99,3 +99,40 @@ def test_adamw_steps_track_the_oracle(nf):
     for got, ref, tol in ((d[0], rp, 1e-6), (d[1], rm, 1e-5), (d[2], rv, 1e-5)):
         got = got.cpu().double().numpy()
         assert np.max(np.abs(got - ref)) <= tol * np.max(np.abs(ref))
+
+
+@pytest.mark.parametrize("m", [4, 16, 64])
+def test_layer_right_after_the_step_sees_the_new_adapter(nf, m):
+    """The optimizer step rewrites the bf16 A and B the layer reads; the
+    forward and backward enqueued right after it on the same stream (no
+    synchronisation in between) must use the new values."""
+    import workloads
+    from parity import assert_close
+    d_out, d_in, r, s = 512, 512, 16, 0.5
+    W = workloads.weight(d_out, d_in, index=3)
+    qt = oracle.quantize(W)
+    enc = nf.nf4_quantize(torch.from_numpy(W).cuda())
+    A0, B0 = workloads.lora_a(r, d_in, 3), workloads.lora_b(d_out, r, 3, std=0.05)
+    X, dY = workloads.activations(m, d_in), workloads.grad_output(m, d_out, 3)
+    params = []
+    for p0 in (A0, B0):
+        master = p0.float().reshape(-1).cuda()
+        param = p0.clone().cuda()
+        grad = (torch.randn(p0.numel(), generator=torch.Generator().manual_seed(p0.numel())) * 0.1).bfloat16().cuda()
+        params.append((master, param.reshape(-1), grad, torch.zeros_like(master), torch.zeros_like(master), param))
+    torch.cuda.synchronize()
+    nf.lora_adamw_step([t[:5] for t in params], lr=0.05, step=1)  # moves every entry by about 0.05
+    A, B = params[0][5], params[1][5]
+    Y, T = nf.qlora_linear_fwd(enc, A, B, s, X.cuda())
+    dX, dA, dB = nf.qlora_linear_bwd(enc, A, B, s, X.cuda(), T, dY.cuda())
+    torch.cuda.synchronize()
+    nf.device_status()
+    A1, B1 = A.cpu(), B.cpu()
+    assert not torch.equal(A1, A0)
+    W_hat = oracle.dequantize(qt, (d_out, d_in))
+    Y_ref, _ = oracle.forward(W_hat, A1, B1, X, s)
+    assert_close(Y.cpu(), Y_ref, "Y after the step")
+    dX_ref, dA_ref, dB_ref = oracle.backward(W_hat, A1, B1, X, dY, s)
+    assert_close(dX.cpu(), dX_ref, "dX after the step")
+    assert_close(dA.cpu(), dA_ref, "dA after the step")
+    assert_close(dB.cpu(), dB_ref, "dB after the step")
