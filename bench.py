@@ -2,32 +2,40 @@
 """Throughput of the NF4-LoRA linear layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME] [--no-graph]
+                    [--workload NAME] [--no-graph] [--no-few]
 
-One step is one pass of the layer over one batch of the workload (default:
-the LLaMA-7B q_proj 4096 x 4096, LoRA r = 64, tokens M in {1, 4, 16}, forward
-plus input gradient, i.e. 6 passes over the NF4 weight).  Inputs are seeded
-and synthetic (``workloads.py``).  Between timed steps the weights rotate over
-enough encoded copies to exceed 4x the L2 cache, so every pass streams its
-weight from HBM.  Steps are replayed from CUDA graphs; the library's own
-launch tracing times the dominant kernel on the stream it runs on.
+One step is one pass of the layer over one batch of the workload.  The
+default workload is the LLaMA-65B layer's seven linears (q/k/v/o 8192 x 8192,
+gate/up 8192 -> 22016, down 22016 -> 8192), NF4 + double quantisation, LoRA
+r = 64, 2048 tokens: forward then backward (dX, dA, dB) of every module in
+layer order.  That step is dense-bf16 tensor bound, so the headline `value`
+is its algorithmic TFLOP/s.  The same line carries, as sub-objects:
 
-Besides the step, the line carries the phases around it where the workload
-has them, each timed on its own with CUDA events: ``quantize`` (encoding of
-the fp32 weights, the LLaMA-65B workload), ``optimizer`` (the AdamW step of
-A and B after a full backward) and ``merge`` (the adapter folded into the
-base and re-encoded, the LLaMA-65B workload), each with its roofline.
-``--only quantize|merge|optimizer`` times one phase alone (a short command to
-profile).
+* ``quantize`` -- the encoding of the seven fp32 weights (nf4_quantize),
+  HBM bound, in GB/s;
+* ``few_token`` -- the LLaMA-7B q_proj 4096 x 4096 at M in {1, 4, 16},
+  forward plus input gradient (the decode-like, HBM-bound path), in GB/s
+  of the weight stream;
+* ``optimizer`` (the AdamW step of A and B) and ``merge`` (the adapter folded
+  into the base and encoded again), each with its roofline.
+
+Inputs are seeded and synthetic (``workloads.py``).  Between timed steps the
+encoded weights rotate over enough copies to exceed 4x the L2 cache, so every
+pass streams its weight from HBM.  The timed steps are replayed from CUDA
+graphs captured without the library's launch tracing; the per-kernel device
+times behind each roofline come from a separate traced pass of the same steps
+right after the timed region.  ``--only quantize|merge|optimizer`` times one
+phase alone (a short command to profile).
 
 Rank 0 prints ONE JSON line.  With N > 1 (torchrun, one process per GPU)
 every rank runs the same per-GPU workload on its own data (weak scaling) and
 the time is the max over ranks.  A forward + input-gradient workload has no
 exchange step (independent replicas); a full-backward workload is a
-data-parallel training step, so after each step the ranks sum their adapter
-gradients dA, dB with one all-reduce (``nf4_base_lora_b200.dp``), inside the
-timed region.  ``--impl reference`` times the CPU oracle (the plain fp64 statement
-of the method) on the host on a bounded sample of the same workload.
+data-parallel training step, so the ranks sum their adapter gradients dA, dB
+with one all-reduce per module (``nf4_base_lora_b200.dp``) inside the timed
+region.  ``--impl reference`` times the CPU oracle (the plain fp64 statement
+of the method) on the host on the same bounded sample of the workload that the
+``cpu_baseline`` key reports.
 """
 from __future__ import annotations
 
@@ -98,13 +106,32 @@ def step_totals(wl):
 
 
 def load_peaks():
+    """Roofline denominators: the measured copy bandwidth and bf16 GEMM
+    rates of this machine's B200s (burst: a kernel timed alone; sustained: a
+    seconds-long loop under the power cap), else the recorded fallback."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
             p = json.load(f)
-        return float(p["hbm_gbs"]), float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), "measured"
+        burst = float(p["bf16_tflops"])
+        return {"hbm": float(p["hbm_gbs"]), "bf16": burst,
+                "bf16_sustained": float(p.get("bf16_tflops_sustained", burst)), "source": "measured"}
     except Exception:
-        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+        return {"hbm": FALLBACK_HBM_GBS, "bf16": FALLBACK_BF16_TFLOPS, "bf16_sustained": 1400.0,
+                "source": "fallback"}
+
+
+def kernel_flops(d_out, d_in, m, r, kernel):
+    """Algorithmic flops of one launch of a fused dequant-GEMM: the base
+    product plus the rank-r term it accumulates (the LoRA-up T B^T for the
+    forward, V A for the input gradient)."""
+    if kernel.startswith("nf4_gemm_fwd"):
+        return 2 * m * d_in * d_out + 2 * m * r * d_out
+    return 2 * m * d_in * d_out + 2 * m * r * d_in
+
+
+def tensor_bound(wl):
+    return max(wl.tokens) > 16
 
 
 def kernel_source_hash(files=None):
@@ -207,22 +234,34 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- oracle arm
+# The CPU oracle is timed on one fixed, bounded sample of the workload: the
+# first ORACLE_ROWS weight rows (a whole number of 256-block groups) of the
+# first module, i.e. that slice's share of every pass of the step.  The
+# cpu_baseline key and the --impl reference arm time the same sample, in the
+# headline's unit.
+ORACLE_ROWS = 256
+
+
+def oracle_rows(mod):
+    unit = max(4, (256 * 64) // mod.d_in)   # rows of one 256-block group
+    return max(unit, ORACLE_ROWS // unit * unit)
+
+
 def oracle_sample_step(oracle, qt, mod, wl, host, rows):
-    """The oracle on a slice of `rows` weight rows (aligned to 256 blocks) of
-    one module: its share of every pass of the step.  Returns algorithmic bytes."""
-    d_in, d_out = mod.d_in, mod.d_out
-    n0 = 0
+    """The oracle on `rows` weight rows of one module: its share of every
+    pass of the step.  Returns (algorithmic bytes, flops) of that share."""
+    d_in = mod.d_in
     n = rows * d_in
-    packed = qt["packed"][n0 * d_in // 2:(n0 + rows) * d_in // 2]
-    q = qt["q"][n0 * d_in // 64:(n0 + rows) * d_in // 64]
-    a2 = qt["a2"][(n0 * d_in // 64) // 256:]
+    packed = qt["packed"][:n // 2]
+    q = qt["q"][:n // 64]
+    a2 = qt["a2"]
     bits = oracle.dequantize_bits(packed, q, a2, float(qt["mu"]), n)
     W_hat = oracle.bf16_bits_to_f32(bits).reshape(rows, d_in)
-    A, B = host["A"], host["B"][n0:n0 + rows]
-    nbytes = 0.0
+    A, B = host["A"], host["B"][:rows]
+    nbytes = nflops = 0.0
     for m in wl.tokens:
         X = host["X"][:m]
-        dY = host["dY"][:m, n0:n0 + rows]
+        dY = host["dY"][:m, :rows]
         oracle.forward(W_hat, A, B, X, wl.scaling)
         if wl.backward == "dx":
             oracle.input_grad_rows(W_hat, A, B, dY, wl.scaling)
@@ -232,7 +271,8 @@ def oracle_sample_step(oracle, qt, mod, wl, host, rows):
             kinds = ("fwd", "full")
         for kind in kinds:
             nbytes += pass_bytes(rows, d_in, m, wl.r, kind)
-    return nbytes
+            nflops += pass_flops(rows, d_in, m, wl.r, kind)
+    return nbytes, nflops
 
 
 def oracle_setup(wl):
@@ -246,66 +286,94 @@ def oracle_setup(wl):
     return oracle, qt, mod, host
 
 
+def oracle_unit(wl):
+    return "TFLOP/s" if tensor_bound(wl) else "GB/s"
+
+
+def oracle_value(wl, nbytes, nflops, seconds):
+    return nflops / seconds / 1e12 if tensor_bound(wl) else nbytes / seconds / 1e9
+
+
+def oracle_sample_text(wl, mod, rows):
+    return "%d of %d weight rows of %s (its share of every pass of the step: %s at M = %s)" % (
+        rows, mod.d_out, mod.name, "fwd + dX" if wl.backward == "dx" else "fwd + dX + dA + dB",
+        "/".join(str(m) for m in wl.tokens))
+
+
+def host_cores():
+    return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+
+
 def time_oracle(wl, budget_s, min_steps=1):
     """Time oracle sample steps for about budget_s seconds of host work."""
     oracle, qt, mod, host = oracle_setup(wl)
-    rows_unit = max(4, (256 * 64) // mod.d_in)   # smallest slice aligned to a 256-block group
-    rows = rows_unit * 16
+    rows = oracle_rows(mod)
     t0 = time.perf_counter()
     oracle_sample_step(oracle, qt, mod, wl, host, rows)
     one = time.perf_counter() - t0
     steps = max(min_steps, int(budget_s / max(one, 1e-3)))
     t0 = time.perf_counter()
-    total = 0.0
+    nb = nf = 0.0
     for _ in range(steps):
-        total += oracle_sample_step(oracle, qt, mod, wl, host, rows)
+        b, f = oracle_sample_step(oracle, qt, mod, wl, host, rows)
+        nb += b
+        nf += f
     dt = time.perf_counter() - t0
-    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
-    return {"value": total / dt / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
-            "sample": "%d of %d weight rows of %s, all passes of the step, %d steps in %.1f s"
-                      % (rows, mod.d_out, mod.name, steps, dt),
-            "seconds": dt, "steps": steps, "step_s": dt / steps}
+    return {"value": oracle_value(wl, nb, nf, dt), "unit": oracle_unit(wl), "cores": host_cores(),
+            "kind": "oracle", "sample": oracle_sample_text(wl, mod, rows) + ", %d steps in %.1f s" % (steps, dt),
+            "seconds": dt, "steps": steps}
 
 
 def run_reference(args, wl):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    n_steps = args.steps + args.warmup
-    per_step_budget = max(0.01, 90.0 / max(1, n_steps))
     oracle, qt, mod, host = oracle_setup(wl)
-    rows_unit = max(4, (256 * 64) // mod.d_in)
-    t0 = time.perf_counter()
-    oracle_sample_step(oracle, qt, mod, wl, host, rows_unit)
-    unit_s = time.perf_counter() - t0
-    rows = rows_unit * max(1, int(per_step_budget / max(unit_s, 1e-4)))
-    rows = min(rows, mod.d_out - mod.d_out % rows_unit)
+    rows = oracle_rows(mod)
     for _ in range(args.warmup):
         oracle_sample_step(oracle, qt, mod, wl, host, rows)
     t0 = time.perf_counter()
-    total = 0.0
+    nb = nf = 0.0
     for _ in range(args.steps):
-        total += oracle_sample_step(oracle, qt, mod, wl, host, rows)
+        b, f = oracle_sample_step(oracle, qt, mod, wl, host, rows)
+        nb += b
+        nf += f
     dt = time.perf_counter() - t0
-    value = total / dt / 1e9
-    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
-    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+    value = oracle_value(wl, nb, nf, dt)
+    unit = oracle_unit(wl)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": workload_config(wl),
-            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
-                             "sample": "%d of %d weight rows of %s per step, all passes" % (rows, mod.d_out, mod.name)},
-            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "data": DATA, "config": workload_config(wl, args.gpus),
+            "cpu_baseline": {"value": value, "unit": unit, "cores": host_cores(), "kind": "oracle",
+                             "sample": oracle_sample_text(wl, mod, rows) + " per step"},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
 # ---------------------------------------------------------------- GPU arm
-def workload_config(wl):
+DATA = ("synthetic: seeded N(0, sigma) fp32 weights (0.1% x10 outliers where the workload has them), "
+        "N(0, 1) bf16 activations and output gradients, random-init bf16 adapters")
+
+
+def parallelism(wl, gpus):
+    if gpus <= 1:
+        return "dp1"
+    if wl.backward == "dx":
+        return "dp%d (independent replicas: no exchange step)" % gpus
+    return "dp%d (token shards; all-reduce of dA, dB per module)" % gpus
+
+
+def workload_config(wl, gpus=1):
+    """The workload as both arms report it (identical keys and values)."""
     return {"workload": wl.name,
             "modules": [[m.name, m.d_out, m.d_in] for m in wl.modules],
             "tokens": list(wl.tokens), "r": wl.r, "alpha": wl.alpha,
             "passes": "fwd+dX" if wl.backward == "dx" else "fwd+bwd(dX,dA,dB)",
-            "weights": "NF4 blocksize 64 + double-quantised scales (8-bit, blocks of 256)"}
+            "weights": "NF4 blocksize 64 + double-quantised scales (8-bit, blocks of 256)",
+            "l2_flush": "encoded weights rotate over copies totalling at least 4x L2, so every pass reads "
+                        "its weight from HBM",
+            "parallelism": parallelism(wl, gpus)}
 
 
 class GpuWorkload:
@@ -384,7 +452,7 @@ def quantize_bytes(d_out, d_in):
     return 4 * n + n // 2 + nb + 4 * ((nb + 255) // 256) + 4
 
 
-def time_quantize(nf, gw, args, stream, device, world, hbm_peak, peak_src):
+def time_quantize(nf, gw, args, stream, device, world, peaks):
     """Encoding of every module's fp32 weight through nf4_quantize, timed on
     its own: K passes over all modules after W warm-up passes (the fp32
     weights total more than 4x L2, so every pass reads them from HBM)."""
@@ -432,20 +500,20 @@ def time_quantize(nf, gw, args, stream, device, world, hbm_peak, peak_src):
     out = {"ms_per_pass": ms, "passes": passes, "value": value, "unit": "GB/s",
            "weights_per_pass": weights, "bytes_per_pass": per_pass,
            "algorithmic": "per module 4n + n/2 + n/64 + 4*ceil(n/16384) + 4 bytes (n weights)",
-           "frac": value / world / hbm_peak,
+           "frac": value / world / peaks["hbm"],
            "kernels": {k: {"launches": len(v), "avg_us": sum(v) / len(v) * 1e3} for k, v in sorted(per_kernel.items())}}
     if enc_ms > 0:
         achieved = enc_bytes / (enc_ms * 1e-3) / 1e9
         bpw = load_traffic_per_weight("nf4_encode")
-        out["roofline"] = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                           "frac": achieved / hbm_peak, "kernel": "nf4_encode",
+        out["roofline"] = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
+                           "frac": achieved / peaks["hbm"], "kernel": "nf4_encode",
                            "traffic": None if bpw is None else bpw * weights / len(wl.modules),
                            "algorithmic": "4n read + n/2 written per launch (fp32 weight in, packed codes out)",
-                           "peak_source": peak_src + " (hbm_gbs)"}
+                           "peak_source": peaks["source"] + " (hbm_gbs)"}
     return out
 
 
-def time_adamw(nf, gw, args, stream, device, world, hbm_peak, peak_src, l2):
+def time_adamw(nf, gw, args, stream, device, world, peaks, l2):
     """The step after the backward: one lora_adamw_step over every module's A
     and B (fp32 master, bf16 copy, bf16 gradient from the backward, fp32
     moments), timed on its own.  The optimizer state rotates over enough
@@ -494,11 +562,11 @@ def time_adamw(nf, gw, args, stream, device, world, hbm_peak, peak_src, l2):
     step_bytes = 28 * n_total
     value = world * step_bytes / (ms * 1e-3) / 1e9
     out = {"ms_per_pass": ms, "passes": passes, "params": n_total, "bytes_per_pass": step_bytes,
-           "value": value, "unit": "GB/s", "frac": value / world / hbm_peak,
+           "value": value, "unit": "GB/s", "frac": value / world / peaks["hbm"],
            "algorithmic": "28 bytes per parameter: fp32 master, m, v read and written, bf16 gradient read, "
                           "bf16 copy written",
            "l2_flush": "rotating %d optimizer-state copies (%.0f MB)" % (copies, copies * per_copy / 1e6),
-           "peak_source": peak_src + " (hbm_gbs)"}
+           "peak_source": peaks["source"] + " (hbm_gbs)"}
     if k_ms:
         out["kernels"] = {"lora_adamw": {"launches": len(k_ms), "avg_us": sum(k_ms) / len(k_ms) * 1e3}}
     return out
@@ -564,39 +632,10 @@ def time_merge(nf, gw, args, stream, device, world, clocks_mhz=1965.0):
     return out
 
 
-def run_ours(args, wl):
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    device = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
-
-    import nf4_base_lora_b200 as nf
-    hbm_peak, tc_peak, peak_src = load_peaks()
-    l2 = torch.cuda.get_device_properties(device).L2_cache_size
-    if args.only:
-        # one phase of the workload on its own (a short command to profile):
-        # the encoding, the merge + re-encoding or the optimizer step
-        gw = GpuWorkload(nf, wl, device, 1, keep_fp32=args.only == "quantize")
-        stream = torch.cuda.Stream(device)
-        if args.only == "quantize":
-            obj = time_quantize(nf, gw, args, stream, device, world, hbm_peak, peak_src)
-        elif args.only == "merge":
-            obj = time_merge(nf, gw, args, stream, device, world)
-        else:
-            with torch.cuda.stream(stream):
-                gw.step(0)  # the backward fills dA, dB
-            obj = time_adamw(nf, gw, args, stream, device, world, hbm_peak, peak_src, l2)
-        if world > 1:
-            dist.barrier()
-            dist.destroy_process_group()
-        if rank == 0:
-            print(json.dumps({"metric": METRIC, "phase": args.only, "n_gpus": world,
-                              "config": workload_config(wl), args.only: obj}), flush=True)
-        return
+def time_workload(nf, wl, args, stream, device, world, peaks, l2, with_e2e):
+    """Time K steps of one workload (replayed from CUDA graphs captured
+    without tracing), then one traced pass of the same steps for the
+    per-kernel device times.  Returns the numbers and the GpuWorkload."""
     plan = step_plan(wl)
     wbytes = sum(weight_bytes(mod.d_out, mod.d_in) for mod in wl.modules)
     # enough encoded copies that consecutive passes of one module never share L2
@@ -608,52 +647,42 @@ def run_ours(args, wl):
     cycle = max(1, copies // len(plan)) if copies > 1 else 1
     step_bytes, step_flops = step_totals(wl)
 
-    stream = torch.cuda.Stream(device)
-    graphs = []
-    nf.trace_start(len(plan) * cycle * 16 + 64)
-    with torch.cuda.stream(stream):
-        gw.step(0)                                   # eager warm-up (JIT-free, sets attributes)
-        torch.cuda.synchronize()
-    launches_per_step = None
-    if not args.no_graph:
-        nf.trace_start(len(plan) * cycle * 16 + 64)
-        for g in range(cycle):
-            graph = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(graph, stream=stream):
-                gw.step(g * len(plan))
-            graphs.append(graph)
-        launches_per_step = nf.trace_count() / cycle
-        nf.trace_stop()
-
     # data-parallel exchange of the adapter gradients (full backward, N > 1)
     exchange = None
     if world > 1 and wl.backward != "dx":
         from nf4_base_lora_b200 import dp
         exchange = dp.LoraGradExchange([t for d in gw.mods for t in (d["dA"], d["dB"])])
 
+    def enqueue(s_index, **kw):
+        gw.step((s_index % cycle) * len(plan), **kw)
+        if exchange is not None:
+            exchange()
+
+    # eager warm-up step, traced only to count the library's launches per step
+    nf.trace_start(len(plan) * 16 + 64)
+    with torch.cuda.stream(stream):
+        gw.step(0)
+    torch.cuda.synchronize()
+    launches_per_step = nf.trace_count()
+    nf.trace_stop()
+
+    graphs = []
+    if not args.no_graph:
+        for g in range(cycle):
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=stream):
+                gw.step(g * len(plan))
+            graphs.append(graph)
+
     def run_steps(k, base):
         with torch.cuda.stream(stream):
-            for s in range(k):
+            for i in range(k):
                 if graphs:
-                    graphs[(base + s) % cycle].replay()
+                    graphs[(base + i) % cycle].replay()
+                    if exchange is not None:
+                        exchange()
                 else:
-                    gw.step(((base + s) % cycle) * len(plan))
-                if exchange is not None:
-                    exchange()
-
-    def run_steps_eager(k, base):
-        with torch.cuda.stream(stream):
-            for s in range(k):
-                gw.step(((base + s) % cycle) * len(plan))
-                if exchange is not None:
-                    exchange()
-
-    if not graphs:
-        nf.trace_start(len(plan) * 16 + 64)
-        run_steps(1, 0)
-        torch.cuda.synchronize()
-        launches_per_step = nf.trace_count()
-        nf.trace_stop()
+                    enqueue(base + i)
 
     run_steps(args.warmup, 0)
     torch.cuda.synchronize()
@@ -679,58 +708,73 @@ def run_ours(args, wl):
         from nf4_base_lora_b200 import dp
         ms = dp.max_over_ranks(ms, device)
     ms_per_step = ms / args.steps
-    value = world * step_bytes / (ms_per_step * 1e-3) / 1e9
+    gbps = world * step_bytes / (ms_per_step * 1e-3) / 1e9
     tflops = world * step_flops / (ms_per_step * 1e-3) / 1e12
 
-    # dominant kernel: device time per launch from the library's tracing.  The
-    # records captured in the graphs hold the last replay of each graph, i.e.
-    # the final cycle of the timed region.
-    records = nf.trace_records() if graphs else []
-    timing_source = "events captured in the step graphs, last replay of each (final cycle of the timed region)"
-    if len(records) < int(launches_per_step or 1) * cycle:
-        # graph-recorded events could not be read back: time the same steps
-        # eagerly with the library's tracing on, right after the timed region
-        k_eager = max(cycle, min(args.steps, 50))
-        nf.trace_start(int(launches_per_step or 64) * k_eager + 64)
-        run_steps_eager(k_eager, args.warmup)
-        torch.cuda.synchronize()
-        records = nf.trace_records()
-        nf.trace_stop()
-        timing_source = "eager traced pass of %d steps after the timed region" % k_eager
-    small = max(wl.tokens) <= 16
-    names = ("nf4_gemm_fwd_few", "nf4_gemm_dx_few") if small else ("nf4_gemm_fwd", "nf4_gemm_dx")
+    # per-kernel device times: a separate pass of the same steps with the
+    # library's launch tracing on (event pairs around each launch, eager)
+    k_eager = max(cycle, min(args.steps, 50))
+    nf.trace_start(int(launches_per_step) * k_eager + 64)
+    with torch.cuda.stream(stream):
+        for i in range(k_eager):
+            enqueue(args.warmup + i)
+    torch.cuda.synchronize()
+    records = nf.trace_records()
+    nf.trace_stop()
+    timing_source = "traced eager pass of %d steps right after the timed region" % k_eager
+    hbm = not tensor_bound(wl)
+    names = ("nf4_gemm_fwd_few", "nf4_gemm_dx_few") if hbm else ("nf4_gemm_fwd", "nf4_gemm_dx")
     dom, kstats = dominant_kernel_stats(records, names)
     roofline = None
     if dom is not None:
         n_launch, tot_ms = kstats[dom]
         avg_ms = tot_ms / n_launch
-        mod = wl.modules[0]
-        if small:
-            per_launch = sum(weight_bytes(m.d_out, m.d_in) for m in wl.modules) / len(wl.modules)
+        # the algorithmic work of the dominant kernel's launches in one step
+        launches = [(mod, m) for _, mod, m, kind in plan
+                    if (kind == "fwd") == dom.startswith("nf4_gemm_fwd")]
+        if hbm:
+            per_launch = sum(weight_bytes(mod.d_out, mod.d_in) for mod, _ in launches) / len(launches)
             achieved = per_launch / (avg_ms * 1e-3) / 1e9
-            roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                        "frac": achieved / hbm_peak, "traffic": load_traffic(dom, wl.name),
+            roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
+                        "frac": achieved / peaks["hbm"], "traffic": load_traffic(dom, wl.name),
                         "kernel": dom, "launches_timed": n_launch, "avg_us": avg_ms * 1e3,
                         "timing": timing_source,
                         "algorithmic": "NF4 weight stream, K*N*(0.5 + 1/64 + 4/16384) bytes per launch",
-                        "peak_source": peak_src + " (hbm_gbs)"}
+                        "peak_source": peaks["source"] + " (hbm_gbs, copy bandwidth)"}
         else:
-            fl = [pass_flops(m.d_out, m.d_in, t, wl.r, "fwd") for m in wl.modules for t in wl.tokens]
-            per_launch = sum(fl) / len(fl)
+            per_launch = sum(kernel_flops(mod.d_out, mod.d_in, m, wl.r, dom) for mod, m in launches) / len(launches)
             achieved = per_launch / (avg_ms * 1e-3) / 1e12
-            roofline = {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s",
-                        "frac": achieved / tc_peak, "traffic": load_traffic(dom, wl.name),
+            roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16"], "unit": "TFLOP/s",
+                        "frac": achieved / peaks["bf16"], "traffic": load_traffic(dom, wl.name),
                         "kernel": dom, "launches_timed": n_launch, "avg_us": avg_ms * 1e3,
                         "timing": timing_source,
-                        "algorithmic": "2*M*K*N + 2*M*r*(K+N) flops per launch",
-                        "peak_source": peak_src + " (bf16_tflops_sustained)"}
+                        "algorithmic": ("2*M*K*N + 2*M*r*N flops per launch (base product + LoRA up)"
+                                        if dom == "nf4_gemm_fwd" else
+                                        "2*M*K*N + 2*M*r*K flops per launch (base product + V A)"),
+                        "peak_source": peaks["source"] + " (bf16_tflops, burst: a kernel timed alone)",
+                        "peak_sustained": peaks["bf16_sustained"],
+                        "frac_of_sustained": achieved / peaks["bf16_sustained"]}
     kernel_table = {k: {"launches": v[0], "avg_us": v[1] / v[0] * 1e3} for k, v in sorted(kstats.items())}
-    quantize = time_quantize(nf, gw, args, stream, device, world, hbm_peak, peak_src) if gw.fp32 else None
-    optimizer = (time_adamw(nf, gw, args, stream, device, world, hbm_peak, peak_src, l2)
-                 if wl.backward != "dx" else None)
-    merge = time_merge(nf, gw, args, stream, device, world) if wl.quantize_timed else None
+    out = {"value": tflops if not hbm else gbps, "unit": "TFLOP/s" if not hbm else "GB/s",
+           "ms_per_step": ms_per_step, "tflops": tflops, "gbps": gbps, "roofline": roofline, "kernels": kernel_table,
+           "launches_per_step": launches_per_step, "copies": copies, "graphs": bool(graphs), "clocks": clocks,
+           "exchange": exchange is not None, "config": workload_config(wl, world)}
+    # weight GB/s: each step passes over every module's encoded weight once per pass of the plan
+    out["weight_gbps"] = world * sum(weight_bytes(mod.d_out, mod.d_in) for _, mod, _, _ in plan) / (
+        ms_per_step * 1e-3) / 1e9
 
-    # end to end through the public API: pinned host inputs -> device -> layer -> host
+    if with_e2e:
+        out["e2e"] = time_e2e(gw, wl, args, stream, device, world, cycle, plan, exchange, step_bytes, step_flops)
+    for g in graphs:
+        del g
+    graphs.clear()
+    return out, gw
+
+
+def time_e2e(gw, wl, args, stream, device, world, cycle, plan, exchange, step_bytes, step_flops):
+    """The same step end to end through the public API: pinned host inputs
+    copied to the device, the layer calls, the outputs copied back, every
+    step inside the timed region."""
     e2e_steps = max(3, min(args.steps, 200))
     hostX = [torch.empty_like(d["X"], device="cpu").pin_memory() for d in gw.mods]
     hostdY = [torch.empty_like(d["dY"], device="cpu").pin_memory() for d in gw.mods]
@@ -775,7 +819,65 @@ def run_ours(args, wl):
     if world > 1:
         from nf4_base_lora_b200 import dp
         ems = dp.max_over_ranks(ems, device)
-    e2e_value = world * step_bytes / (ems / e2e_steps * 1e-3) / 1e9
+    sec = ems / e2e_steps * 1e-3
+    value = world * (step_flops / sec / 1e12 if tensor_bound(wl) else step_bytes / sec / 1e9)
+    return {"value": value, "unit": "TFLOP/s" if tensor_bound(wl) else "GB/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": e2e_steps, "ms_per_step": ems / e2e_steps}
+
+
+FEW_TOKEN_WORKLOAD = "q_proj4096_r64_m1-4-16"
+
+
+def run_ours(args, wl):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
+
+    import nf4_base_lora_b200 as nf
+    peaks = load_peaks()
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    stream = torch.cuda.Stream(device)
+    if args.only:
+        # one phase of the workload on its own (a short command to profile):
+        # the encoding, the merge + re-encoding or the optimizer step
+        gw = GpuWorkload(nf, wl, device, 1, keep_fp32=args.only == "quantize")
+        if args.only == "quantize":
+            obj = time_quantize(nf, gw, args, stream, device, world, peaks)
+        elif args.only == "merge":
+            obj = time_merge(nf, gw, args, stream, device, world)
+        else:
+            with torch.cuda.stream(stream):
+                gw.step(0)  # the backward fills dA, dB
+            obj = time_adamw(nf, gw, args, stream, device, world, peaks, l2)
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "phase": args.only, "n_gpus": world,
+                              "config": workload_config(wl, world), args.only: obj}), flush=True)
+        return
+
+    head, gw = time_workload(nf, wl, args, stream, device, world, peaks, l2, with_e2e=True)
+    quantize = time_quantize(nf, gw, args, stream, device, world, peaks) if gw.fp32 else None
+    optimizer = time_adamw(nf, gw, args, stream, device, world, peaks, l2) if wl.backward != "dx" else None
+    merge = time_merge(nf, gw, args, stream, device, world) if wl.quantize_timed and not args.no_merge else None
+    del gw
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+    few = None
+    if tensor_bound(wl) and not args.no_few:
+        fwl = workloads.WORKLOADS[FEW_TOKEN_WORKLOAD]
+        fobj, fgw = time_workload(nf, fwl, args, stream, device, world, peaks, l2, with_e2e=False)
+        del fgw
+        few = {k: fobj[k] for k in ("value", "unit", "ms_per_step", "roofline", "kernels", "launches_per_step",
+                                    "clocks", "config")}
+        few["steps"] = args.steps
 
     cpu_baseline = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -784,32 +886,23 @@ def run_ours(args, wl):
 
     if world > 1:
         dist.barrier()
-        for g in graphs:
-            del g
-        graphs.clear()
         dist.destroy_process_group()
     if rank != 0:
         return
-    line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic (seeded N(0, sigma) weights with 0.1% x10 outliers, N(0,1) activations)",
-            "config": dict(workload_config(wl), l2_flush="rotating %d encoded weight copies (%.0f MB > 4x L2)"
-                           % (copies, copies * wbytes / 1e6) if copies > 1 else "weights larger than 4x L2",
-                           graphs=bool(graphs),
-                           parallelism="dp%d%s" % (world, "" if world == 1 else
-                                                   " (all-reduce of dA, dB per step)" if exchange is not None
-                                                   else " (independent replicas: no exchange step)")),
-            "tflops": tflops,
-            "roofline": roofline,
-            "cpu_baseline": cpu_baseline,
-            "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "steps": e2e_steps},
-            "gpu_launches": int(round(launches_per_step * args.steps)) if launches_per_step else 0,
-            "kernels": kernel_table,
-            "clocks": clocks}
+    line = {"metric": METRIC, "value": head["value"], "unit": head["unit"], "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": DATA, "config": head["config"],
+            "roofline": head["roofline"], "cpu_baseline": cpu_baseline, "e2e": head["e2e"],
+            "gpu_launches": int(head["launches_per_step"] * args.steps),
+            "clocks": head["clocks"],
+            "tflops": head["tflops"], "weight_gbps": head["weight_gbps"],
+            "graphs": head["graphs"], "weight_copies": head["copies"],
+            "kernels": head["kernels"]}
     if quantize is not None:
         line["quantize"] = quantize
+    if few is not None:
+        line["few_token"] = few
     if optimizer is not None:
         line["optimizer"] = optimizer
     if merge is not None:
@@ -820,11 +913,13 @@ def run_ours(args, wl):
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--workload", default="q_proj4096_r64_m1-4-16", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--workload", default="llama65b_layer_r64_m2048", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--no-few", action="store_true", help="skip the few-token sub-object")
+    ap.add_argument("--no-merge", action="store_true", help="skip the merge + re-encoding phase")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--only", choices=("quantize", "merge", "optimizer"),

@@ -146,9 +146,12 @@ int nf4_quantize(const float* W, int64_t d_out, int64_t d_in, const nf4_tensor* 
  * array (16 MiB + 128 KiB) stays resident on every GPU that loads the library
  * until the process exits.  Larger weights return NF4_ERR_UNSUPPORTED_SHAPE.
  * The call allocates nothing; the caller still passes W and `out`.
- * The first call on a device looks up the array's device address with that
- * device current; make that first call before any stream capture on the
- * device.  Every call shares the one array, so calls whose kernels overlap
+ * Every call looks up the array's device address on the current device (a
+ * host-side lookup, nothing is cached), so the call stays correct after a
+ * cudaDeviceReset, which may place the array elsewhere.  The first call on a
+ * device may load the library's device code there; make that first call
+ * before any stream capture on the device.  Every call shares the one array,
+ * so calls whose kernels overlap
  * on the GPU (different streams without ordering) race on it; calls on one
  * stream, or otherwise ordered, are safe.  Results are bit-identical to
  * nf4_quantize.  Returns NF4_OK or an error status (no message is recorded).
@@ -304,6 +307,20 @@ const char* nf4lora_last_error_string(void);
  * bounded wait since the last call.  Returns NF4_ERR_CUDA if the
  * synchronisation fails. */
 int nf4lora_device_status(void* stream);
+
+/*
+ * nf4lora_check_bounded_wait -- self-check of the failure detector shared by
+ * every kernel above (no counterpart in the pages: it guards the library, not
+ * the method).  Enqueues one small kernel that, like a layer kernel, holds
+ * tensor memory and has a bulk copy in flight, and then waits on a barrier
+ * that nothing ever arrives on.  The wait gives up after limit_ns
+ * nanoseconds (1e5 <= limit_ns <= 1e9), records NF4_ERR_TIMEOUT in the
+ * device status word, drains the copy, frees the tensor memory and returns,
+ * so the context stays usable.  A later nf4lora_device_status() returns
+ * NF4_ERR_TIMEOUT once, then NF4_OK.  Allocates nothing.  Returns NF4_OK
+ * (enqueued), NF4_ERR_INVALID_ARG, NF4_ERR_DEVICE or NF4_ERR_CUDA.
+ */
+int nf4lora_check_bounded_wait(int64_t limit_ns, void* stream);
 
 /* ---------------------------------------------------------------- tracing */
 

@@ -32,7 +32,8 @@ ABI_SYMBOLS = ("nf4_packed_bytes", "nf4_tensor_from_buffer", "nf4_quantize_works
                "qlora_fwd_workspace_bytes", "qlora_bwd_workspace_bytes", "nf4_quantize",
                "nf4_quantize_noalloc", "nf4_dequantize", "qlora_linear_fwd", "qlora_linear_bwd",
                "nf4_merge_workspace_bytes", "nf4_merge_lora", "nf4_merge_requantize",
-               "lora_adamw_step", "nf4lora_last_error_string", "nf4lora_device_status", "nf4lora_trace_start",
+               "lora_adamw_step", "nf4lora_last_error_string", "nf4lora_device_status", "nf4lora_check_bounded_wait",
+               "nf4lora_trace_start",
                "nf4lora_trace_stop", "nf4lora_trace_count", "nf4lora_trace_get", "nf4lora_version")
 
 
@@ -83,6 +84,7 @@ def _load() -> ctypes.CDLL:
         "lora_adamw_step": (I, [ctypes.POINTER(AdamwTensorStruct), I, ctypes.POINTER(AdamwHparamsStruct), P]),
         "nf4lora_last_error_string": (ctypes.c_char_p, []),
         "nf4lora_device_status": (I, [P]),
+        "nf4lora_check_bounded_wait": (I, [I64, P]),
         "nf4lora_trace_start": (I, [I]),
         "nf4lora_trace_stop": (I, []),
         "nf4lora_trace_count": (I, []),
@@ -331,6 +333,13 @@ def lora_adamw_step(tensors, lr: float, beta1: float = 0.9, beta2: float = 0.999
 def device_status() -> None:
     """Raise Nf4Error(NF4_ERR_TIMEOUT) if a kernel abandoned a bounded wait."""
     _check(lib.nf4lora_device_status(_stream()))
+
+
+def check_bounded_wait(limit_ns: int = 1000000) -> None:
+    """Enqueue the library's self-check of its bounded waits: a kernel whose
+    wait on a barrier nothing arrives on gives up after limit_ns.  The next
+    device_status() then raises Nf4Error(NF4_ERR_TIMEOUT)."""
+    _check(lib.nf4lora_check_bounded_wait(int(limit_ns), _stream()))
 
 
 def trace_start(max_launches: int = 4096) -> None:

@@ -78,21 +78,27 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
     return ok != 0;
 }
 
-// Bounded wait for the phase with the given parity to complete.  On timeout
-// it records the failure in the device status word and in *abort (a shared
-// flag every role polls) and returns false.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+// Bounded wait for the phase with the given parity to complete, giving up
+// after limit_ns.  On timeout it records the failure in the device status
+// word and in *abort (a shared flag every role polls) and returns false.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                              uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
+        if (global_timer_ns() - t0 > limit_ns) {
             *abort = 1;
             atomicExch(&g_device_status, kStatusTimeout);
             return false;
         }
     }
+}
+
+// The wait every kernel of the library uses: bounded by kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+    return mbar_wait_for(bar, parity, abort, kWaitLimitNs);
 }
 
 // Bounded wait that ignores the abort flag: used only to drain copies that
@@ -143,6 +149,16 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
 __device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes)
                  : "memory");
+}
+
+// Untiled bulk copy of `bytes` (a multiple of 16) from global memory to this
+// CTA's shared memory, completing on `bar` (both addresses 16-byte aligned).
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
 }
 
 // ------------------------------------------------------------------ programmatic dependent launch

@@ -6,11 +6,13 @@
 // file-scope __device__ array sized for kNoallocMaxBlocks blocks, which every
 // GPU that loads the library keeps until the process exits.  Host code must
 // not pass the symbol itself to a kernel (on the host it names a stand-in, not
-// device memory): the device address is fetched with cudaGetSymbolAddress
-// once per device, with that device current, on the first call made on it.
+// device memory): the device address is looked up with cudaGetSymbolAddress on
+// every call, with the caller's device current.  The lookup is a host-side
+// table read once the library's device code is loaded on that device, so
+// nothing is cached across calls: after a cudaDeviceReset (which unloads the
+// module, so the array may come back at another address) the next call finds
+// the new address.
 #include <cuda_runtime.h>
-
-#include <mutex>
 
 #include "nf4lora.h"
 #include "kernels.h"
@@ -26,22 +28,10 @@ constexpr int64_t kScratchBytes = kAbsmaxBytes + kNoallocMaxTiles * 8;   // + 12
 
 static __device__ __align__(256) unsigned char g_quant_scratch[kScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of g_quant_scratch on the current device (set-up on first use).
-cudaError_t scratch_address(int dev, void** out) {
-    std::lock_guard<std::mutex> lk(g_mu);
-    if (g_scratch_ptr[dev] == nullptr) {
-        void* p = nullptr;
-        const cudaError_t e = cudaGetSymbolAddress(&p, g_quant_scratch);
-        if (e != cudaSuccess) return e;
-        g_scratch_ptr[dev] = p;
-    }
-    *out = g_scratch_ptr[dev];
-    return cudaSuccess;
-}
+// Device address of g_quant_scratch on the current device.  The first call
+// on a device may load the library's device code there (lazy module loading),
+// which is why the first call should come before any stream capture.
+cudaError_t scratch_address(void** out) { return cudaGetSymbolAddress(out, g_quant_scratch); }
 
 }  // namespace
 
@@ -64,13 +54,13 @@ extern "C" int nf4_quantize_noalloc(const float* W, int64_t d_out, int64_t d_in,
     const int64_t n = d_out * d_in, n_blocks = n / 64;
     if (n_blocks > kNoallocMaxBlocks) return NF4_ERR_UNSUPPORTED_SHAPE;  // beyond the fixed scratch
     int dev = 0, major = 0, sms = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return NF4_ERR_CUDA;
+    if (cudaGetDevice(&dev) != cudaSuccess) return NF4_ERR_CUDA;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return NF4_ERR_CUDA;
     if (major != 10) return NF4_ERR_DEVICE;
     void* scratch = nullptr;
-    if (scratch_address(dev, &scratch) != cudaSuccess) return NF4_ERR_CUDA;
+    if (scratch_address(&scratch) != cudaSuccess) return NF4_ERR_CUDA;
     unsigned char* base = static_cast<unsigned char*>(scratch);
     // Every scratch word the kernels read is written earlier in the same call,
     // so nothing needs clearing between calls.

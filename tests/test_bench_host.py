@@ -55,12 +55,36 @@ def test_default_step_is_six_passes_over_the_weight():
 
 def test_reference_arm_json_line():
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
-                          "--warmup", "3"], capture_output=True, text=True, timeout=600, cwd=ROOT)
+                          "--warmup", "3"], capture_output=True, text=True, timeout=900, cwd=ROOT)
     assert out.returncode == 0, out.stderr[-2000:]
     lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
     assert len(lines) == 1
     d = json.loads(lines[0])
-    assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == "GB/s" and d["higher_is_better"]
+    # the default workload is the LLaMA-65B layer's linears, a tensor-bound step
+    assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == "TFLOP/s" and d["higher_is_better"]
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
-    assert d["e2e"] == {"value": d["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
-    assert d["config"]["workload"] == "q_proj4096_r64_m1-4-16"
+    assert d["e2e"] == {"value": d["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert d["config"] == bench.workload_config(workloads.WORKLOADS["llama65b_layer_r64_m2048"], 1)
+
+
+def test_both_arms_time_the_same_oracle_sample():
+    """cpu_baseline (GPU arm) and the reference arm describe one sample and
+    one config: the same rows of the same module, the same keys."""
+    for name, wl in workloads.WORKLOADS.items():
+        mod = wl.modules[0]
+        rows = bench.oracle_rows(mod)
+        assert rows * mod.d_in % (64 * 256) == 0 or rows == mod.d_out
+        assert rows <= mod.d_out
+        assert bench.oracle_unit(wl) == ("TFLOP/s" if max(wl.tokens) > 16 else "GB/s")
+        assert bench.workload_config(wl, 1) == bench.workload_config(wl, 1)
+
+
+def test_kernel_flops_split_the_pass_flops():
+    """The fused forward and input-gradient kernels carry the base product and
+    their own rank-r term; with the LoRA-down / V products (2 M r K, 2 M r N)
+    they add up to the pass flops of the layer formulas."""
+    for K, N, m, r in ((4096, 11008, 4096, 64), (8192, 8192, 2048, 64), (512, 512, 16, 8)):
+        fwd = bench.kernel_flops(N, K, m, r, "nf4_gemm_fwd")
+        dx = bench.kernel_flops(N, K, m, r, "nf4_gemm_dx")
+        assert fwd + 2 * m * r * K == bench.pass_flops(N, K, m, r, "fwd")
+        assert dx + 2 * m * r * N == bench.pass_flops(N, K, m, r, "dx")

@@ -4,8 +4,9 @@ from X, one shared workspace).
 
 A full oracle product at these sizes takes minutes, so the check is sampled
 where the outputs separate cleanly: rows of Y and dX depend only on their own
-token row, so a handful of rows (first, last, and seeded picks) is compared
-against the fp64 oracle computed for those rows alone.  The rank-r gradients
+token row, so one row inside every 128-row tile, the rows on both sides of
+every 256-row boundary, and the first and last row are compared against the
+fp64 oracle computed for those rows alone (every column of each).  The rank-r gradients
 dA and dB need no pass over the base weight and are compared whole.  The
 weight the kernels decode is first checked to be, byte for byte, the oracle's
 encoding of the same fp32 weight, so the sampled rows test the fused GEMMs
@@ -41,11 +42,26 @@ CASES = [(name, i, mod) for name, wl in workloads.WORKLOADS.items() if name != "
          for i, mod in _unique_modules(wl)]
 
 
-def _sample_rows(m, k=6, seed=7):
+def _sample_rows(m):
+    """Token rows that reach every CTA tile of a launch: one row inside each
+    128-row tile (at an offset that moves from tile to tile, 128 t + 37 t mod
+    128), both rows on either side of every 256-row boundary (where the 256-
+    and 128-row tile shapes split differently), and the first and last row."""
     rows = {0, m - 1}
-    rng = np.random.default_rng(seed)
-    rows.update(int(x) for x in rng.integers(0, m, size=k))
+    for t in range((m + 127) // 128):
+        rows.add(min(m - 1, 128 * t + (37 * t) % 128))
+    for b in range(256, m, 256):
+        rows.update((b - 1, b))
     return np.array(sorted(rows))
+
+
+def test_sample_rows_cover_every_tile():
+    for m in (17, 300, 2048, 4096, 8192):
+        rows = _sample_rows(m)
+        assert rows[0] == 0 and rows[-1] == m - 1
+        assert set(rows // 128) == set(range((m + 127) // 128))
+        for b in range(256, m, 256):
+            assert b - 1 in rows and b in rows
 
 
 @pytest.mark.parametrize("name,index,mod", CASES,

@@ -43,6 +43,7 @@ CASES = [
     (9472, 1408, 5, 16),      # few tokens: two splits of 11 blocks (a ragged block quad)
     (256, 256, 7, 256),       # largest rank, few tokens
     (384, 256, 40, 256),      # largest rank, many tokens
+    (5120, 4096, 4096, 16),   # 320 CTA tiles of 256 x 256: more than two waves, compared whole
 ]
 
 
