@@ -322,6 +322,19 @@ int nf4lora_device_status(void* stream);
  */
 int nf4lora_check_bounded_wait(int64_t limit_ns, void* stream);
 
+/*
+ * Debug build (no counterpart in the pages).  Built with NF4LORA_DEBUG
+ * (python nf4_base_lora_b200/build.py --debug -> lib/libnf4lora_debug.so),
+ * the kernels check the index and alignment of their memory accesses; the
+ * first check that fails records (site << 16) | source line and that access
+ * is skipped instead of faulting.  nf4lora_debug_site() synchronises
+ * `stream`, stores that word (0 if every check passed) in *site and clears
+ * it.  In a release build no check runs and the word stays 0.
+ * nf4lora_debug_build() returns 1 in a debug build, 0 otherwise.
+ */
+int nf4lora_debug_site(void* stream, unsigned int* site);
+int nf4lora_debug_build(void);
+
 /* ---------------------------------------------------------------- tracing */
 
 /* Start timing the library's own kernel launches (host-side tracing): each

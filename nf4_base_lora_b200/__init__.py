@@ -20,7 +20,9 @@ from typing import Optional, Tuple
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "lib", "libnf4lora.so")
+# NF4LORA_DEBUG=1 loads the bounds-checking build (python nf4_base_lora_b200/build.py --debug)
+LIB_PATH = os.path.join(_HERE, "lib", "libnf4lora_debug.so" if os.environ.get("NF4LORA_DEBUG") == "1"
+                        else "libnf4lora.so")
 
 NF4_OK = 0
 STATUS_NAMES = {0: "NF4_OK", -1: "NF4_ERR_INVALID_ARG", -2: "NF4_ERR_UNSUPPORTED_SHAPE",
@@ -33,7 +35,7 @@ ABI_SYMBOLS = ("nf4_packed_bytes", "nf4_tensor_from_buffer", "nf4_quantize_works
                "nf4_quantize_noalloc", "nf4_dequantize", "qlora_linear_fwd", "qlora_linear_bwd",
                "nf4_merge_workspace_bytes", "nf4_merge_lora", "nf4_merge_requantize",
                "lora_adamw_step", "nf4lora_last_error_string", "nf4lora_device_status", "nf4lora_check_bounded_wait",
-               "nf4lora_trace_start",
+               "nf4lora_debug_site", "nf4lora_debug_build", "nf4lora_trace_start",
                "nf4lora_trace_stop", "nf4lora_trace_count", "nf4lora_trace_get", "nf4lora_version")
 
 
@@ -61,8 +63,8 @@ class Nf4Error(RuntimeError):
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
-        raise ImportError("libnf4lora.so is not built (%s); run python -m nf4_base_lora_b200.build"
-                          % LIB_PATH)
+        raise ImportError("%s is not built; run python nf4_base_lora_b200/build.py%s"
+                          % (LIB_PATH, " --debug" if "debug" in os.path.basename(LIB_PATH) else ""))
     lib = ctypes.CDLL(LIB_PATH)
     P, I64, SZ, I, F = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int,
                         ctypes.c_float)
@@ -85,6 +87,8 @@ def _load() -> ctypes.CDLL:
         "nf4lora_last_error_string": (ctypes.c_char_p, []),
         "nf4lora_device_status": (I, [P]),
         "nf4lora_check_bounded_wait": (I, [I64, P]),
+        "nf4lora_debug_site": (I, [P, ctypes.POINTER(ctypes.c_uint)]),
+        "nf4lora_debug_build": (I, []),
         "nf4lora_trace_start": (I, [I]),
         "nf4lora_trace_stop": (I, []),
         "nf4lora_trace_count": (I, []),
@@ -340,6 +344,14 @@ def check_bounded_wait(limit_ns: int = 1000000) -> None:
     wait on a barrier nothing arrives on gives up after limit_ns.  The next
     device_status() then raises Nf4Error(NF4_ERR_TIMEOUT)."""
     _check(lib.nf4lora_check_bounded_wait(int(limit_ns), _stream()))
+
+
+def debug_site() -> int:
+    """The first failed access check of a debug build, as (site << 16) | line,
+    since the last call (0: none; always 0 in a release build)."""
+    v = ctypes.c_uint(0)
+    _check(lib.nf4lora_debug_site(_stream(), ctypes.byref(v)))
+    return int(v.value)
 
 
 def trace_start(max_launches: int = 4096) -> None:

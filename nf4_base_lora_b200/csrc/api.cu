@@ -14,6 +14,7 @@
 
 namespace nf4lora {
 __device__ int g_device_status = 0;
+__device__ unsigned int g_debug_site = 0;
 }
 
 using namespace nf4lora;
@@ -367,6 +368,32 @@ int nf4lora_device_status(void* stream) {
     return ok();
 }
 
-const char* nf4lora_version(void) { return "nf4lora 0.1.0 sm_100a"; }
+int nf4lora_debug_site(void* stream, unsigned int* site) {
+    if (site == nullptr) return fail(NF4_ERR_INVALID_ARG, "site is NULL");
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return fail(NF4_ERR_CUDA, "stream synchronisation failed: %s", cudaGetErrorString(cudaGetLastError()));
+    unsigned int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_debug_site, sizeof(v)) != cudaSuccess ||
+        cudaMemcpyToSymbol(g_debug_site, &zero, sizeof(zero)) != cudaSuccess)
+        return fail(NF4_ERR_CUDA, "debug word access failed");
+    *site = v;
+    return ok();
+}
+
+int nf4lora_debug_build(void) {
+#ifdef NF4LORA_DEBUG
+    return 1;
+#else
+    return 0;
+#endif
+}
+
+const char* nf4lora_version(void) {
+#ifdef NF4LORA_DEBUG
+    return "nf4lora 0.2.0 sm_100a debug";
+#else
+    return "nf4lora 0.2.0 sm_100a";
+#endif
+}
 
 }  // extern "C"

@@ -22,6 +22,37 @@ constexpr int kStatusTimeout = 1;
 // in nanoseconds).  A healthy wait lasts microseconds.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
+// ------------------------------------------------------------------ debug checks
+// In a build with NF4LORA_DEBUG defined, kernels check the index and
+// alignment of their shared- and global-memory accesses; the first check that
+// fails records (site << 16) | source line in g_debug_site and the access is
+// skipped, so a bad index reports itself instead of faulting.  In a release
+// build every check is the constant true and costs nothing.
+extern __device__ unsigned int g_debug_site;
+
+#ifdef NF4LORA_DEBUG
+__device__ __forceinline__ bool debug_check(bool ok, unsigned int site, unsigned int line) {
+    if (!ok) atomicCAS(&g_debug_site, 0u, (site << 16) | (line & 0xFFFFu));
+    return ok;
+}
+#define NF4_CHECK(cond, site) ::nf4lora::debug_check((cond), (site), __LINE__)
+#else
+#define NF4_CHECK(cond, site) true
+#endif
+
+// [p, p + bytes) lies inside [lo, lo + len) and p is `align`-byte aligned:
+// in_span for global memory (generic addresses), in_smem for shared memory,
+// whose alignment rules apply to the shared-window address.
+__device__ __forceinline__ bool in_span(const void* p, uint32_t bytes, const void* lo, int64_t len, uint32_t align) {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p), b = reinterpret_cast<uintptr_t>(lo);
+    return a >= b && a + bytes <= b + static_cast<uintptr_t>(len) && (a % align) == 0;
+}
+__device__ __forceinline__ bool in_smem(const void* p, uint32_t bytes, const void* lo, int64_t len, uint32_t align) {
+    const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(p));
+    const uint32_t b = static_cast<uint32_t>(__cvta_generic_to_shared(lo));
+    return a >= b && static_cast<int64_t>(a) + bytes <= static_cast<int64_t>(b) + len && (a % align) == 0;
+}
+
 __device__ __forceinline__ uint64_t global_timer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -52,14 +83,20 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// A waiting thread is suspended in hardware until the phase completes or
+// kSuspendHintNs passes, instead of spinning: a spinning warp would issue
+// instructions (and take issue slots from the warps doing the work) for as
+// long as it waits.
+constexpr uint32_t kSuspendHintNs = 1000000;  // 1 ms per try; the bound below still applies
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "n"(kSuspendHintNs)
         : "memory");
     return ok != 0;
 }
@@ -70,10 +107,10 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "n"(kSuspendHintNs)
         : "memory");
     return ok != 0;
 }

@@ -1,45 +1,25 @@
-// Few-token (M <= 16) fused NF4-LoRA forward, weights decoded straight into
-// the operand registers of warp-level tensor instructions (mma.sync
-// m16n8k16, bf16 in, fp32 accumulate):
-//
-//   Y[t, n] = sum_k X[t, k] W_hat[n, k] + sum_j T2[t, j] [B | B][n, j]
-//
-// ("第 04 篇：QLoRA 原理" §6.1-§6.3; T2 holds the rank-r intermediate
-// s X A^T as a bf16 hi | lo pair.)
-//
-// With at most 16 tokens the layer is a streamed matrix-vector product: per
-// weight the GPU reads 4.127 bits and decodes them, and the 16 dot products
-// are a small tail.  One thread (TMA) streams the CTA's packed codes into
-// shared memory; each thread then decodes its slice with a register-held
-// codebook (csrc/decode.cuh), restores bf16(level[code] * s_b) and hands the pairs to the
-// tensor instruction as its A fragment (16 weight rows x 16 k; the activations
-// are the B fragment, 16 k x 8 tokens).  A decoded weight never goes back to
-// memory.
-//
-// The contraction index inside each 16-wide MMA chunk is permuted so that a
-// thread's operand comes from whole 64-blocks (one scale per row and block):
-// thread (g, q) of a warp covers weight rows g and g + 8 of a 16-row group
-// and block q of four consecutive blocks; chunk c takes k = 4c .. 4c+3 of each
-// thread's block.  The activation fragment uses the same permutation, which
-// leaves the sums unchanged.
+// Few-token (M <= 16) fused NF4-LoRA input gradient on warp-level tensor
+// instructions (mma.sync m16n8k16, bf16 in, fp32 accumulate), the weight
+// decoded on chip and never written back to memory ("第 04 篇：QLoRA 原理"
+// §2.4: the frozen base still passes the input gradient).  The forward
+// counterpart is in fewfwd.cu.
 //
 // Split-K: the CTAs that share one output tile form a thread-block cluster
 // along grid.z.  Inside a CTA every warp puts its fp32 partials into shared
-// memory and each thread adds up four outputs (the two warps of a row group,
+// memory and each thread adds up four outputs (the warps of a column block,
 // in order); every CTA of rank > 0 then pushes its partial tile into a slot of
 // rank 0 (distributed shared memory) before a cluster barrier, after which
 // rank 0 adds the slots in rank order and writes bf16 rows.  The rank-r
-// extension, once the kernel that produced T2 has finished (programmatic
+// extension, once the kernel that produced V2 has finished (programmatic
 // dependent launch), is shared out among the ranks.  The summation order is
 // fixed, so the result is the same on every run.
 //
 // Launch overlap: the kernel releases its own dependents as soon as it starts
-// (the next layer call's rank-r kernel may then stage its factor rows while
-// this one runs), and asks L2 for the rows of B its extension will read.  It
-// reads the activations and the encoded weight before its own wait: the
-// rank-r kernel it depends on released it only after waiting for the kernel
-// before that, so every earlier write is complete; global loads go through
-// L2 (ld.global.cg), never a possibly stale L1 line.
+// and asks L2 for the rows of A its extension will read.  It reads dY and the
+// encoded weight before its own wait: the rank-r kernel it depends on
+// released it only after waiting for the kernel before that, so every
+// earlier write is complete; global loads go through L2 (ld.global.cg),
+// never a possibly stale L1 line.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -61,10 +41,6 @@ constexpr int kTok = 16;           // token rows of the MMA
 constexpr int kMaxSplit = 8;       // CTAs per cluster (portable cluster size)
 constexpr int kPartFloats = kTile * kTok;  // one CTA's partial tile, fp32
 
-// contraction blocks staged per segment (four block quads: two per warp of a
-// row group, 16 x 16 x 64 activations = 4 16-byte pieces per thread)
-constexpr int kFwdSegBlocks = 16;
-
 __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                           uint32_t b0, uint32_t b1) {
     asm volatile(
@@ -81,268 +57,10 @@ __device__ __forceinline__ void split_range(int total, int parts, int p, int& be
     end = begin + per + (p < extra ? 1 : 0);
 }
 
-// Tensor-instruction roles: A = 16 weight rows x 16 k (decoded), B = 16 k x 8
-// tokens (activations), D = 16 rows x 8 tokens; two MMAs cover 16 tokens.
-// A warp works on 16 weight rows (thread (g, q): rows g and g + 8) and four
-// consecutive 64-blocks at a time (thread q streams block q whole: 32 bytes
-// per row, one scale per row); MMA chunk c of the quad takes k = 4c .. 4c+3
-// of each thread's block.
-//
-// Activations are staged as [token][block][64 + 4] with a token stride of
-// 16 x 68 + 16 elements (2208 bytes): the 8-byte fragment loads of a
-// half-warp (4 tokens x 4 blocks) then fall in 16 different bank pairs.
-constexpr int kFwdBlockStride = 68;
-constexpr int kFwdTokStride = kFwdSegBlocks * kFwdBlockStride + 16;
-constexpr int kFwdQuadBytes = kTile * 128;  // codes of 4 blocks x 128 rows
-constexpr int kFwdMaxSplit = kMaxSplit;      // partial-tile slots of rank 0: kFwdMaxSplit - 1
-constexpr int kFwdSmemV2 = 1024 + 4 * kFwdQuadBytes + (kFwdMaxSplit - 1) * kPartFloats * 4 + kTok * kFwdTokStride * 2;
 // row stride (floats) of the per-warp partial tiles [token][row] gathered for
 // the reduction: 132 puts the 8 x 4 (row, token) pairs of a fragment store in
 // distinct banks and keeps the rows 16-byte aligned
 constexpr int kSumStride = 132;
-static_assert(2 * kTok * kSumStride * 4 <= 4 * kFwdQuadBytes, "the forward's partial tiles reuse the code buffers");
-
-// Asks L2 for `bytes` (a multiple of 16) from a 16-byte aligned address.
-__device__ __forceinline__ void prefetch_l2_range(const void* src, uint32_t bytes) {
-    const uint8_t* p = static_cast<const uint8_t*>(src);
-    for (uint32_t off = 0; off < bytes; off += 32768u) prefetch_l2_bulk(p + off, min(32768u, bytes - off));
-}
-
-// Registers capped at 96 (48K of the SM's 64K) so that the CTAs of the kernel
-// producing T2, which this one overlaps, keep room on the same SM.
-__global__ void __maxnreg__(96) k_few_fwd(const __grid_constant__ CUtensorMap map_codes, const FewArgs a) {
-    extern __shared__ __align__(16) uint8_t smem_raw[];
-    __shared__ uint64_t bar_q[4];
-    __shared__ int s_abort;
-    pdl_launch_dependents();
-    // [codes: 4 quads x 128 rows x 128 B, 128-byte swizzle; after the loop the
-    //  partial tiles][slots for the other ranks' partial tiles][activations]
-    const uint32_t raw = smem_u32(smem_raw);
-    uint8_t* s_codes = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-    float* s_part = reinterpret_cast<float*>(s_codes + 4 * kFwdQuadBytes);  // [kFwdMaxSplit - 1][2048]
-    uint16_t* sX = reinterpret_cast<uint16_t*>(s_part + (kFwdMaxSplit - 1) * kPartFloats);  // [16][kFwdTokStride]
-
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, q = lane & 3;
-    const int rgp = warp & 7;  // 16-row group of the CTA's 128 rows
-    const int qs = warp >> 3;  // which block quads: qs, qs + 2
-    const int splits = static_cast<int>(gridDim.z);
-    const int rank = static_cast<int>(cluster_ctarank());
-    const int M = a.M, N = a.N, K = a.K;
-    const int bpr = K / 64;
-    int kb0, kb1;
-    split_range(bpr, splits, rank, kb0, kb1);
-    const int row0 = blockIdx.x * kTile;
-    // thread 0: barriers, then the first segment's codes in flight at once
-    auto issue_codes = [&](int seg0, int nquads) {
-        for (int j = 0; j < nquads; ++j) {
-            mbar_arrive_expect_tx(&bar_q[j], kFwdQuadBytes);
-            tma_load_2d(s_codes + j * kFwdQuadBytes, &map_codes, &bar_q[j], 32 * (seg0 + 4 * j), row0);
-        }
-    };
-    const int nq_first = (min(kb1 - kb0, kFwdSegBlocks) + 3) / 4;
-    if (tid == 0) {
-        for (int j = 0; j < 4; ++j) mbar_init(&bar_q[j], 1);
-        s_abort = 0;
-        fence_barrier_init();
-        if (kb0 < kb1) {
-            tma_prefetch_desc(&map_codes);
-            issue_codes(kb0, nq_first);
-        }
-    } else if (tid == 32 && a.ext_act != nullptr) {
-        // the CTA's rows of B (N is a multiple of 8, so the range is too)
-        const int rows = min(kTile, N - row0);
-        prefetch_l2_range(a.ext_w + static_cast<int64_t>(row0) * a.r, static_cast<uint32_t>(rows * a.r * 2));
-    }
-
-    const int lr = 16 * rgp + g;  // local row of nA (nB = nA + 8 is local row lr + 8)
-    const int nA = row0 + lr, nB = nA + 8;
-    const bool okA = nA < N, okB = nB < N;
-    const bool two_halves = M > 8;
-
-    float acc0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, acc1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    __syncthreads();
-    cluster_arrive_relaxed();  // barriers initialised (made visible by the init fence)
-    const float mu = __ldcg(a.scale_mean);
-    volatile int* abort_flag = &s_abort;
-
-    int seg_i = 0, issued_seg = 0, issued_nq = kb0 < kb1 ? nq_first : 0;
-    for (int seg0 = kb0; seg0 < kb1; seg0 += kFwdSegBlocks, ++seg_i) {
-        const int nb = min(kb1 - seg0, kFwdSegBlocks);
-        const int nquads = (nb + 3) / 4;
-        const int nbp = 4 * nquads;  // staged blocks; nb .. nbp - 1 and tokens >= M are zeros
-        if (seg_i > 0) {
-            __syncthreads();  // the previous segment's codes and activations are no longer read
-            if (*abort_flag) break;  // the same value in every thread: no wait can set it here
-            if (tid == 0) issue_codes(seg0, nquads);
-            issued_seg = seg_i;
-            issued_nq = nquads;
-        }
-        // activations of the segment (L2 hits) and this thread's block scales;
-        // a token row has `per` 16-byte pieces (128 in a full segment)
-        const int per = nbp * 8;
-        uint4 xv[4];
-        int xt[4], xpc[4];
-#pragma unroll
-        for (int p = 0; p < 4; ++p) {
-            const int i = tid + p * kThreads;
-            xt[p] = per == 128 ? (i >> 7) : i / per;
-            xpc[p] = i - xt[p] * per;
-            xv[p] = make_uint4(0, 0, 0, 0);
-            if (xt[p] < M && xpc[p] < nb * 8)
-                xv[p] = __ldcg(reinterpret_cast<const uint4*>(a.act + static_cast<int64_t>(xt[p]) * K + seg0 * 64) +
-                              xpc[p]);
-        }
-        int qA[2], qB[2];
-        float aA[2], aB[2];
-        bool inA[2], inB[2];  // the item's block exists (else its weights are zero)
-#pragma unroll
-        for (int it = 0; it < 2; ++it) {
-            const int j = qs + 2 * it, lb = 4 * j + q, blk = seg0 + lb;
-            const bool in = j < nquads && lb < nb;
-            const int64_t biA = static_cast<int64_t>(nA) * bpr + blk, biB = static_cast<int64_t>(nB) * bpr + blk;
-            inA[it] = in && okA;
-            inB[it] = in && okB;
-            qA[it] = inA[it] ? static_cast<int>(__ldcg(a.qscale + biA)) : 0;
-            qB[it] = inB[it] ? static_cast<int>(__ldcg(a.qscale + biB)) : 0;
-            aA[it] = inA[it] ? __ldcg(a.scale2 + (biA >> 8)) : 0.0f;
-            aB[it] = inB[it] ? __ldcg(a.scale2 + (biB >> 8)) : 0.0f;
-        }
-#pragma unroll
-        for (int p = 0; p < 4; ++p) {
-            const int t = xt[p], pc = xpc[p];
-            if (t < kTok) {
-                const int lb = pc >> 3, kk = (pc & 7) * 8;
-                uint2* dst = reinterpret_cast<uint2*>(sX + t * kFwdTokStride + lb * kFwdBlockStride + kk);
-                dst[0] = make_uint2(xv[p].x, xv[p].y);
-                dst[1] = make_uint2(xv[p].z, xv[p].w);
-            }
-        }
-        __syncthreads();
-        // decode and multiply as each quad's codes land
-#pragma unroll
-        for (int it = 0; it < 2; ++it) {
-            const int j = qs + 2 * it;
-            if (j >= nquads) break;
-            if (!mbar_wait(&bar_q[j], seg_i & 1, abort_flag)) break;
-            const int lb = 4 * j + q;
-            const float sA = inA[it] ? nf4_block_scale(static_cast<int8_t>(qA[it]), aA[it], mu) : 0.0f;
-            const float sB = inB[it] ? nf4_block_scale(static_cast<int8_t>(qB[it]), aB[it], mu) : 0.0f;
-            // rows lr and lr + 8 of the quad, 16-byte chunks 2q and 2q + 1 (block q), swizzled by row
-            const uint8_t* qbase = s_codes + j * kFwdQuadBytes;
-            const uint4 cA0 = *reinterpret_cast<const uint4*>(qbase + lr * 128 + (((2 * q) ^ g) << 4));
-            const uint4 cA1 = *reinterpret_cast<const uint4*>(qbase + lr * 128 + (((2 * q + 1) ^ g) << 4));
-            const uint4 cB0 = *reinterpret_cast<const uint4*>(qbase + (lr + 8) * 128 + (((2 * q) ^ g) << 4));
-            const uint4 cB1 = *reinterpret_cast<const uint4*>(qbase + (lr + 8) * 128 + (((2 * q + 1) ^ g) << 4));
-            const uint16_t* x0 = sX + g * kFwdTokStride + lb * kFwdBlockStride;
-            const uint16_t* x8 = x0 + 8 * kFwdTokStride;
-            const uint32_t wA[8] = {cA0.x, cA0.y, cA0.z, cA0.w, cA1.x, cA1.y, cA1.z, cA1.w};
-            const uint32_t wB[8] = {cB0.x, cB0.y, cB0.z, cB0.w, cB1.x, cB1.y, cB1.z, cB1.w};
-            uint32_t PA[4], HA[4], PB[4], HB[4];  // register codebooks of the two rows
-            nf4_table(sA, PA, HA);
-            nf4_table(sB, PB, HB);
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                uint32_t a0, a1, a2, a3;  // rows g (a0, a2) and g + 8 (a1, a3), k = 4c + {0,1} / {2,3}
-                nf4_lookup4(wA[c >> 1] >> (16 * (c & 1)), PA, HA, a0, a2);
-                nf4_lookup4(wB[c >> 1] >> (16 * (c & 1)), PB, HB, a1, a3);
-                const uint2 xb = *reinterpret_cast<const uint2*>(x0 + 4 * c);
-                mma_16816(acc0, a0, a1, a2, a3, xb.x, xb.y);
-                if (two_halves) {
-                    const uint2 xc = *reinterpret_cast<const uint2*>(x8 + 4 * c);
-                    mma_16816(acc1, a0, a1, a2, a3, xc.x, xc.y);
-                }
-            }
-        }
-    }
-    if (tid == 0 && *abort_flag) {
-        // let the copies still in flight land before the CTA can exit
-        for (int j = 0; j < issued_nq; ++j) mbar_drain(&bar_q[j], issued_seg & 1);
-    }
-
-    // rank-r extension: [B | B] rows of this CTA against T2, once the kernel
-    // producing T2 has finished (programmatic dependent launch).  Its 16-wide
-    // chunks are dealt round-robin to the ranks of the cluster (and to the two
-    // warps of a row group), which add them to the partials they push.
-    if (a.pdl) pdl_wait();
-    if (a.ext_act != nullptr) {
-        const int nchunks = 2 * a.r64 / 16;
-        const uint16_t* bA = a.ext_w + static_cast<int64_t>(nA) * a.r;
-        const uint16_t* bB = a.ext_w + static_cast<int64_t>(nB) * a.r;
-        for (int ch = rank + splits * qs; ch < nchunks; ch += 2 * splits) {
-            const int j0 = ch * 16;
-            const int jj = (j0 % a.r64) + 2 * q;  // column of B (same in both halves of T2)
-            const bool lo_ok = jj < a.r, hi_ok = jj + 8 < a.r;
-            const uint32_t a0 = (okA && lo_ok) ? __ldcg(reinterpret_cast<const uint32_t*>(bA + jj)) : 0u;
-            const uint32_t a1 = (okB && lo_ok) ? __ldcg(reinterpret_cast<const uint32_t*>(bB + jj)) : 0u;
-            const uint32_t a2 = (okA && hi_ok) ? __ldcg(reinterpret_cast<const uint32_t*>(bA + jj + 8)) : 0u;
-            const uint32_t a3 = (okB && hi_ok) ? __ldcg(reinterpret_cast<const uint32_t*>(bB + jj + 8)) : 0u;
-            const uint16_t* t0 = a.ext_act + static_cast<int64_t>(g) * 2 * a.r64 + j0 + 2 * q;
-            const uint32_t b0 = g < M ? __ldcg(reinterpret_cast<const uint32_t*>(t0)) : 0u;
-            const uint32_t b1 = g < M ? __ldcg(reinterpret_cast<const uint32_t*>(t0 + 8)) : 0u;
-            mma_16816(acc0, a0, a1, a2, a3, b0, b1);
-            if (two_halves) {
-                const uint16_t* t8 = t0 + 8 * 2 * a.r64;
-                const uint32_t c0 = g + 8 < M ? __ldcg(reinterpret_cast<const uint32_t*>(t8)) : 0u;
-                const uint32_t c1 = g + 8 < M ? __ldcg(reinterpret_cast<const uint32_t*>(t8 + 8)) : 0u;
-                mma_16816(acc1, a0, a1, a2, a3, c0, c1);
-            }
-        }
-    }
-
-    // every warp's partials into shared memory (the code buffers are free:
-    // every copy has landed and been read), s_sum[qs][token][local row]; then
-    // thread tid adds up token tid / 32, rows 4 (tid % 32) .. + 3: the two
-    // warps of the row group in order
-    __syncthreads();
-    float* s_sum = reinterpret_cast<float*>(s_codes);
-    {
-        // acc0: tokens 2q, 2q + 1 of rows lr (0, 1) and lr + 8 (2, 3); acc1: tokens + 8
-        float* d0 = s_sum + qs * kTok * kSumStride + (2 * q) * kSumStride + lr;
-        float* d8 = d0 + 8 * kSumStride;
-        d0[0] = acc0[0];
-        d0[kSumStride] = acc0[1];
-        d0[8] = acc0[2];
-        d0[kSumStride + 8] = acc0[3];
-        d8[0] = acc1[0];
-        d8[kSumStride] = acc1[1];
-        d8[8] = acc1[2];
-        d8[kSumStride + 8] = acc1[3];
-    }
-    __syncthreads();
-    const int ot = tid >> 5, orow = 4 * (tid & 31);
-    float4 o = *reinterpret_cast<const float4*>(s_sum + ot * kSumStride + orow);
-    {
-        const float4 o1 = *reinterpret_cast<const float4*>(s_sum + (kTok + ot) * kSumStride + orow);
-        o.x += o1.x;
-        o.y += o1.y;
-        o.z += o1.z;
-        o.w += o1.w;
-    }
-    // ranks > 0 push into rank 0's slots; the cluster barrier (every CTA has
-    // started, then every push is visible) orders them before rank 0's sums,
-    // and no CTA touches another's shared memory after it
-    cluster_wait_acquire();
-    if (rank != 0)
-        st_cluster_f4(cluster_map(smem_u32(s_part + (rank - 1) * kPartFloats + 4 * tid), 0), o.x, o.y, o.z, o.w);
-    cluster_arrive_release();
-    cluster_wait_acquire();
-    if (rank == 0) {
-        for (int rk = 1; rk < splits; ++rk) {
-            const float4 v = *reinterpret_cast<const float4*>(s_part + (rk - 1) * kPartFloats + 4 * tid);
-            o.x += v.x;
-            o.y += v.y;
-            o.z += v.z;
-            o.w += v.w;
-        }
-        const int n = row0 + orow;  // N is a multiple of 8: rows n .. n + 3 all exist or none does
-        if (ot < M && n < N) {
-            uint2 packed;
-            packed.x = pack_bf16x2(o.x, o.y);
-            packed.y = pack_bf16x2(o.z, o.w);
-            *reinterpret_cast<uint2*>(a.out + static_cast<int64_t>(ot) * N + n) = packed;
-        }
-    }
-}
 
 // ---------------------------------------------------------------- input gradient
 // dX^T[k, t] = sum_n W_hat[n, k] dY[t, n] + sum_j [A ; A][j, k] V2[t, j]:
@@ -642,15 +360,7 @@ cudaError_t launch_cluster(Kern kern, bool (&configured)[64], int smem, const ch
 
 }  // namespace
 
-int few_max_split(bool forward) { return forward ? kFwdMaxSplit : kDxMaxSplit; }
-
-cudaError_t launch_few_fwd(const CUtensorMap& map_codes, const FewArgs& a, int splits, cudaStream_t stream) {
-    if (a.M < 1 || a.M > kTok || a.K % 64 != 0 || a.N % 8 != 0 || splits > a.K / 64 || splits > kFwdMaxSplit)
-        return cudaErrorInvalidValue;
-    static bool configured[64] = {};
-    return launch_cluster(k_few_fwd, configured, kFwdSmemV2, "nf4_gemm_fwd_few", a, (a.N + kTile - 1) / kTile, splits,
-                          stream, map_codes);
-}
+int few_max_split(bool forward) { return forward ? kMaxSplit : kDxMaxSplit; }
 
 cudaError_t launch_few_dx(const CUtensorMap& map_codes, const FewArgs& a, int splits, cudaStream_t stream) {
     if (a.M < 1 || a.M > kTok || a.K % 64 != 0 || a.N % 8 != 0 || splits > (a.N + 31) / 32 || splits > kDxMaxSplit ||

@@ -65,9 +65,28 @@ struct FewArgs {
     int pdl;                   // launched as a programmatic dependent of the ext_act producer
 };
 int few_max_split(bool forward);
-// map_codes: the packed codes as bytes [N, K / 2], box {128 bytes, 128 rows},
+// Plan of the few-token forward (fewfwd.cu): clusters of cs CTAs along the
+// contraction, O weight octets per cluster, the ring of quad stages and the
+// shared-memory layout.
+struct FewFwdPlan {
+    int cs;          // CTAs per cluster (1 or 2), splitting the block quads
+    int O;           // weight octets (8 rows) per cluster
+    int clusters;
+    int nq0;         // block quads of rank 0 (rank 1 takes the rest)
+    int WQ;          // quad slots: warps w with w % WQ equal share a quad
+    int NR;          // ring stages
+    int nbox, box_rows, code_bytes;  // TMA boxes of the codes of one stage
+    int xbox_rows, xbox_bytes;       // TMA box of one activation block: 16 token rows (8 when M <= 8)
+    int slot;        // bytes per stage (codes + activations), a multiple of 1024
+    int qrow, q_bytes, step_bytes, t2_bytes, b_bytes, recv_bytes;
+    int smem;        // dynamic shared memory
+};
+bool few_fwd_plan(int M, int N, int K, int r, int num_sms, FewFwdPlan* out);
+// map_codes: the packed codes as bytes [N, K / 2], box {128 bytes, plan.box_rows
+// rows}, 128-byte swizzle; map_x: the activations as bf16 [M, K], box {64, 16},
 // 128-byte swizzle
-cudaError_t launch_few_fwd(const CUtensorMap& map_codes, const FewArgs& a, int splits, cudaStream_t stream);
+cudaError_t launch_few_fwd(const CUtensorMap& map_codes, const CUtensorMap& map_x, const FewArgs& a,
+                           const FewFwdPlan& p, cudaStream_t stream);
 // map_codes: the packed codes as bytes [N, K / 2], box {64 bytes, 256 rows},
 // 64-byte swizzle
 cudaError_t launch_few_dx(const CUtensorMap& map_codes, const FewArgs& a, int splits, cudaStream_t stream);

@@ -377,9 +377,18 @@ int layer_fwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, fl
                                  c.stream)) != cudaSuccess)
             return -2;
         const FewArgs fa = few_args(c, X, static_cast<int>(M), T2, B, r, r64, Y);
-        const int splits = few_splits(ceil_div(c.d_out, 128), static_cast<int>(c.d_in / 64), c.num_sms, true);
-        if (!map_codes(&m.a, c.codes, c.d_out, c.d_in, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return -1;
-        return note(launch_few_fwd(m.a, fa, splits, c.stream)) == cudaSuccess ? 0 : -2;
+        FewFwdPlan fp;
+        if (!few_fwd_plan(static_cast<int>(M), static_cast<int>(c.d_out), static_cast<int>(c.d_in), r, c.num_sms,
+                          &fp))
+        {
+            note(cudaErrorInvalidConfiguration);
+            return -2;
+        }
+        if (!map_codes(&m.a, c.codes, c.d_out, c.d_in, 128, static_cast<uint32_t>(fp.box_rows),
+                       CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !map_bf16(&m.b, X, c.d_in, M, c.d_in, static_cast<uint32_t>(fp.xbox_rows)))
+            return -1;
+        return note(launch_few_fwd(m.a, m.b, fa, fp, c.stream)) == cudaSuccess ? 0 : -2;
     }
     int rc = lora_down(c, A, r, s, X, M, T2, T_saved, part);
     if (rc) return rc;

@@ -44,6 +44,8 @@ CASES = [
     (256, 256, 7, 256),       # largest rank, few tokens
     (384, 256, 40, 256),      # largest rank, many tokens
     (5120, 4096, 4096, 16),   # 320 CTA tiles of 256 x 256: more than two waves, compared whole
+    (11008, 4096, 16, 64),    # few tokens, 19 weight octets per cluster: the stage ring is refilled
+    (4096, 11008, 3, 64),     # few tokens, 22 block quads per CTA: the stage ring is refilled
 ]
 
 
