@@ -74,6 +74,7 @@ constexpr int kMaxRing = 24;
 constexpr int kMaxPPW = 4;                        // octet pairs per warp (largest instance)
 constexpr int kMaxBoxRows = 256;
 constexpr int kStageLoads = 8;                    // scale codes per thread per staging round
+constexpr int kEarly = 2;                         // stages thread 0 issues before the CTA barrier
 constexpr int kSmemLimit = 227 * 1024 - 1024;  // room for the static barriers
 
 __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -146,7 +147,7 @@ __device__ __forceinline__ Geometry geometry(const FewArgs& a, const FewFwdPlan&
     return G;
 }
 
-template <int PPW>
+template <int PPW, bool TWO>
 __global__ void __launch_bounds__(kThreads, 1) k_few_fwd(const __grid_constant__ CUtensorMap map_codes,
                                                           const __grid_constant__ CUtensorMap map_x, const FewArgs a,
                                                           const FewFwdPlan p) {
@@ -174,8 +175,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_few_fwd(const __grid_constant__
     const int WP = kWarps / p.WQ;
     const int P = (G.Oc + 1) / 2;  // octet pairs of this CTA
     const bool lora = a.ext_act != nullptr && G.own1 > G.own0;
-    const bool two = M > 8;        // tokens 8 .. 15 exist
-    const int n_first = min(p.NR, G.nqc);  // stages issued at the start, one per warp
+    constexpr bool two = TWO;      // tokens 8 .. 15 exist (M > 8)
+    const int n_first = min(p.NR, G.nqc);  // stages issued at the start
 
     // one stage: the codes of the O octets and the quad's four activation
     // blocks (rows beyond M and blocks beyond K read as zeros), by one thread
@@ -195,6 +196,25 @@ __global__ void __launch_bounds__(kThreads, 1) k_few_fwd(const __grid_constant__
                 tma_load_2d(xs + b * kXBox, &map_x, &bar_full[slot], 256 * quad + 64 * b, 0);
         s_fills[slot] += 1;
     };
+
+    // thread 0 initialises the barriers and puts the first stages in flight
+    // before anything else, so that the weight stream starts at once
+    if (tid == 0) {
+        tma_prefetch_desc(&map_codes);
+        tma_prefetch_desc(&map_x);
+        for (int i = 0; i < p.NR; ++i) {
+            mbar_init(&bar_full[i], 1);
+            s_done[i] = 0;
+            s_fills[i] = 0;
+        }
+        mbar_init(&bar_lora, 1);
+        mbar_init(&bar_b, 1);
+        mbar_init(&bar_staged, kWarps * 31);  // lanes 1 .. 31 of every warp stage the scales
+        s_abort = 0;
+        s_lora = 0;
+        fence_barrier_init();
+        for (int i = 0; i < min(n_first, kEarly); ++i) issue_stage(i);
+    }
 
     // lanes 1 .. 31 of every warp stage the block-scale codes and the
     // second-level steps of the CTA's rows; their first loads are issued
@@ -223,35 +243,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_few_fwd(const __grid_constant__
         }
     }
     const float mu = __ldcg(a.scale_mean);
-
-    if (tid == 0) {
-        for (int i = 0; i < p.NR; ++i) {
-            mbar_init(&bar_full[i], 1);
-            s_done[i] = 0;
-            s_fills[i] = 0;
-        }
-        mbar_init(&bar_lora, 1);
-        mbar_init(&bar_b, 1);
-        mbar_init(&bar_staged, kWarps * 31);  // lanes 1 .. 31 of every warp stage the scales
-        s_abort = 0;
-        s_lora = 0;
-        fence_barrier_init();
-    }
     __syncthreads();
     if (p.cs > 1) cluster_arrive_relaxed();  // barriers initialised; the peer may address this CTA after its wait
     volatile int* abort_flag = &s_abort;
 
     if (lane == 0) {
-        // the first stages in flight at once, one per warp, so that no warp
-        // waits for another's copies to be queued
-        if (warp < n_first) {
-            if (warp == 0) {
-                tma_prefetch_desc(&map_codes);
-                tma_prefetch_desc(&map_x);
-            }
-            issue_stage(warp);
-        }
-        if (warp == n_first - 1 && lora) {
+        // the rest of the first stages, spread over the warps (the ring may
+        // be deeper than there are warps)
+        for (int i = warp; i < n_first; i += kWarps)
+            if (i >= kEarly) issue_stage(i);
+        if (warp == min(n_first, kWarps) - 1 && lora) {
             // the owner's rows of B (written before the kernel this one depends
             // on released it), then T2 once that kernel has finished
             const uint32_t bb = static_cast<uint32_t>(8 * (G.own1 - G.own0) * 2 * a.r);
@@ -314,12 +315,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_few_fwd(const __grid_constant__
 
     const uint32_t ring_s = smem_u32(ring);
     const uint32_t sq_s = smem_u32(s_q), sstep_s = smem_u32(s_step);
-    // the lane's 8-byte code pieces of its block, rotated by q words (a row's
+    // the lane's 8-byte code pieces of its block in the order jj ^ q (a row's
     // 16-byte chunks are swizzled by the row index, which is g modulo 8)
     uint32_t coff[4];
 #pragma unroll
     for (int jj = 0; jj < 4; ++jj) {
-        const int pw = (jj + q) & 3;
+        const int pw = jj ^ q;
         coff[jj] = static_cast<uint32_t>((((2 * q + (pw >> 1)) ^ g) << 4) + 8 * (pw & 1));
     }
     for (int i = wq; i < G.nqc; i += p.WQ) {
@@ -330,7 +331,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_few_fwd(const __grid_constant__
         (void)st;
         const int bl = 4 * i + q;                    // this lane's block, relative to kb0
         const bool blk_ok = G.kb0 + bl < G.kb1;
-        const uint32_t x0 = st_s + p.code_bytes + q * kXBox + g * 128;  // block q, token g (g + 8: + 1024)
+        // block q, token g (g + 8: + 1024); the 16-byte chunk of word j is
+        // j ^ 2q, stored at chunk j ^ 2q ^ g of the swizzled row (x0 is
+        // 128-byte aligned, so the XOR reaches only the chunk bits)
+        const uint32_t x0 = (st_s + p.code_bytes + q * kXBox + g * 128) | (((2 * q) ^ g) << 4);
 #pragma unroll
         for (int pp = 0; pp < PPW; ++pp) {
             const int pr = wp + pp * WP;
@@ -364,11 +368,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_few_fwd(const __grid_constant__
                 }
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
-                    // rotated word j = stored word (j + 2q) & 7: chunks 2 cw, 2 cw + 1 of the
-                    // lane's block and the activations of the same 16-byte chunk
-                    const uint32_t xoff = ((((j + 2 * q) & 7) ^ g) << 4);
-                    const uint4 xa = lds128(x0 + xoff);                                   // tokens 0 .. 7
-                    const uint4 xb = two ? lds128(x0 + 1024 + xoff) : make_uint4(0, 0, 0, 0);  // tokens 8 .. 15
+                    // word j of the walk = stored word j ^ 2q of the lane's block and
+                    // the activations of the same 16-byte chunk
+                    const uint32_t xj = x0 ^ static_cast<uint32_t>(j << 4);
+                    const uint4 xa = lds128(xj);                                       // tokens 0 .. 7
+                    const uint4 xb = two ? lds128(xj + 1024) : make_uint4(0, 0, 0, 0);  // tokens 8 .. 15
                     uint32_t r0[4], r1[4];  // A fragments of the two chunks: rows g, g + 8
                     {
                         const uint32_t sel = w[0][j] & 0x77777777u;
@@ -376,13 +380,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_few_fwd(const __grid_constant__
                         lookup4_sel(sel, pick, PT[0], HT[0], r0[0], r0[2]);
                         lookup4_sel(sel >> 16, pick >> 16, PT[0], HT[0], r1[0], r1[2]);
                     }
-                    if (has1) {
+                    {
+                        // a missing second octet has zero codes and a zero table
                         const uint32_t sel = w[1][j] & 0x77777777u;
                         const uint32_t pick = ((w[1][j] >> 1) & 0x44444444u) | 0x32103210u;
                         lookup4_sel(sel, pick, PT[1], HT[1], r0[1], r0[3]);
                         lookup4_sel(sel >> 16, pick >> 16, PT[1], HT[1], r1[1], r1[3]);
-                    } else {
-                        r0[1] = r0[3] = r1[1] = r1[3] = 0u;
                     }
                     mma_16816(acc[pp][0], r0[0], r0[1], r0[2], r0[3], xa.x, xa.y);
                     mma_16816(acc[pp][0], r1[0], r1[1], r1[2], r1[3], xa.z, xa.w);
@@ -559,19 +562,20 @@ int max_clusters_of_two(int smem) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, k_few_fwd<kMaxPPW>, &cfg) != cudaSuccess) n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, k_few_fwd<kMaxPPW, true>, &cfg) != cudaSuccess) n = 0;
     cached[dev] = n;
     cached_smem[dev] = smem;
     return n;
 }
 
-template <int PPW>
+template <int PPW, bool TWO>
 bool configure_kernel() {
     cudaFuncAttributes fa{};
-    if (cudaFuncGetAttributes(&fa, k_few_fwd<PPW>) != cudaSuccess || fa.maxThreadsPerBlock < kThreads) return false;
-    return cudaFuncSetAttribute(k_few_fwd<PPW>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) ==
+    if (cudaFuncGetAttributes(&fa, k_few_fwd<PPW, TWO>) != cudaSuccess || fa.maxThreadsPerBlock < kThreads)
+        return false;
+    return cudaFuncSetAttribute(k_few_fwd<PPW, TWO>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) ==
                cudaSuccess &&
-           cudaFuncSetAttribute(k_few_fwd<PPW>, cudaFuncAttributePreferredSharedMemoryCarveout,
+           cudaFuncSetAttribute(k_few_fwd<PPW, TWO>, cudaFuncAttributePreferredSharedMemoryCarveout,
                                 cudaSharedmemCarveoutMaxShared) == cudaSuccess;
 }
 
@@ -579,7 +583,9 @@ bool configure(int dev) {
     static bool configured[64] = {};
     if (dev < 0 || dev >= 64) return false;
     if (!configured[dev]) {
-        if (!configure_kernel<2>() || !configure_kernel<4>()) return false;
+        if (!configure_kernel<2, false>() || !configure_kernel<4, false>() || !configure_kernel<2, true>() ||
+            !configure_kernel<4, true>())
+            return false;
         configured[dev] = true;
     }
     return true;
@@ -665,8 +671,12 @@ cudaError_t launch_few_fwd(const CUtensorMap& map_codes, const CUtensorMap& map_
     cfg.numAttrs = n;
     TraceScope trace("nf4_gemm_fwd_few", stream);
     const int P = (p.O + 1) / 2, WP = kWarps / p.WQ;
-    if ((P + WP - 1) / WP <= 2) return cudaLaunchKernelEx(&cfg, k_few_fwd<2>, map_codes, map_x, a, p);
-    return cudaLaunchKernelEx(&cfg, k_few_fwd<4>, map_codes, map_x, a, p);
+    const bool two = a.M > 8;
+    if ((P + WP - 1) / WP <= 2)
+        return two ? cudaLaunchKernelEx(&cfg, k_few_fwd<2, true>, map_codes, map_x, a, p)
+                   : cudaLaunchKernelEx(&cfg, k_few_fwd<2, false>, map_codes, map_x, a, p);
+    return two ? cudaLaunchKernelEx(&cfg, k_few_fwd<4, true>, map_codes, map_x, a, p)
+               : cudaLaunchKernelEx(&cfg, k_few_fwd<4, false>, map_codes, map_x, a, p);
 }
 
 }  // namespace nf4lora

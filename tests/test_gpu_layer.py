@@ -46,6 +46,7 @@ CASES = [
     (5120, 4096, 4096, 16),   # 320 CTA tiles of 256 x 256: more than two waves, compared whole
     (11008, 4096, 16, 64),    # few tokens, 19 weight octets per cluster: the stage ring is refilled
     (4096, 11008, 3, 64),     # few tokens, 22 block quads per CTA: the stage ring is refilled
+    (256, 16384, 5, 16),      # few tokens, one octet per cluster: a ring of 24 stages, deeper than the 16 warps
 ]
 
 
