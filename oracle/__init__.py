@@ -88,6 +88,9 @@ def _load():
         lib.oracle_num_groups.argtypes = [I64]
         lib.oracle_packed_bytes.restype = I64
         lib.oracle_packed_bytes.argtypes = [I64]
+        lib.oracle_nf4_dequantize_scales.argtypes = [P, P, I64, P]
+        lib.oracle_packed_bytes_nodq.restype = I64
+        lib.oracle_packed_bytes_nodq.argtypes = [I64]
         _lib = lib
     return _lib
 
@@ -131,6 +134,12 @@ def num_groups(n: int) -> int:
 
 def packed_bytes(n: int) -> int:
     return int(_load().oracle_packed_bytes(n))
+
+
+def packed_bytes_nodq(n: int) -> int:
+    """Storage of the encoding without double quantisation (codes and one
+    fp32 scale per block)."""
+    return int(_load().oracle_packed_bytes_nodq(n))
 
 
 def absmax(w: np.ndarray) -> np.ndarray:
@@ -212,13 +221,35 @@ def dequantize_bits(packed: np.ndarray, q: np.ndarray, a2: np.ndarray, mu: float
     return out
 
 
+def quantize_nodq(w: np.ndarray) -> Dict[str, np.ndarray]:
+    """The encoding without double quantisation ("第 04 篇" §5.1: one fp32
+    scale per block of 64): packed codes and the fp32 absmax of each block,
+    stored as is."""
+    w = np.ascontiguousarray(w, np.float32)
+    amax = absmax(w)
+    codes = encode(w, amax)
+    return {"packed": pack(codes), "absmax": amax, "codes": codes}
+
+
+def dequantize_scales_bits(packed: np.ndarray, scales: np.ndarray, n: int) -> np.ndarray:
+    """bfloat16 bit patterns of bf16(level[code] * s_b) with the fp32 block
+    scales given, length n."""
+    out = np.zeros(n, np.uint16)
+    _load().oracle_nf4_dequantize_scales(_p(np.ascontiguousarray(packed, np.uint8)),
+                                         _p(np.ascontiguousarray(scales, np.float32)), n, _p(out))
+    return out
+
+
 def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
     return (bits.astype(np.uint32) << 16).view(np.float32)
 
 
 def dequantize(qt: Dict[str, np.ndarray], shape) -> np.ndarray:
-    """Dequantised weight as fp32 (every value exactly a bfloat16)."""
+    """Dequantised weight as fp32 (every value exactly a bfloat16), from
+    either encoding (``quantize`` or ``quantize_nodq``)."""
     n = int(np.prod(shape))
+    if "q" not in qt:
+        return bf16_bits_to_f32(dequantize_scales_bits(qt["packed"], qt["absmax"], n)).reshape(shape)
     bits = dequantize_bits(qt["packed"], qt["q"], qt["a2"], float(qt["mu"]), n)
     return bf16_bits_to_f32(bits).reshape(shape)
 

@@ -274,6 +274,22 @@ void oracle_nf4_dequantize(const uint8_t* packed, const int8_t* q,
     }
 }
 
+/* Dequantised weight from plain fp32 block scales (the encoding without
+ * double quantisation, [QP] §5.1: one 32-bit scale per block of 64):
+ * w_hat = bf16(c[code] * s_b) with s_b = scale[b], the same look-up, scale
+ * and conversion as above without the two-level restore. */
+void oracle_nf4_dequantize_scales(const uint8_t* packed, const float* scale,
+                                  int64_t n, uint16_t* w_bf16) {
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) {
+        float s = scale[i / NF4_BLOCK];
+        uint8_t byte = packed[i / 2];
+        uint8_t code = (i % 2 == 0) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 15);
+        float v = NF4_LEVELS[code] * s;
+        w_bf16[i] = oracle_bf16_bits(v);
+    }
+}
+
 /* Whole encoding of one tensor, in the pages' order. */
 void oracle_nf4_quantize(const float* w, int64_t n, uint8_t* packed,
                          int8_t* q, float* a2, float* mu_out, float* absmax_ws,
@@ -292,4 +308,10 @@ void oracle_nf4_quantize(const float* w, int64_t n, uint8_t* packed,
  * §8.1). */
 int64_t oracle_packed_bytes(int64_t n) {
     return (n + 1) / 2 + oracle_num_blocks(n) + 4 * oracle_num_groups(n) + 4;
+}
+
+/* Storage without double quantisation: n/2 code bytes and one fp32 scale per
+ * block ([QP] §5.1: 32 bits per 64 weights, 0.5 bit per weight). */
+int64_t oracle_packed_bytes_nodq(int64_t n) {
+    return (n + 1) / 2 + 4 * oracle_num_blocks(n);
 }
