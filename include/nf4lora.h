@@ -79,6 +79,14 @@ typedef enum {
  *   scale_mean  [1] fp32, the mean of all first-level absmax scales.
  * Restored block scale: s_b = fp32(qscale_b * fp32(scale2_g / 127)) + mean;
  * weight: w_hat = bf16_rne(fp32(level[code] * s_b))  ([QP] §6.1).
+ *
+ * The same codes with plain fp32 block scales (no double quantisation,
+ * [QP] §5.1: one 32-bit scale per block of 64 weights, 0.5 bit per weight):
+ *   absmax      [n_b] fp32, the absmax a_b of each block, stored as is.
+ * A tensor with absmax != NULL is in this format: s_b = absmax_b, and qscale,
+ * scale2 and scale_mean are not read (they may be NULL).  With absmax ==
+ * NULL the double-quantised scales above are used.  Every entry point below
+ * accepts either format.
  */
 typedef struct {
     int64_t d_out;
@@ -87,6 +95,7 @@ typedef struct {
     int8_t* qscale;
     float* scale2;
     float* scale_mean;
+    float* absmax;
 } nf4_tensor;
 
 /* ---------------------------------------------------------------- sizing */
@@ -98,10 +107,19 @@ typedef struct {
 size_t nf4_packed_bytes(int64_t d_out, int64_t d_in);
 
 /* Fill `t` with pointers into one caller-owned device buffer `base` of
- * `bytes` >= nf4_packed_bytes(d_out, d_in) bytes (256-byte aligned).  Host
- * only; touches no device memory.  Returns NF4_OK or an error status. */
+ * `bytes` >= nf4_packed_bytes(d_out, d_in) bytes (256-byte aligned); sets
+ * t->absmax = NULL (the double-quantised format).  Host only; touches no
+ * device memory.  Returns NF4_OK or an error status. */
 int nf4_tensor_from_buffer(nf4_tensor* t, void* base, size_t bytes, int64_t d_out,
                            int64_t d_in);
+
+/* The same for the fp32-block-scale format (no double quantisation): the
+ * codes and one fp32 scale per block, each part padded to 256 bytes; the
+ * unpadded storage is n/2 + 4 n_b bytes, 4.5 bits per weight ([QP] §5.1).
+ * nf4_tensor_from_buffer_nodq sets qscale, scale2 and scale_mean to NULL. */
+size_t nf4_packed_bytes_nodq(int64_t d_out, int64_t d_in);
+int nf4_tensor_from_buffer_nodq(nf4_tensor* t, void* base, size_t bytes, int64_t d_out,
+                                int64_t d_in);
 
 /* Workspace (device bytes, 256-byte aligned) that each call needs. */
 size_t nf4_quantize_workspace_bytes(int64_t d_out, int64_t d_in);
@@ -125,9 +143,12 @@ size_t qlora_bwd_workspace_bytes(int64_t M, int64_t d_out, int64_t d_in, int r);
  *      tree (adjacent pairs, level by level) ([QP] §5.2);
  *   5. per group of 256 blocks, scale2 = max |a_b - mean| and
  *      qscale_b = rint((a_b - mean) / scale2 * 127) ([QP] §5.2, §3.3).
+ * When out->absmax != NULL (the fp32-block-scale format) steps 4 and 5 are
+ * skipped: a_b itself is written to out->absmax, and ws may be NULL.
  * Requirements: d_out >= 1, d_in >= 64, d_in % 64 == 0; W 16-byte aligned;
- * ws >= nf4_quantize_workspace_bytes(d_out, d_in).  Results are bit-identical
- * to the stated arithmetic on every run.  Non-finite W is undefined.
+ * ws >= nf4_quantize_workspace_bytes(d_out, d_in) for the double-quantised
+ * format.  Results are bit-identical to the stated arithmetic on every run.
+ * Non-finite W is undefined.
  */
 int nf4_quantize(const float* W, int64_t d_out, int64_t d_in, const nf4_tensor* out,
                  void* ws, size_t ws_bytes, void* stream);
@@ -145,7 +166,9 @@ int nf4_quantize(const float* W, int64_t d_out, int64_t d_in, const nf4_tensor* 
  * at most 4,194,304 blocks of 64 weights (d_out * d_in <= 268,435,456); that
  * array (16 MiB + 128 KiB) stays resident on every GPU that loads the library
  * until the process exits.  Larger weights return NF4_ERR_UNSUPPORTED_SHAPE.
- * The call allocates nothing; the caller still passes W and `out`.
+ * The call allocates nothing; the caller still passes W and `out`.  An
+ * `out` in the fp32-block-scale format (out->absmax != NULL) needs no scratch
+ * and so has no such size limit.
  * Every call looks up the array's device address on the current device (a
  * host-side lookup, nothing is cached), so the call stays correct after a
  * cudaDeviceReset, which may place the array elsewhere.  The first call on a

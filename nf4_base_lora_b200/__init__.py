@@ -30,7 +30,8 @@ STATUS_NAMES = {0: "NF4_OK", -1: "NF4_ERR_INVALID_ARG", -2: "NF4_ERR_UNSUPPORTED
                 -6: "NF4_ERR_TIMEOUT", -7: "NF4_ERR_DEVICE"}
 
 # Every symbol the C ABI exports (include/nf4lora.h), in declaration order.
-ABI_SYMBOLS = ("nf4_packed_bytes", "nf4_tensor_from_buffer", "nf4_quantize_workspace_bytes",
+ABI_SYMBOLS = ("nf4_packed_bytes", "nf4_tensor_from_buffer", "nf4_packed_bytes_nodq",
+               "nf4_tensor_from_buffer_nodq", "nf4_quantize_workspace_bytes",
                "qlora_fwd_workspace_bytes", "qlora_bwd_workspace_bytes", "nf4_quantize",
                "nf4_quantize_noalloc", "nf4_dequantize", "qlora_linear_fwd", "qlora_linear_bwd",
                "nf4_merge_workspace_bytes", "nf4_merge_lora", "nf4_merge_requantize",
@@ -42,7 +43,8 @@ ABI_SYMBOLS = ("nf4_packed_bytes", "nf4_tensor_from_buffer", "nf4_quantize_works
 class Nf4TensorStruct(ctypes.Structure):
     _fields_ = [("d_out", ctypes.c_int64), ("d_in", ctypes.c_int64),
                 ("codes", ctypes.c_void_p), ("qscale", ctypes.c_void_p),
-                ("scale2", ctypes.c_void_p), ("scale_mean", ctypes.c_void_p)]
+                ("scale2", ctypes.c_void_p), ("scale_mean", ctypes.c_void_p),
+                ("absmax", ctypes.c_void_p)]
 
 
 class AdamwTensorStruct(ctypes.Structure):
@@ -72,6 +74,8 @@ def _load() -> ctypes.CDLL:
     sig = {
         "nf4_packed_bytes": (SZ, [I64, I64]),
         "nf4_tensor_from_buffer": (I, [S, P, SZ, I64, I64]),
+        "nf4_packed_bytes_nodq": (SZ, [I64, I64]),
+        "nf4_tensor_from_buffer_nodq": (I, [S, P, SZ, I64, I64]),
         "nf4_quantize_workspace_bytes": (SZ, [I64, I64]),
         "qlora_fwd_workspace_bytes": (SZ, [I64, I64, I64, I]),
         "qlora_bwd_workspace_bytes": (SZ, [I64, I64, I64, I]),
@@ -136,6 +140,10 @@ def nf4_packed_bytes(d_out: int, d_in: int) -> int:
     return int(lib.nf4_packed_bytes(d_out, d_in))
 
 
+def nf4_packed_bytes_nodq(d_out: int, d_in: int) -> int:
+    return int(lib.nf4_packed_bytes_nodq(d_out, d_in))
+
+
 def nf4_quantize_workspace_bytes(d_out: int, d_in: int) -> int:
     return int(lib.nf4_quantize_workspace_bytes(d_out, d_in))
 
@@ -149,18 +157,22 @@ def qlora_bwd_workspace_bytes(M: int, d_out: int, d_in: int, r: int) -> int:
 
 
 class NF4Tensor:
-    """An encoded weight: one device buffer holding the packed codes, the
-    int8 scale codes, the fp32 group scales and the fp32 mean."""
+    """An encoded weight: one device buffer holding the packed codes and the
+    block scales: with double_quant (the default) the int8 scale codes, the
+    fp32 group scales and the fp32 mean; without it one fp32 scale per block
+    of 64 weights."""
 
-    def __init__(self, d_out: int, d_in: int, device="cuda", buffer: Optional[torch.Tensor] = None):
-        nbytes = nf4_packed_bytes(d_out, d_in)
+    def __init__(self, d_out: int, d_in: int, device="cuda", buffer: Optional[torch.Tensor] = None,
+                 double_quant: bool = True):
+        nbytes = nf4_packed_bytes(d_out, d_in) if double_quant else nf4_packed_bytes_nodq(d_out, d_in)
         if nbytes == 0:
             raise Nf4Error(-2, "unsupported weight shape [%d, %d]" % (d_out, d_in))
         self.buffer = buffer if buffer is not None else torch.zeros(nbytes, dtype=torch.uint8, device=device)
         self.struct = Nf4TensorStruct()
-        _check(lib.nf4_tensor_from_buffer(ctypes.byref(self.struct), _ptr(self.buffer),
-                                          self.buffer.numel(), d_out, d_in))
+        fill = lib.nf4_tensor_from_buffer if double_quant else lib.nf4_tensor_from_buffer_nodq
+        _check(fill(ctypes.byref(self.struct), _ptr(self.buffer), self.buffer.numel(), d_out, d_in))
         self.d_out, self.d_in = d_out, d_in
+        self.double_quant = double_quant
 
     def _view(self, attr: str, dtype, count: int) -> torch.Tensor:
         off = getattr(self.struct, attr) - self.buffer.data_ptr()
@@ -184,18 +196,29 @@ class NF4Tensor:
     def scale_mean(self) -> torch.Tensor:
         return self._view("scale_mean", torch.float32, 1)
 
+    @property
+    def absmax(self) -> torch.Tensor:
+        """fp32 block scales (only without double quantisation)."""
+        if self.double_quant:
+            raise AttributeError("a double-quantised tensor stores no fp32 block scales")
+        return self._view("absmax", torch.float32, self.d_out * self.d_in // 64)
+
 
 # ---------------------------------------------------------------- entry points
 def nf4_quantize(W: torch.Tensor, out: Optional[NF4Tensor] = None,
-                 workspace: Optional[torch.Tensor] = None) -> NF4Tensor:
-    """Encode fp32 W [d_out, d_in] (CUDA) to NF4 + double-quantised scales.
-    `workspace` (uint8, >= nf4_quantize_workspace_bytes) is allocated when
-    not given."""
+                 workspace: Optional[torch.Tensor] = None, double_quant: bool = True) -> NF4Tensor:
+    """Encode fp32 W [d_out, d_in] (CUDA) to NF4 codes with double-quantised
+    scales, or with fp32 block scales when double_quant is False (the format
+    of `out` decides when it is given).  `workspace` (uint8, >=
+    nf4_quantize_workspace_bytes; only the double-quantised format uses it)
+    is allocated when not given."""
     if W.dtype != torch.float32 or not W.is_cuda or not W.is_contiguous() or W.dim() != 2:
         raise ValueError("W must be a contiguous 2-D float32 CUDA tensor")
     d_out, d_in = W.shape
-    out = out if out is not None else NF4Tensor(d_out, d_in, W.device)
-    ws = workspace if workspace is not None else _workspace(nf4_quantize_workspace_bytes(d_out, d_in), W.device)
+    out = out if out is not None else NF4Tensor(d_out, d_in, W.device, double_quant=double_quant)
+    ws = workspace
+    if ws is None and out.double_quant:
+        ws = _workspace(nf4_quantize_workspace_bytes(d_out, d_in), W.device)
     _check(lib.nf4_quantize(_ptr(W), d_out, d_in, ctypes.byref(out.struct), _ptr(ws),
                             0 if ws is None else ws.numel(), _stream()))
     return out
@@ -304,9 +327,10 @@ def nf4_merge_lora(w: NF4Tensor, A: torch.Tensor, B: torch.Tensor, scaling: floa
 
 def nf4_merge_requantize(w: NF4Tensor, A: torch.Tensor, B: torch.Tensor, scaling: float,
                          out: Optional[NF4Tensor] = None, workspace: Optional[torch.Tensor] = None) -> NF4Tensor:
-    """The merged weight encoded again (NF4 + double quantisation); `out` may be `w`."""
+    """The merged weight encoded again, in the format of `out` (when not
+    given, that of `w`); `out` may be `w`."""
     r = _adapter(w, A, B)
-    out = out if out is not None else NF4Tensor(w.d_out, w.d_in, A.device)
+    out = out if out is not None else NF4Tensor(w.d_out, w.d_in, A.device, double_quant=w.double_quant)
     ws = workspace if workspace is not None else _workspace(nf4_merge_workspace_bytes(w.d_out, w.d_in), A.device)
     _check(lib.nf4_merge_requantize(ctypes.byref(w.struct), _ptr(A), _ptr(B), r, scaling, ctypes.byref(out.struct),
                                     _ptr(ws), 0 if ws is None else ws.numel(), _stream()))

@@ -65,6 +65,13 @@ int check_tensor(const nf4_tensor* w) {
     if (!valid_weight_shape(w->d_out, w->d_in))
         return fail(NF4_ERR_UNSUPPORTED_SHAPE, "weight [%lld, %lld]: need d_out >= 1, d_in >= 64, d_in %% 64 == 0",
                     (long long)w->d_out, (long long)w->d_in);
+    if (w->absmax != nullptr) {
+        // fp32 block scales, no double quantisation
+        if (!w->codes) return fail(NF4_ERR_INVALID_ARG, "nf4_tensor has NULL codes");
+        if (!aligned16(w->codes) || !aligned16(w->absmax))
+            return fail(NF4_ERR_MISALIGNED, "nf4_tensor member not aligned (codes/absmax: 16 B)");
+        return NF4_OK;
+    }
     if (!w->codes || !w->qscale || !w->scale2 || !w->scale_mean)
         return fail(NF4_ERR_INVALID_ARG, "nf4_tensor has a NULL member");
     if (!aligned16(w->codes) || !aligned16(w->qscale) || !aligned16(w->scale2) ||
@@ -129,6 +136,31 @@ int nf4_tensor_from_buffer(nf4_tensor* t, void* base, size_t bytes, int64_t d_ou
     t->scale2 = reinterpret_cast<float*>(p);
     p += align256(ng * 4);
     t->scale_mean = reinterpret_cast<float*>(p);
+    t->absmax = nullptr;
+    return ok();
+}
+
+size_t nf4_packed_bytes_nodq(int64_t d_out, int64_t d_in) {
+    if (!valid_weight_shape(d_out, d_in)) return 0;
+    const int64_t n = d_out * d_in, nb = n / 64;
+    return static_cast<size_t>(align256(n / 2) + align256(nb * 4));
+}
+
+int nf4_tensor_from_buffer_nodq(nf4_tensor* t, void* base, size_t bytes, int64_t d_out, int64_t d_in) {
+    if (t == nullptr || base == nullptr) return fail(NF4_ERR_INVALID_ARG, "NULL tensor or buffer");
+    if (!valid_weight_shape(d_out, d_in))
+        return fail(NF4_ERR_UNSUPPORTED_SHAPE, "weight [%lld, %lld]: need d_in %% 64 == 0", (long long)d_out, (long long)d_in);
+    if (reinterpret_cast<uintptr_t>(base) & 255u) return fail(NF4_ERR_MISALIGNED, "buffer not 256-byte aligned");
+    if (bytes < nf4_packed_bytes_nodq(d_out, d_in)) return fail(NF4_ERR_INVALID_ARG, "buffer too small");
+    const int64_t n = d_out * d_in;
+    uint8_t* p = static_cast<uint8_t*>(base);
+    t->d_out = d_out;
+    t->d_in = d_in;
+    t->codes = p;
+    t->qscale = nullptr;
+    t->scale2 = nullptr;
+    t->scale_mean = nullptr;
+    t->absmax = reinterpret_cast<float*>(p + align256(n / 2));
     return ok();
 }
 
@@ -156,12 +188,22 @@ int nf4_quantize(const float* W, int64_t d_out, int64_t d_in, const nf4_tensor* 
     if (out->d_out != d_out || out->d_in != d_in)
         return fail(NF4_ERR_INVALID_ARG, "out describes [%lld, %lld], W is [%lld, %lld]", (long long)out->d_out,
                     (long long)out->d_in, (long long)d_out, (long long)d_in);
+    const int64_t n = d_out * d_in, nb = n / 64;
+    if (out->absmax != nullptr) {
+        // fp32 block scales: the encoder writes them directly, no workspace
+        int sms = 0;
+        rc = check_device(&sms);
+        if (rc) return rc;
+        cudaError_t e = launch_nf4_quantize(W, n, out->codes, nullptr, nullptr, nullptr, out->absmax, nullptr, sms,
+                                            static_cast<cudaStream_t>(stream));
+        if (e != cudaSuccess) return fail(NF4_ERR_CUDA, "nf4_quantize launch: %s", cudaGetErrorString(e));
+        return ok();
+    }
     rc = check_ws(ws, ws_bytes, quant_ws_bytes(d_out, d_in));
     if (rc) return rc;
     int sms = 0;
     rc = check_device(&sms);
     if (rc) return rc;
-    const int64_t n = d_out * d_in, nb = n / 64;
     uint8_t* w8 = static_cast<uint8_t*>(ws);
     float* absmax = reinterpret_cast<float*>(w8);
     double* tile_sums = reinterpret_cast<double*>(w8 + align256(nb * 4));
@@ -179,8 +221,8 @@ int nf4_dequantize(const nf4_tensor* w, uint16_t* W_hat, void* stream) {
     int sms = 0;
     rc = check_device(&sms);
     if (rc) return rc;
-    cudaError_t e = launch_nf4_dequantize(w->codes, w->qscale, w->scale2, w->scale_mean, w->d_out * w->d_in, W_hat,
-                                          sms, static_cast<cudaStream_t>(stream));
+    cudaError_t e = launch_nf4_dequantize(w->codes, w->qscale, w->scale2, w->scale_mean, w->absmax,
+                                          w->d_out * w->d_in, W_hat, sms, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail(NF4_ERR_CUDA, "nf4_dequantize launch: %s", cudaGetErrorString(e));
     return ok();
 }
@@ -199,7 +241,7 @@ int qlora_linear_fwd(const nf4_tensor* w, const uint16_t* A, const uint16_t* B, 
     int sms = 0;
     rc = check_device(&sms);
     if (rc) return rc;
-    LayerCtx c{w->codes, w->qscale, w->scale2, w->scale_mean, w->d_out, w->d_in, kPlanSMs,
+    LayerCtx c{w->codes, w->qscale, w->scale2, w->scale_mean, w->absmax, w->d_out, w->d_in, kPlanSMs,
                static_cast<cudaStream_t>(stream)};
     rc = layer_fwd(c, A, B, r, scaling, X, M, Y, T_saved, static_cast<uint8_t*>(ws));
     if (rc == -1) return fail(NF4_ERR_CUDA, "qlora_linear_fwd: tensor map encoding failed");
@@ -237,7 +279,7 @@ int qlora_linear_bwd(const nf4_tensor* w, const uint16_t* A, const uint16_t* B, 
     int sms = 0;
     rc = check_device(&sms);
     if (rc) return rc;
-    LayerCtx c{w->codes, w->qscale, w->scale2, w->scale_mean, w->d_out, w->d_in, kPlanSMs,
+    LayerCtx c{w->codes, w->qscale, w->scale2, w->scale_mean, w->absmax, w->d_out, w->d_in, kPlanSMs,
                static_cast<cudaStream_t>(stream)};
     rc = layer_bwd(c, A, B, r, scaling, X, T_saved, dY, M, dX, dA, dB, accumulate_grads,
                    static_cast<uint8_t*>(ws));
@@ -272,8 +314,8 @@ int nf4_merge_lora(const nf4_tensor* w, const uint16_t* A, const uint16_t* B, in
     int sms = 0;
     rc = check_device(&sms);
     if (rc) return rc;
-    const cudaError_t e = launch_merge_lora(w->codes, w->qscale, w->scale2, w->scale_mean, A, B, r, w->d_out, w->d_in,
-                                            scaling, W_merged, static_cast<cudaStream_t>(stream));
+    const cudaError_t e = launch_merge_lora(w->codes, w->qscale, w->scale2, w->scale_mean, w->absmax, A, B, r,
+                                            w->d_out, w->d_in, scaling, W_merged, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail(NF4_ERR_CUDA, "nf4_merge_lora launch: %s", cudaGetErrorString(e));
     return ok();
 }
@@ -298,13 +340,16 @@ int nf4_merge_requantize(const nf4_tensor* w, const uint16_t* A, const uint16_t*
     float* absmax = reinterpret_cast<float*>(w8 + align256(n * 4));
     double* tile_sums = reinterpret_cast<double*>(w8 + align256(n * 4) + align256(n / 64 * 4));
     const cudaStream_t st = static_cast<cudaStream_t>(stream);
-    cudaError_t e = launch_merge_lora(w->codes, w->qscale, w->scale2, w->scale_mean, A, B, r, w->d_out, w->d_in,
-                                      scaling, merged, st);
+    cudaError_t e = launch_merge_lora(w->codes, w->qscale, w->scale2, w->scale_mean, w->absmax, A, B, r, w->d_out,
+                                      w->d_in, scaling, merged, st);
     if (e != cudaSuccess) return fail(NF4_ERR_CUDA, "nf4_merge_requantize launch: %s", cudaGetErrorString(e));
     // the merged weight is complete before the encoder starts (an ordinary
     // launch), so `out` may be `w` itself
-    e = launch_nf4_quantize(merged, n, out->codes, out->qscale, out->scale2, out->scale_mean, absmax, tile_sums, sms,
-                            st);
+    if (out->absmax != nullptr)
+        e = launch_nf4_quantize(merged, n, out->codes, nullptr, nullptr, nullptr, out->absmax, nullptr, sms, st);
+    else
+        e = launch_nf4_quantize(merged, n, out->codes, out->qscale, out->scale2, out->scale_mean, absmax, tile_sums,
+                                sms, st);
     if (e != cudaSuccess) return fail(NF4_ERR_CUDA, "nf4_merge_requantize launch: %s", cudaGetErrorString(e));
     return ok();
 }

@@ -228,9 +228,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_few_fwd(const __grid_constant__
     const uint32_t magic = G.nbc > 1 ? 0xFFFFFFFFu / static_cast<uint32_t>(G.nbc) + 1u : 0u;
     const int g0s = (G.row0 * bpr + G.kb0) >> 8;
     const int g1s = ((G.row0 + G.rows - 1) * bpr + G.kb1 - 1) >> 8;
+    // fp32 block scales (no double quantisation): staged as floats after the
+    // CTA barrier, and no second-level steps
+    const bool fp32_scales = a.absmax != nullptr;
     int8_t v[kStageLoads];
     float a2 = 0.0f;
-    if (stager) {
+    if (stager && !fp32_scales) {
         if (sidx <= g1s - g0s) a2 = __ldcg(a.scale2 + g0s + sidx);
 #pragma unroll
         for (int u = 0; u < kStageLoads; ++u) {
@@ -242,7 +245,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_few_fwd(const __grid_constant__
             }
         }
     }
-    const float mu = __ldcg(a.scale_mean);
+    const float mu = fp32_scales ? 0.0f : __ldcg(a.scale_mean);
     __syncthreads();
     if (p.cs > 1) cluster_arrive_relaxed();  // barriers initialised; the peer may address this CTA after its wait
     volatile int* abort_flag = &s_abort;
@@ -270,6 +273,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_few_fwd(const __grid_constant__
                 bulk_load(s_t2, a.ext_act, t2b, &bar_lora);
             s_lora = 1;
         }
+    } else if (fp32_scales) {
+        float* s_qf = reinterpret_cast<float*>(s_q);
+        for (int e = sidx; e < nq_el; e += nst) {
+            const int lr = G.nbc > 1 ? static_cast<int>(__umulhi(static_cast<uint32_t>(e), magic)) : e;
+            const int qi = lr * p.qrow + (e - lr * G.nbc);
+            if (NF4_CHECK(4 * (qi + 1) <= p.q_bytes, 14))
+                s_qf[qi] = __ldcg(a.absmax + (G.row0 + lr) * bpr + G.kb0 + (e - lr * G.nbc));
+        }
+        mbar_arrive(&bar_staged);
     } else {
         // store the first round; later rounds (large row counts only) load and
         // store in turn
@@ -350,10 +362,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_few_fwd(const __grid_constant__
                         const int bi = (G.row0 + lr) * bpr + G.kb0 + bl;
                         const int qi = lr * p.qrow + bl;
                         const int si = (bi >> 8) - g0;
-                        if (NF4_CHECK(qi < p.q_bytes, 3) && NF4_CHECK(si >= 0 && 4 * (si + 1) <= p.step_bytes, 4))
+                        if (fp32_scales) {
+                            if (NF4_CHECK(4 * (qi + 1) <= p.q_bytes, 3))
+                                sc = lds_f32(sq_s + 4 * static_cast<uint32_t>(qi));
+                        } else if (NF4_CHECK(qi < p.q_bytes, 3) &&
+                                   NF4_CHECK(si >= 0 && 4 * (si + 1) <= p.step_bytes, 4)) {
                             sc = __fadd_rn(__fmul_rn(static_cast<float>(lds_s8(sq_s + qi)),
                                                      lds_f32(sstep_s + 4 * static_cast<uint32_t>(si))),
                                            mu);
+                        }
                     }
                     nf4_table(sc, PT[o], HT[o]);
                     const uint32_t crow = st_s + lr * 128;
@@ -595,7 +612,7 @@ bool configure(int dev) {
 
 // Host plan: cluster size, octets per CTA, quad slots per pair group, ring
 // depth and the shared-memory layout (see the kernel's comment).
-bool few_fwd_plan(int M, int N, int K, int r, int num_sms, FewFwdPlan* out) {
+bool few_fwd_plan(int M, int N, int K, int r, int num_sms, bool fp32_scales, FewFwdPlan* out) {
     if (M < 1 || M > kTok || N % 8 != 0 || K % 64 != 0 || r < 1 || r > 256) return false;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || !configure(dev)) return false;
@@ -622,7 +639,7 @@ bool few_fwd_plan(int M, int N, int K, int r, int num_sms, FewFwdPlan* out) {
     p.xbox_bytes = p.xbox_rows * 128;
     p.slot = (p.code_bytes + kXStage + 1023) / 1024 * 1024;
     p.qrow = nbc;
-    p.q_bytes = (8 * p.O * p.qrow + 15) / 16 * 16;
+    p.q_bytes = (8 * p.O * p.qrow * (fp32_scales ? 4 : 1) + 15) / 16 * 16;
     const int64_t ngroups = (int64_t(8) * p.O * nb) / 256 + 2;
     p.step_bytes = static_cast<int>((ngroups * 4 + 15) / 16 * 16);
     p.t2_bytes = M * 4 * r64;

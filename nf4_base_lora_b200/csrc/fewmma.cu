@@ -166,7 +166,8 @@ __global__ void __maxnreg__(112) k_few_dx(const __grid_constant__ CUtensorMap ma
             for (int e = 0; e < 4; ++e) acc[m][h][e] = 0.0f;
     __syncthreads();
     cluster_arrive_relaxed();  // barriers initialised (made visible by the init fence)
-    const float mu = __ldcg(a.scale_mean);
+    const bool fp32_scales = a.absmax != nullptr;  // no double quantisation
+    const float mu = fp32_scales ? 0.0f : __ldcg(a.scale_mean);
     volatile int* abort_flag = &s_abort;
     uint8_t* my_tile = s_tiles + warp * kDxTileBytes;
     const uint32_t my_tile_u32 = smem_u32(my_tile);
@@ -200,8 +201,8 @@ __global__ void __maxnreg__(112) k_few_dx(const __grid_constant__ CUtensorMap ma
             const int c = sc0 + rw + 8 * it, n = 32 * c + lane;
             const bool ok = c < sc1 && n < N && blk_ok;
             const int64_t bi = static_cast<int64_t>(n) * bpr + blk;
-            qv[it] = ok ? static_cast<int>(__ldcg(a.qscale + bi)) : 0;
-            a2v[it] = ok ? __ldcg(a.scale2 + (bi >> 8)) : 0.0f;
+            qv[it] = ok && !fp32_scales ? static_cast<int>(__ldcg(a.qscale + bi)) : 0;
+            a2v[it] = ok ? __ldcg(fp32_scales ? a.absmax + bi : a.scale2 + (bi >> 8)) : 0.0f;
         }
 #pragma unroll
         for (int p = 0; p < 8; ++p) {
@@ -217,7 +218,8 @@ __global__ void __maxnreg__(112) k_few_dx(const __grid_constant__ CUtensorMap ma
             if (!mbar_wait(&bar_c[(c - sc0) / 8], seg_i & 1, abort_flag)) break;
             const int n = 32 * c + lane;
             const bool ok = n < N && blk_ok;
-            const float sc = ok ? nf4_block_scale(static_cast<int8_t>(qv[it]), a2v[it], mu) : 0.0f;
+            const float sc =
+                ok ? (fp32_scales ? a2v[it] : nf4_block_scale(static_cast<int8_t>(qv[it]), a2v[it], mu)) : 0.0f;
             // the row's 32 code bytes of block cb: 16-byte chunks 2 cb, 2 cb + 1, swizzled by row
             const uint8_t* crow = s_codes + lr * 64;
             const int sw = (lr >> 1) & 3;

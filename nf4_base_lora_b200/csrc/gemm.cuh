@@ -67,6 +67,7 @@ struct GemmArgs {
     const int8_t* qscale;
     const float* scale2;
     const float* scale_mean;
+    const float* absmax;      // fp32 block scales, or NULL (double-quantised scales above)
     int64_t w_rows;           // d_out of the encoded weight
     int64_t w_blocks_per_row; // d_in / 64
     // epilogue
@@ -426,7 +427,9 @@ __global__ void __launch_bounds__(GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI, 
             if (ew < C::kDecWarps) {
                 const int team = ew / C::kTeamWarps;
                 const int dt = threadIdx.x - 64 - team * C::kTeamThreads;
-                const float mu = __ldg(args.scale_mean);
+                // fp32 block scales (no double quantisation) when absmax is set
+                const bool fp32_scales = args.absmax != nullptr;
+                const float mu = fp32_scales ? 0.0f : __ldg(args.scale_mean);
                 constexpr bool kMNdec = C::kDecA ? (ASRC == SRC_DEC_MN) : (BSRC == SRC_DEC_MN);
                 constexpr int kCB = C::kDecMN / 64;           // 64-blocks across the decoded tile
                 const int tile_mn0 = C::kDecA ? r0 : c0;
@@ -475,8 +478,13 @@ __global__ void __launch_bounds__(GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI, 
                     ok_pf[slot] = it < n_main && wrow < args.w_rows && wblk < args.w_blocks_per_row;
                     if (ok_pf[slot]) {
                         const int64_t bidx = wrow * args.w_blocks_per_row + wblk;
-                        q_pf[slot] = __ldg(args.qscale + bidx);
-                        a2_pf[slot] = __ldg(args.scale2 + (bidx >> 8));
+                        if (fp32_scales) {
+                            q_pf[slot] = 0;
+                            a2_pf[slot] = __ldg(args.absmax + bidx);
+                        } else {
+                            q_pf[slot] = __ldg(args.qscale + bidx);
+                            a2_pf[slot] = __ldg(args.scale2 + (bidx >> 8));
+                        }
                     }
                 };
 #pragma unroll
@@ -488,7 +496,8 @@ __global__ void __launch_bounds__(GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI, 
                         const int it = base_it + u * kStride;
                         if (it >= n_main) break;
                         const bool valid = ok_pf[u];
-                        const float sc = valid ? nf4_block_scale(q_pf[u], a2_pf[u], mu) : 0.0f;
+                        const float sc =
+                            valid ? (fp32_scales ? a2_pf[u] : nf4_block_scale(q_pf[u], a2_pf[u], mu)) : 0.0f;
                         fetch(it + kPf * kStride, u);
                         if (!mbar_wait(&bar_full[it % LS], (it / LS) & 1u, abort_flag) ||
                             (it >= DS && !mbar_wait(&bar_dempty[it % DS], ((it / DS) & 1u) ^ 1u, abort_flag))) {

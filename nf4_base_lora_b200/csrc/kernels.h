@@ -7,13 +7,17 @@
 
 namespace nf4lora {
 
+// Double quantisation: qscale, scale2, scale_mean and both workspaces set.
+// fp32 block scales: qscale, scale2, scale_mean and ws_tile_sums NULL, and
+// ws_absmax is the tensor's absmax array (the stored scales).
 cudaError_t launch_nf4_quantize(const float* W, int64_t n, uint8_t* codes, int8_t* qscale,
                                 float* scale2, float* scale_mean, float* ws_absmax,
                                 double* ws_tile_sums, int num_sms, cudaStream_t stream);
 
+// absmax NULL: double-quantised scales; else the fp32 block scales.
 cudaError_t launch_nf4_dequantize(const uint8_t* codes, const int8_t* qscale, const float* scale2,
-                                  const float* scale_mean, int64_t n, uint16_t* out, int num_sms,
-                                  cudaStream_t stream);
+                                  const float* scale_mean, const float* absmax, int64_t n, uint16_t* out,
+                                  int num_sms, cudaStream_t stream);
 
 // AdamW step of up to kAdamwMaxTensors adapter tensors per launch (fp32
 // master p, bf16 copy p16 or NULL, bf16 gradient g, fp32 moments m, v; n
@@ -38,7 +42,8 @@ cudaError_t launch_adamw(const AdamwBatch& b, const AdamwConsts& c, int num_sms,
 // W'[N, K] fp32 = fp32(W_hat + s B A) from an encoded weight and the adapter
 // (rank sum in fp64, ascending j).
 cudaError_t launch_merge_lora(const uint8_t* codes, const int8_t* qscale, const float* scale2,
-                              const float* scale_mean, const uint16_t* A, const uint16_t* B, int r, int64_t N,
+                              const float* scale_mean, const float* absmax, const uint16_t* A, const uint16_t* B,
+                              int r, int64_t N,
                               int64_t K, float s, float* out, cudaStream_t stream);
 
 // Few-token (M <= 16) rank-r intermediates as bf16 hi | lo pairs; each is a
@@ -57,6 +62,7 @@ struct FewArgs {
     const int8_t* qscale;      // [N K / 64]
     const float* scale2;       // [ceil(N K / 64 / 256)]
     const float* scale_mean;   // [1]
+    const float* absmax;       // [N K / 64] fp32 block scales, or NULL (double-quantised scales)
     int M, N, K;               // tokens, d_out, d_in
     const uint16_t* ext_act;   // T2 / V2 [M, 2 r64] (bf16 hi | lo)
     const uint16_t* ext_w;     // forward: B [N, r]; input grad: A [r, K]
@@ -81,7 +87,7 @@ struct FewFwdPlan {
     int qrow, q_bytes, step_bytes, t2_bytes, b_bytes, recv_bytes;
     int smem;        // dynamic shared memory
 };
-bool few_fwd_plan(int M, int N, int K, int r, int num_sms, FewFwdPlan* out);
+bool few_fwd_plan(int M, int N, int K, int r, int num_sms, bool fp32_scales, FewFwdPlan* out);
 // map_codes: the packed codes as bytes [N, K / 2], box {128 bytes, plan.box_rows
 // rows}, 128-byte swizzle; map_x: the activations as bf16 [M, K], box {64, 16},
 // 128-byte swizzle

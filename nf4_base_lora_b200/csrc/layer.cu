@@ -283,6 +283,7 @@ static FewArgs few_args(const LayerCtx& c, const uint16_t* act, int M, const uin
     a.qscale = c.qscale;
     a.scale2 = c.scale2;
     a.scale_mean = c.scale_mean;
+    a.absmax = c.absmax;
     a.M = M;
     a.N = static_cast<int>(c.d_out);
     a.K = static_cast<int>(c.d_in);
@@ -364,6 +365,7 @@ int layer_fwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, fl
     g.qscale = c.qscale;
     g.scale2 = c.scale2;
     g.scale_mean = c.scale_mean;
+    g.absmax = c.absmax;
     g.w_rows = c.d_out;
     g.w_blocks_per_row = c.d_in / 64;
     g.k_main = ceil_div(c.d_in, 64);
@@ -379,7 +381,7 @@ int layer_fwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, fl
         const FewArgs fa = few_args(c, X, static_cast<int>(M), T2, B, r, r64, Y);
         FewFwdPlan fp;
         if (!few_fwd_plan(static_cast<int>(M), static_cast<int>(c.d_out), static_cast<int>(c.d_in), r, c.num_sms,
-                          &fp))
+                          c.absmax != nullptr, &fp))
         {
             note(cudaErrorInvalidConfiguration);
             return -2;
@@ -463,6 +465,7 @@ int layer_bwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, fl
         g.qscale = c.qscale;
         g.scale2 = c.scale2;
         g.scale_mean = c.scale_mean;
+    g.absmax = c.absmax;
         g.w_rows = c.d_out;
         g.w_blocks_per_row = c.d_in / 64;
         g.k_main = ceil_div(c.d_out, 64);

@@ -16,6 +16,7 @@ struct LayerCtx {
     const int8_t* qscale;
     const float* scale2;
     const float* scale_mean;
+    const float* absmax;  // fp32 block scales, or NULL (the double-quantised scales above)
     int64_t d_out;
     int64_t d_in;
     int num_sms;

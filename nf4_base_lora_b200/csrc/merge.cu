@@ -39,6 +39,7 @@ __global__ void __launch_bounds__(256) k_merge_lora(const uint8_t* __restrict__ 
                                                    const int8_t* __restrict__ qscale,
                                                    const float* __restrict__ scale2,
                                                    const float* __restrict__ scale_mean,
+                                                   const float* __restrict__ absmax,
                                                    const uint16_t* __restrict__ A, const uint16_t* __restrict__ B,
                                                    int r, int64_t N, int64_t K, float s,
                                                    float* __restrict__ out) {
@@ -94,7 +95,7 @@ __global__ void __launch_bounds__(256) k_merge_lora(const uint8_t* __restrict__ 
     }
 
     // epilogue: W_hat of the tile's block in each row, then the merged value
-    const float mu = *scale_mean;
+    const float mu = absmax ? 0.0f : *scale_mean;
     const int64_t bpr = K / 64, blk = k0 / 64;
     const double sd = static_cast<double>(s);
 #pragma unroll
@@ -102,7 +103,7 @@ __global__ void __launch_bounds__(256) k_merge_lora(const uint8_t* __restrict__ 
         const int64_t n = n0 + rb + i;
         if (n >= N) break;
         const int64_t bi = n * bpr + blk;
-        const float sc = nf4_block_scale(qscale[bi], scale2[bi >> 8], mu);
+        const float sc = absmax ? absmax[bi] : nf4_block_scale(qscale[bi], scale2[bi >> 8], mu);
         // codes of elements k0 + cb, + 1 and k0 + 32 + cb, + 1 of row n: one byte
         // each, the even element in the high nibble
         const uint8_t* row = codes + (n * K + k0) / 2;
@@ -122,15 +123,15 @@ __global__ void __launch_bounds__(256) k_merge_lora(const uint8_t* __restrict__ 
 }  // namespace
 
 cudaError_t launch_merge_lora(const uint8_t* codes, const int8_t* qscale, const float* scale2,
-                              const float* scale_mean, const uint16_t* A, const uint16_t* B, int r, int64_t N,
-                              int64_t K, float s, float* out, cudaStream_t stream) {
+                              const float* scale_mean, const float* absmax, const uint16_t* A, const uint16_t* B,
+                              int r, int64_t N, int64_t K, float s, float* out, cudaStream_t stream) {
     if (N < 1 || K < 64 || K % 64 != 0 || r < 1) return cudaErrorInvalidValue;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(static_cast<unsigned>(K / kMergeCols), static_cast<unsigned>((N + kMergeRows - 1) / kMergeRows));
     cfg.blockDim = dim3(256);
     cfg.stream = stream;
     TraceScope trace("nf4_merge_lora", stream);
-    return cudaLaunchKernelEx(&cfg, k_merge_lora, codes, qscale, scale2, scale_mean, A, B, r, N, K, s, out);
+    return cudaLaunchKernelEx(&cfg, k_merge_lora, codes, qscale, scale2, scale_mean, absmax, A, B, r, N, K, s, out);
 }
 
 }  // namespace nf4lora

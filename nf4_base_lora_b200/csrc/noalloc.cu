@@ -45,20 +45,29 @@ extern "C" int nf4_quantize_noalloc(const float* W, int64_t d_out, int64_t d_in,
     if ((reinterpret_cast<uintptr_t>(W) & 15u) != 0) return NF4_ERR_MISALIGNED;
     const size_t packed = nf4_packed_bytes(d_out, d_in);
     if (packed == 0) return NF4_ERR_UNSUPPORTED_SHAPE;
-    if (out->d_out != d_out || out->d_in != d_in || !out->codes || !out->qscale || !out->scale2 ||
-        !out->scale_mean)
+    const bool fp32_scales = out->absmax != nullptr;  // no double quantisation: no scratch at all
+    if (out->d_out != d_out || out->d_in != d_in || !out->codes ||
+        (!fp32_scales && (!out->qscale || !out->scale2 || !out->scale_mean)))
         return NF4_ERR_INVALID_ARG;
-    if ((reinterpret_cast<uintptr_t>(out->codes) & 15u) || (reinterpret_cast<uintptr_t>(out->qscale) & 15u) ||
-        (reinterpret_cast<uintptr_t>(out->scale2) & 15u) || (reinterpret_cast<uintptr_t>(out->scale_mean) & 3u))
+    if ((reinterpret_cast<uintptr_t>(out->codes) & 15u) ||
+        (fp32_scales && (reinterpret_cast<uintptr_t>(out->absmax) & 15u)) ||
+        (!fp32_scales &&
+         ((reinterpret_cast<uintptr_t>(out->qscale) & 15u) || (reinterpret_cast<uintptr_t>(out->scale2) & 15u) ||
+          (reinterpret_cast<uintptr_t>(out->scale_mean) & 3u))))
         return NF4_ERR_MISALIGNED;
     const int64_t n = d_out * d_in, n_blocks = n / 64;
-    if (n_blocks > kNoallocMaxBlocks) return NF4_ERR_UNSUPPORTED_SHAPE;  // beyond the fixed scratch
+    if (!fp32_scales && n_blocks > kNoallocMaxBlocks) return NF4_ERR_UNSUPPORTED_SHAPE;  // beyond the fixed scratch
     int dev = 0, major = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return NF4_ERR_CUDA;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return NF4_ERR_CUDA;
     if (major != 10) return NF4_ERR_DEVICE;
+    if (fp32_scales) {
+        const cudaError_t e = launch_nf4_quantize(W, n, out->codes, nullptr, nullptr, nullptr, out->absmax, nullptr,
+                                                  sms, static_cast<cudaStream_t>(stream));
+        return e == cudaSuccess ? NF4_OK : NF4_ERR_CUDA;
+    }
     void* scratch = nullptr;
     if (scratch_address(&scratch) != cudaSuccess) return NF4_ERR_CUDA;
     unsigned char* base = static_cast<unsigned char*>(scratch);

@@ -1,5 +1,9 @@
 // NF4 + double-quantisation encoder and the materialising decoder.
 //
+// Without double quantisation ("第 04 篇" §5.1: one fp32 scale per block of
+// 64, 0.5 bit per weight) only k_nf4_encode runs, writing the fp32 absmax of
+// every block as the stored scale.
+//
 // Encoding of one fp32 weight ("第 04 篇：QLoRA 原理" §3.4, §4.3, §5.2; the
 // compassingai.com QLoRA page, "NF4 量化機制詳解"), three launches:
 //   k_nf4_encode   per 64-block: absmax (half-warp shuffle reduction), IEEE
@@ -155,14 +159,18 @@ __global__ void __launch_bounds__(256, 3) k_nf4_encode(const float* __restrict__
         __syncthreads();
         // fp64 pairwise tree over the tile's 256 scales (zero-padded: x + 0 == x
         // keeps the carried-up elements of a short tail unchanged): five levels
-        // inside each warp's aligned run of 32, three over the eight warp sums
-        double t = pairwise_warp(s_sum[tid]);
-        __syncthreads();  // every s_sum read before warp 0's lanes reuse it
-        if (lane == 0) s_sum[warp] = t;
-        __syncthreads();
-        if (warp == 0) {
-            t = pairwise_warp(lane < 8 ? s_sum[lane] : 0.0);
-            if (lane == 0) tile_sums[tile] = t;
+        // inside each warp's aligned run of 32, three over the eight warp sums.
+        // Without double quantisation (tile_sums NULL, the same for the whole
+        // grid) there is no mean to form.
+        if (tile_sums != nullptr) {
+            double t = pairwise_warp(s_sum[tid]);
+            __syncthreads();  // every s_sum read before warp 0's lanes reuse it
+            if (lane == 0) s_sum[warp] = t;
+            __syncthreads();
+            if (warp == 0) {
+                t = pairwise_warp(lane < 8 ? s_sum[lane] : 0.0);
+                if (lane == 0) tile_sums[tile] = t;
+            }
         }
         __syncthreads();
     }
@@ -263,21 +271,23 @@ __global__ void __launch_bounds__(256) k_dq_quantize(const float* __restrict__ a
 }
 
 // Materialising decoder: each thread decodes 16 weights (8 code bytes) of one
-// block; w_hat = bf16_rne(level[code] * s_b).
+// block; w_hat = bf16_rne(level[code] * s_b), with s_b restored from the
+// double-quantised scales or, when absmax is given, the block's fp32 absmax.
 __global__ void __launch_bounds__(256) k_nf4_dequantize(const uint8_t* __restrict__ codes,
                                                        const int8_t* __restrict__ qscale,
                                                        const float* __restrict__ scale2,
                                                        const float* __restrict__ mean_ptr,
+                                                       const float* __restrict__ absmax,
                                                        int64_t n, uint16_t* __restrict__ out) {
     __shared__ float s_lut[16];
     if (threadIdx.x < 16) s_lut[threadIdx.x] = nf4_level(threadIdx.x);
     __syncthreads();
-    const float mu = *mean_ptr;
+    const float mu = absmax ? 0.0f : *mean_ptr;
     const int64_t n_units = n / 16;
     for (int64_t u = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; u < n_units;
          u += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const int64_t b = u >> 2;  // 4 units per 64-block
-        const float s = nf4_block_scale(qscale[b], scale2[b >> 8], mu);
+        const float s = absmax ? absmax[b] : nf4_block_scale(qscale[b], scale2[b >> 8], mu);
         const uint2 c = __ldcs(reinterpret_cast<const uint2*>(codes) + u);
         uint32_t o[8];
 #pragma unroll
@@ -328,6 +338,7 @@ cudaError_t launch_nf4_quantize(const float* W, int64_t n, uint8_t* codes, int8_
         e = cudaLaunchKernelEx(&cfg, k_nf4_encode, W, n_blocks, codes, ws_absmax, ws_tile_sums);
         if (e != cudaSuccess) return e;
     }
+    if (qscale == nullptr) return e;  // fp32 block scales: ws_absmax is the output
     {
         TraceScope trace("dq_mean", stream);
         cudaLaunchConfig_t cfg = config(1, 1024, stream);
@@ -349,14 +360,14 @@ cudaError_t launch_nf4_quantize(const float* W, int64_t n, uint8_t* codes, int8_
 }
 
 cudaError_t launch_nf4_dequantize(const uint8_t* codes, const int8_t* qscale, const float* scale2,
-                                  const float* scale_mean, int64_t n, uint16_t* out, int num_sms,
-                                  cudaStream_t stream) {
+                                  const float* scale_mean, const float* absmax, int64_t n, uint16_t* out,
+                                  int num_sms, cudaStream_t stream) {
     const int64_t units = n / 16;
     int64_t grid = (units + 255) / 256;
     if (grid > int64_t(num_sms) * 16) grid = int64_t(num_sms) * 16;
     TraceScope trace("nf4_dequantize", stream);
     cudaLaunchConfig_t cfg = config(grid, 256, stream);
-    return cudaLaunchKernelEx(&cfg, k_nf4_dequantize, codes, qscale, scale2, scale_mean, n, out);
+    return cudaLaunchKernelEx(&cfg, k_nf4_dequantize, codes, qscale, scale2, scale_mean, absmax, n, out);
 }
 
 }  // namespace nf4lora

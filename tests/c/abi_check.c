@@ -33,6 +33,20 @@ int main(void) {
     CHECK(((uintptr_t)t.qscale & 255u) == 0 && ((uintptr_t)t.scale2 & 255u) == 0);
     CHECK(nf4_tensor_from_buffer(&t, (void*)base, bytes - 1, d_out, d_in) != NF4_OK);
 
+    CHECK(t.absmax == NULL); /* the double-quantised format */
+
+    /* fp32 block scales (no double quantisation): n/2 + 4 n/64 bytes, each part padded to 256 */
+    const size_t bytes_nodq = nf4_packed_bytes_nodq(d_out, d_in);
+    CHECK(bytes_nodq >= (size_t)(n / 2 + 4 * (n / 64)));
+    CHECK(bytes_nodq < (size_t)(n / 2 + 4 * (n / 64) + 2 * 256));
+    CHECK(nf4_packed_bytes_nodq(4096, 100) == 0);
+    nf4_tensor u;
+    memset(&u, 0xff, sizeof u);
+    CHECK(nf4_tensor_from_buffer_nodq(&u, (void*)base, bytes_nodq, d_out, d_in) == NF4_OK);
+    CHECK((uintptr_t)u.codes == base && u.qscale == NULL && u.scale2 == NULL && u.scale_mean == NULL);
+    CHECK((uintptr_t)u.absmax - base >= (uintptr_t)(n / 2) && ((uintptr_t)u.absmax & 255u) == 0);
+    CHECK(nf4_tensor_from_buffer_nodq(&u, (void*)base, bytes_nodq - 1, d_out, d_in) != NF4_OK);
+
     CHECK(nf4_quantize_workspace_bytes(d_out, d_in) > 0);
     CHECK(qlora_fwd_workspace_bytes(16, d_out, d_in, 64) > 0);
     CHECK(qlora_bwd_workspace_bytes(4096, d_out, d_in, 64) > qlora_bwd_workspace_bytes(16, d_out, d_in, 64));
@@ -47,6 +61,9 @@ int main(void) {
     CHECK(strlen(nf4lora_last_error_string()) > 0);
     CHECK(qlora_linear_fwd(&t, A, B, 64, 0.25f, NULL, 0, NULL, NULL, NULL, 0, NULL) == NF4_OK); /* empty batch */
     CHECK(nf4_merge_lora(&t, A, B, 0, 1.0f, (float*)Y, NULL) == NF4_ERR_INVALID_ARG);
+    CHECK(qlora_linear_fwd(&u, A, B, 64, 0.25f, NULL, 16, Y, NULL, NULL, 0, NULL) == NF4_ERR_INVALID_ARG);
+    u.codes = NULL;
+    CHECK(qlora_linear_fwd(&u, A, B, 64, 0.25f, Y, 16, Y, NULL, NULL, 0, NULL) == NF4_ERR_INVALID_ARG);
 
     lora_adamw_tensor at;
     memset(&at, 0, sizeof at);

@@ -49,3 +49,19 @@ def test_noalloc_rejects_sizes_beyond_its_scratch(nf):
     s = nf.Nf4TensorStruct(d_out, d_in, 1 << 20, 1 << 21, 1 << 22, 1 << 23)
     status = nf.lib.nf4_quantize_noalloc(ctypes.c_void_p(1 << 24), d_out, d_in, ctypes.byref(s), None)
     assert status == -2
+
+
+def test_noalloc_quantize_fp32_scales(nf):
+    """The fp32-block-scale format needs no scratch: the same bytes as
+    nf4_quantize into that format."""
+    d_out, d_in = 300, 448
+    W = torch.from_numpy(workloads.weight(d_out, d_in, outliers=True, index=1)).cuda()
+    ref = nf.nf4_quantize(W, double_quant=False)
+    got = nf.NF4Tensor(d_out, d_in, W.device, double_quant=False)
+    got.buffer.fill_(0xAB)
+    status = nf.lib.nf4_quantize_noalloc(ctypes.c_void_p(W.data_ptr()), d_out, d_in, ctypes.byref(got.struct),
+                                         ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert status == 0
+    torch.cuda.synchronize()
+    assert torch.equal(got.codes, ref.codes)
+    assert torch.equal(got.absmax.view(torch.int32), ref.absmax.view(torch.int32))
