@@ -205,8 +205,11 @@ int nf4_dequantize(const nf4_tensor* w, uint16_t* W_hat, void* stream);
  * arrays hi = bf16(T), lo = bf16(T - hi) (about 16 significant bits), so the
  * adapter branch is not limited to bfloat16 precision ([QP] §6.3: the adapter
  * dtype may be wider than the base compute dtype).
- * Requirements: 0 <= M < 2^31, 1 <= r <= 256, r % 8 == 0, d_in % 64 == 0,
+ * Requirements: 0 <= M < 2^31, 1 <= r <= 256, d_in % 64 == 0,
  * d_out % 8 == 0, ws >= qlora_fwd_workspace_bytes(M, d_out, d_in, r).
+ * A rank that is not a multiple of 8 runs as the next multiple of 8 on
+ * zero-padded copies of A, B and T that the workspace holds (three more
+ * small copy launches; the zero rows and columns contribute exact zeros).
  * M = 0 (an empty batch) does nothing and returns NF4_OK; X, Y and T_saved
  * may then be NULL.
  */

@@ -92,7 +92,6 @@ int check_layer_common(const nf4_tensor* w, const uint16_t* A, const uint16_t* B
     if (rc) return rc;
     if (w->d_out % 8 != 0) return fail(NF4_ERR_UNSUPPORTED_SHAPE, "d_out = %lld must be a multiple of 8", (long long)w->d_out);
     if (r < 1 || r > 256) return fail(NF4_ERR_INVALID_ARG, "r = %d outside [1, 256]", r);
-    if (r % 8 != 0) return fail(NF4_ERR_UNSUPPORTED_SHAPE, "r = %d must be a multiple of 8", r);
     if (!std::isfinite(scaling)) return fail(NF4_ERR_INVALID_ARG, "scaling is not finite");
     if (M < 0 || M >= (int64_t(1) << 31)) return fail(NF4_ERR_INVALID_ARG, "M = %lld outside [0, 2^31)", (long long)M);
     if (!A || !B) return fail(NF4_ERR_INVALID_ARG, "A or B is NULL");

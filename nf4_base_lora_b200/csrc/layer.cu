@@ -349,14 +349,17 @@ static int lora_down(const LayerCtx& c, const uint16_t* A, int r, float s, const
     return reduce(ra, c.num_sms, c.stream) == cudaSuccess ? 0 : -2;
 }
 
-int64_t fwd_workspace_bytes(int64_t M, int64_t d_out, int64_t d_in, int r, int num_sms) {
+static int64_t fwd_core_bytes(int64_t M, int64_t d_out, int64_t d_in, int r, int num_sms) {
+    (void)d_out;
     const int r64 = round64(r);
     const int64_t part = M <= kSmallM ? 0 : int64_t(split_down(M, d_in, num_sms).splits) * M * r64;
     return align256(M * r64 * 4) + align256(part * 4);
 }
 
-int layer_fwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, float s, const uint16_t* X,
-              int64_t M, uint16_t* Y, float* T_saved, uint8_t* ws) {
+// The layer for a rank that is a multiple of 8 (B's rows, r bf16, are then
+// whole 16-byte units, as the tensor maps and the vector loads need).
+static int layer_fwd_r8(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, float s,
+                        const uint16_t* X, int64_t M, uint16_t* Y, float* T_saved, uint8_t* ws) {
     const int r64 = round64(r), kx = r64 / 64;
     uint16_t* T2 = reinterpret_cast<uint16_t*>(ws);
     float* part = reinterpret_cast<float*>(ws + align256(M * r64 * 4));
@@ -415,7 +418,7 @@ int layer_fwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, fl
     return e == cudaSuccess ? 0 : -2;
 }
 
-int64_t bwd_workspace_bytes(int64_t M, int64_t d_out, int64_t d_in, int r, int num_sms) {
+static int64_t bwd_core_bytes(int64_t M, int64_t d_out, int64_t d_in, int r, int num_sms) {
     const int r64 = round64(r);
     int64_t part = int64_t(split_down(M, d_in, num_sms).splits) * M * r64;
     part = std::max<int64_t>(part, int64_t(split_v(M, d_out, num_sms).splits) * M * r64);
@@ -424,9 +427,9 @@ int64_t bwd_workspace_bytes(int64_t M, int64_t d_out, int64_t d_in, int r, int n
     return 2 * align256(M * r64 * 4) + align256(part * 4);
 }
 
-int layer_bwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, float s, const uint16_t* X,
-              const float* T_saved, const uint16_t* dY, int64_t M, uint16_t* dX, uint16_t* dA, uint16_t* dB,
-              int accumulate, uint8_t* ws) {
+static int layer_bwd_r8(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, float s,
+                        const uint16_t* X, const float* T_saved, const uint16_t* dY, int64_t M, uint16_t* dX,
+                        uint16_t* dA, uint16_t* dB, int accumulate, uint8_t* ws) {
     const int r64 = round64(r), kx = r64 / 64;
     uint16_t* V2 = reinterpret_cast<uint16_t*>(ws);
     uint16_t* T2 = reinterpret_cast<uint16_t*>(ws + align256(M * r64 * 4));
@@ -560,6 +563,121 @@ int layer_bwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, fl
         ra.accumulate = accumulate;
         if (reduce(ra, c.num_sms, c.stream) != cudaSuccess) return -2;
     }
+    return 0;
+}
+
+// ------------------------------------------------------------------ any rank
+// A rank that is not a multiple of 8 runs as the next multiple r8 on padded
+// copies in the workspace: A with zero rows r .. r8-1, B with zero columns,
+// T_saved with zero columns; dA and dB are produced padded and their first r
+// rows / columns copied out (copied in first when accumulating).  The zero
+// rows and columns add exact zeros to every product and sum, so the results
+// are those of rank r.
+
+// dst[i, j] (dst_rows x dst_cols, leading dimension ld_dst) = src[i, j] for
+// i < src_rows and j < src_cols, else 0.
+template <typename T>
+__global__ void k_repack(const T* __restrict__ src, int64_t src_rows, int src_cols, int64_t ld_src,
+                         T* __restrict__ dst, int64_t dst_rows, int dst_cols, int64_t ld_dst) {
+    const int64_t total = dst_rows * dst_cols;
+    for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
+         e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t i = e / dst_cols;
+        const int j = static_cast<int>(e - i * dst_cols);
+        dst[i * ld_dst + j] = (i < src_rows && j < src_cols) ? src[i * ld_src + j] : T(0);
+    }
+}
+
+template <typename T>
+static cudaError_t repack(const T* src, int64_t src_rows, int src_cols, int64_t ld_src, T* dst, int64_t dst_rows,
+                          int dst_cols, int64_t ld_dst, int num_sms, cudaStream_t st) {
+    const int64_t total = dst_rows * dst_cols;
+    if (total <= 0) return cudaSuccess;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(std::min<int64_t>((total + 255) / 256, int64_t(num_sms) * 8)));
+    cfg.blockDim = dim3(256);
+    cfg.stream = st;
+    TraceScope trace("repack_rank", st);
+    return note(cudaLaunchKernelEx(&cfg, k_repack<T>, src, src_rows, src_cols, ld_src, dst, dst_rows, dst_cols,
+                                   ld_dst));
+}
+
+static inline int round8(int r) { return (r + 7) / 8 * 8; }
+
+// Padded copies after the core workspace: A [r8, d_in], B [d_out, r8],
+// T [M, r8] (fp32), and for the backward dA [r8, d_in], dB [d_out, r8].
+struct RankPad {
+    uint16_t* A;
+    uint16_t* B;
+    float* T;
+    uint16_t* dA;
+    uint16_t* dB;
+    int64_t bytes;
+};
+
+static RankPad rank_pad(uint8_t* base, int64_t M, int64_t d_out, int64_t d_in, int r, bool backward) {
+    RankPad p{};
+    if (r % 8 == 0) return p;
+    const int r8 = round8(r);
+    int64_t off = 0;
+    auto take = [&](int64_t bytes) {
+        uint8_t* q = base ? base + off : nullptr;
+        off += align256(bytes);
+        return q;
+    };
+    p.A = reinterpret_cast<uint16_t*>(take(int64_t(r8) * d_in * 2));
+    p.B = reinterpret_cast<uint16_t*>(take(d_out * r8 * 2));
+    p.T = reinterpret_cast<float*>(take(M * r8 * 4));
+    if (backward) {
+        p.dA = reinterpret_cast<uint16_t*>(take(int64_t(r8) * d_in * 2));
+        p.dB = reinterpret_cast<uint16_t*>(take(d_out * r8 * 2));
+    }
+    p.bytes = off;
+    return p;
+}
+
+int64_t fwd_workspace_bytes(int64_t M, int64_t d_out, int64_t d_in, int r, int num_sms) {
+    return fwd_core_bytes(M, d_out, d_in, r, num_sms) + rank_pad(nullptr, M, d_out, d_in, r, false).bytes;
+}
+
+int64_t bwd_workspace_bytes(int64_t M, int64_t d_out, int64_t d_in, int r, int num_sms) {
+    return bwd_core_bytes(M, d_out, d_in, r, num_sms) + rank_pad(nullptr, M, d_out, d_in, r, true).bytes;
+}
+
+int layer_fwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, float s, const uint16_t* X,
+              int64_t M, uint16_t* Y, float* T_saved, uint8_t* ws) {
+    if (r % 8 == 0) return layer_fwd_r8(c, A, B, r, s, X, M, Y, T_saved, ws);
+    const int r8 = round8(r);
+    const RankPad p = rank_pad(ws + fwd_core_bytes(M, c.d_out, c.d_in, r, c.num_sms), M, c.d_out, c.d_in, r, false);
+    if (repack(A, r, static_cast<int>(c.d_in), c.d_in, p.A, r8, static_cast<int>(c.d_in), c.d_in, c.num_sms,
+               c.stream) != cudaSuccess ||
+        repack(B, c.d_out, r, r, p.B, c.d_out, r8, r8, c.num_sms, c.stream) != cudaSuccess)
+        return -2;
+    const int rc = layer_fwd_r8(c, p.A, p.B, r8, s, X, M, Y, T_saved ? p.T : nullptr, ws);
+    if (rc) return rc;
+    if (T_saved && repack<float>(p.T, M, r8, r8, T_saved, M, r, r, c.num_sms, c.stream) != cudaSuccess) return -2;
+    return 0;
+}
+
+int layer_bwd(const LayerCtx& c, const uint16_t* A, const uint16_t* B, int r, float s, const uint16_t* X,
+              const float* T_saved, const uint16_t* dY, int64_t M, uint16_t* dX, uint16_t* dA, uint16_t* dB,
+              int accumulate, uint8_t* ws) {
+    if (r % 8 == 0) return layer_bwd_r8(c, A, B, r, s, X, T_saved, dY, M, dX, dA, dB, accumulate, ws);
+    const int r8 = round8(r);
+    const int d_in = static_cast<int>(c.d_in);
+    const RankPad p = rank_pad(ws + bwd_core_bytes(M, c.d_out, c.d_in, r, c.num_sms), M, c.d_out, c.d_in, r, true);
+    if (repack(A, r, d_in, c.d_in, p.A, r8, d_in, c.d_in, c.num_sms, c.stream) != cudaSuccess ||
+        repack(B, c.d_out, r, r, p.B, c.d_out, r8, r8, c.num_sms, c.stream) != cudaSuccess ||
+        (T_saved && repack<float>(T_saved, M, r, r, p.T, M, r8, r8, c.num_sms, c.stream) != cudaSuccess) ||
+        (accumulate && dA && repack(dA, r, d_in, c.d_in, p.dA, r8, d_in, c.d_in, c.num_sms, c.stream) != cudaSuccess) ||
+        (accumulate && dB && repack(dB, c.d_out, r, r, p.dB, c.d_out, r8, r8, c.num_sms, c.stream) != cudaSuccess))
+        return -2;
+    const int rc = layer_bwd_r8(c, p.A, p.B, r8, s, X, T_saved ? p.T : nullptr, dY, M, dX, dA ? p.dA : nullptr,
+                                dB ? p.dB : nullptr, accumulate, ws);
+    if (rc) return rc;
+    if ((dA && repack(p.dA, r8, d_in, c.d_in, dA, r, d_in, c.d_in, c.num_sms, c.stream) != cudaSuccess) ||
+        (dB && repack(p.dB, c.d_out, r8, r8, dB, c.d_out, r, r, c.num_sms, c.stream) != cudaSuccess))
+        return -2;
     return 0;
 }
 

@@ -57,7 +57,11 @@ int main(void) {
     const uint16_t* B = (const uint16_t*)((uintptr_t)1 << 25);
     uint16_t* Y = (uint16_t*)((uintptr_t)1 << 27);
     CHECK(qlora_linear_fwd(&t, A, B, 64, 0.25f, NULL, 16, Y, NULL, NULL, 0, NULL) == NF4_ERR_INVALID_ARG);
-    CHECK(qlora_linear_fwd(&t, A, B, 12, 0.25f, Y, 16, Y, NULL, NULL, 0, NULL) == NF4_ERR_UNSUPPORTED_SHAPE);
+    CHECK(qlora_linear_fwd(&t, A, B, 0, 0.25f, Y, 16, Y, NULL, NULL, 0, NULL) == NF4_ERR_INVALID_ARG);   /* r < 1 */
+    CHECK(qlora_linear_fwd(&t, A, B, 257, 0.25f, Y, 16, Y, NULL, NULL, 0, NULL) == NF4_ERR_INVALID_ARG); /* r > 256 */
+    /* any rank in [1, 256]: r = 12 passes the argument checks and needs a workspace */
+    CHECK(qlora_linear_fwd(&t, A, B, 12, 0.25f, Y, 16, Y, NULL, NULL, 0, NULL) == NF4_ERR_WORKSPACE);
+    CHECK(qlora_fwd_workspace_bytes(16, d_out, d_in, 12) > qlora_fwd_workspace_bytes(16, d_out, d_in, 16));
     CHECK(strlen(nf4lora_last_error_string()) > 0);
     CHECK(qlora_linear_fwd(&t, A, B, 64, 0.25f, NULL, 0, NULL, NULL, NULL, 0, NULL) == NF4_OK); /* empty batch */
     CHECK(nf4_merge_lora(&t, A, B, 0, 1.0f, (float*)Y, NULL) == NF4_ERR_INVALID_ARG);

@@ -83,10 +83,12 @@ def test_host_validation_without_device(nf):
     f = ctypes.c_float(2.0)
     # NULL X
     assert L.qlora_linear_fwd(ctypes.byref(s), A, B, 8, f, None, 16, Y, None, ws, 1 << 30, None) == -1
-    # r not a multiple of 8
-    assert L.qlora_linear_fwd(ctypes.byref(s), A, B, 12, f, X, 16, Y, None, ws, 1 << 30, None) == -2
+    # any rank in [1, 256] passes the host checks (r = 12 runs padded to 16): here, without a
+    # device, the call then stops at the device check
+    assert L.qlora_linear_fwd(ctypes.byref(s), A, B, 12, f, X, 16, Y, None, ws, 1 << 30, None) == -5
     # r out of range
     assert L.qlora_linear_fwd(ctypes.byref(s), A, B, 0, f, X, 16, Y, None, ws, 1 << 30, None) == -1
+    assert L.qlora_linear_fwd(ctypes.byref(s), A, B, 257, f, X, 16, Y, None, ws, 1 << 30, None) == -1
     # misaligned X
     assert L.qlora_linear_fwd(ctypes.byref(s), A, B, 8, f, P((1 << 26) + 2), 16, Y, None, ws, 1 << 30, None) == -3
     # workspace too small / NULL

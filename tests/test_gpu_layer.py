@@ -47,6 +47,11 @@ CASES = [
     (11008, 4096, 16, 64),    # few tokens, 19 weight octets per cluster: the stage ring is refilled
     (4096, 11008, 3, 64),     # few tokens, 22 block quads per CTA: the stage ring is refilled
     (256, 16384, 5, 16),      # few tokens, one octet per cluster: a ring of 24 stages, deeper than the 16 warps
+    (256, 512, 4, 1),         # ranks that are not multiples of 8 (padded internally): few tokens
+    (384, 320, 16, 5),
+    (264, 320, 130, 12),      # and many tokens
+    (512, 768, 300, 5),
+    (384, 256, 40, 251),
 ]
 
 
@@ -111,6 +116,24 @@ def test_accumulate_and_skipped_outputs(nf):
     assert torch.equal(only_dx, dX)
     assert_close(dA2, 2 * dA.float(), "dA accumulated")
     assert_close(dB2, 2 * dB.float(), "dB accumulated")
+
+
+@pytest.mark.parametrize("m,r", [(7, 5), (200, 12)])
+def test_accumulate_with_a_rank_off_the_multiple_of_8(nf, m, r):
+    """dA and dB are accumulated through their padded copies: 2x the single
+    gradient, and T from the forward is the oracle's."""
+    c, W_hat, w, dev = setup(nf, 256, 320, m, r)
+    _, T = nf.qlora_linear_fwd(w, dev["A"], dev["B"], c.scaling, dev["X"])
+    dX, dA, dB = nf.qlora_linear_bwd(w, dev["A"], dev["B"], c.scaling, dev["X"], T, dev["dY"])
+    _, dA2, dB2 = nf.qlora_linear_bwd(w, dev["A"], dev["B"], c.scaling, dev["X"], None, dev["dY"],
+                                      need_dx=False, dA=dA.clone(), dB=dB.clone(), accumulate=True)
+    torch.cuda.synchronize()
+    nf.device_status()
+    _, T_ref = oracle.forward(W_hat, c.A, c.B, c.X, c.scaling)
+    assert_close(T, T_ref, "T", max_rel=1e-5, mean_rel=1e-6, round_ref=False)
+    _, dA_ref, dB_ref = oracle.backward(W_hat, c.A, c.B, c.X, c.dY, c.scaling)
+    assert_close(dA2, 2 * dA_ref, "dA accumulated")
+    assert_close(dB2, 2 * dB_ref, "dB accumulated")
 
 
 def test_layer_is_deterministic(nf):
