@@ -97,6 +97,16 @@ def step_plan(wl):
     return plan
 
 
+def exchange_points(plan):
+    """{pass index: module index} of the pass after which a module's adapter
+    gradients are final for the step (its last full backward pass)."""
+    last = {}
+    for p, (i, _, _, kind) in enumerate(plan):
+        if kind == "full":
+            last[i] = p
+    return {p: i for i, p in last.items()}
+
+
 def step_totals(wl):
     b = f = 0.0
     for _, mod, m, kind in step_plan(wl):
@@ -410,29 +420,36 @@ class GpuWorkload:
         self.plan = step_plan(wl)
         self.sms = torch.cuda.get_device_properties(device).multi_processor_count
 
-    def step(self, copy_base, X=None, dY=None, outs=None):
-        """Enqueue one step; pass p uses encoded copy (copy_base + p)."""
+    def step(self, copy_base, X=None, dY=None, outs=None, after_pass=None):
+        """Enqueue one step; pass p uses encoded copy (copy_base + p);
+        after_pass(p), if given, runs after each pass is enqueued."""
+        for p in range(len(self.plan)):
+            self.step_pass(copy_base, p, X, dY, outs)
+            if after_pass is not None:
+                after_pass(p)
+
+    def step_pass(self, copy_base, p, X=None, dY=None, outs=None):
         nf, wl = self.nf, self.wl
-        for p, (i, mod, m, kind) in enumerate(self.plan):
-            d = self.mods[i]
-            enc = d["encs"][(copy_base + p) % len(d["encs"])]
-            x = (X[i] if X is not None else d["X"])[:m]
-            if kind == "fwd":
-                # a full backward follows: the forward keeps T = s X A^T (fp32) for it,
-                # as a training step does; a dX-only backward needs no T
-                keep = wl.backward != "dx"
-                nf.qlora_linear_fwd(enc, d["A"], d["B"], wl.scaling, x, save_t=keep,
-                                    Y=(outs[i]["Y"][m] if outs else d["Y"][m]), workspace=self.ws,
-                                    T=d["T"][m])
+        i, mod, m, kind = self.plan[p]
+        d = self.mods[i]
+        enc = d["encs"][(copy_base + p) % len(d["encs"])]
+        x = (X[i] if X is not None else d["X"])[:m]
+        if kind == "fwd":
+            # a full backward follows: the forward keeps T = s X A^T (fp32) for it,
+            # as a training step does; a dX-only backward needs no T
+            keep = wl.backward != "dx"
+            nf.qlora_linear_fwd(enc, d["A"], d["B"], wl.scaling, x, save_t=keep,
+                                Y=(outs[i]["Y"][m] if outs else d["Y"][m]), workspace=self.ws,
+                                T=d["T"][m])
+        else:
+            dy = (dY[i] if dY is not None else d["dY"])[:m]
+            if kind == "dx":
+                nf.qlora_linear_bwd(enc, d["A"], d["B"], wl.scaling, None, None, dy, need_da=False,
+                                    need_db=False, dX=(outs[i]["dX"][m] if outs else d["dX"][m]),
+                                    workspace=self.ws)
             else:
-                dy = (dY[i] if dY is not None else d["dY"])[:m]
-                if kind == "dx":
-                    nf.qlora_linear_bwd(enc, d["A"], d["B"], wl.scaling, None, None, dy, need_da=False,
-                                        need_db=False, dX=(outs[i]["dX"][m] if outs else d["dX"][m]),
-                                        workspace=self.ws)
-                else:
-                    nf.qlora_linear_bwd(enc, d["A"], d["B"], wl.scaling, x, d["T"][m], dy, dA=d["dA"], dB=d["dB"],
-                                        dX=(outs[i]["dX"][m] if outs else d["dX"][m]), workspace=self.ws)
+                nf.qlora_linear_bwd(enc, d["A"], d["B"], wl.scaling, x, d["T"][m], dy, dA=d["dA"], dB=d["dB"],
+                                    dX=(outs[i]["dX"][m] if outs else d["dX"][m]), workspace=self.ws)
 
 
 def dominant_kernel_stats(records, names):
@@ -647,16 +664,23 @@ def time_workload(nf, wl, args, stream, device, world, peaks, l2, with_e2e):
     cycle = max(1, copies // len(plan)) if copies > 1 else 1
     step_bytes, step_flops = step_totals(wl)
 
-    # data-parallel exchange of the adapter gradients (full backward, N > 1)
+    # data-parallel exchange of the adapter gradients (full backward, N > 1):
+    # module i's dA, dB are all-reduced on a side stream as soon as its last
+    # backward pass of the step is enqueued, overlapping the later passes
     exchange = None
-    if world > 1 and wl.backward != "dx":
+    if (world > 1 or getattr(args, "force_exchange", False)) and wl.backward != "dx":
         from nf4_base_lora_b200 import dp
-        exchange = dp.LoraGradExchange([t for d in gw.mods for t in (d["dA"], d["dB"])])
+        exchange = dp.OverlappedGradExchange([[d["dA"], d["dB"]] for d in gw.mods])
+    exchange_after = exchange_points(plan)
+
+    def after_pass(p):
+        if exchange is not None and p in exchange_after:
+            exchange.launch(exchange_after[p])
 
     def enqueue(s_index, **kw):
-        gw.step((s_index % cycle) * len(plan), **kw)
+        gw.step((s_index % cycle) * len(plan), after_pass=after_pass, **kw)
         if exchange is not None:
-            exchange()
+            exchange.finish()
 
     # eager warm-up step, traced only to count the library's launches per step
     nf.trace_start(len(plan) * 16 + 64)
@@ -666,21 +690,35 @@ def time_workload(nf, wl, args, stream, device, world, peaks, l2, with_e2e):
     launches_per_step = nf.trace_count()
     nf.trace_stop()
 
+    # one graph per step, or with an exchange one per pass (the collectives
+    # run eagerly on their side stream between the replays)
     graphs = []
     if not args.no_graph:
         for g in range(cycle):
-            graph = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(graph, stream=stream):
-                gw.step(g * len(plan))
-            graphs.append(graph)
+            if exchange is None:
+                graph = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(graph, stream=stream):
+                    gw.step(g * len(plan))
+                graphs.append([graph])
+            else:
+                per_pass = []
+                for p in range(len(plan)):
+                    graph = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(graph, stream=stream):
+                        gw.step_pass(g * len(plan), p)
+                    per_pass.append(graph)
+                graphs.append(per_pass)
 
     def run_steps(k, base):
         with torch.cuda.stream(stream):
             for i in range(k):
                 if graphs:
-                    graphs[(base + i) % cycle].replay()
+                    for p, graph in enumerate(graphs[(base + i) % cycle]):
+                        graph.replay()
+                        if exchange is not None:
+                            after_pass(p)
                     if exchange is not None:
-                        exchange()
+                        exchange.finish()
                 else:
                     enqueue(base + i)
 
@@ -764,14 +802,13 @@ def time_workload(nf, wl, args, stream, device, world, peaks, l2, with_e2e):
         ms_per_step * 1e-3) / 1e9
 
     if with_e2e:
-        out["e2e"] = time_e2e(gw, wl, args, stream, device, world, cycle, plan, exchange, step_bytes, step_flops)
-    for g in graphs:
-        del g
+        out["e2e"] = time_e2e(gw, wl, args, stream, device, world, cycle, plan, exchange, after_pass, step_bytes,
+                              step_flops)
     graphs.clear()
     return out, gw
 
 
-def time_e2e(gw, wl, args, stream, device, world, cycle, plan, exchange, step_bytes, step_flops):
+def time_e2e(gw, wl, args, stream, device, world, cycle, plan, exchange, after_pass, step_bytes, step_flops):
     """The same step end to end through the public API: pinned host inputs
     copied to the device, the layer calls, the outputs copied back, every
     step inside the timed region."""
@@ -795,9 +832,9 @@ def time_e2e(gw, wl, args, stream, device, world, cycle, plan, exchange, step_by
             for i in range(len(gw.mods)):
                 devX[i].copy_(hostX[i], non_blocking=True)
                 devdY[i].copy_(hostdY[i], non_blocking=True)
-            gw.step((s % cycle) * len(plan), X=devX, dY=devdY, outs=outs)
+            gw.step((s % cycle) * len(plan), X=devX, dY=devdY, outs=outs, after_pass=after_pass)
             if exchange is not None:
-                exchange()
+                exchange.finish()
             for i in range(len(gw.mods)):
                 for m in wl.tokens:
                     hostY[i][m].copy_(outs[i]["Y"][m], non_blocking=True)
@@ -834,8 +871,17 @@ def run_ours(args, wl):
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
-    if world > 1:
+    if world > 1 or getattr(args, "force_exchange", False):
         import datetime
+        if world == 1:
+            # a group of one rank, so that --force-exchange runs the collective path
+            import socket
+            with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as sk:
+                sk.bind(("127.0.0.1", 0))
+                os.environ.setdefault("MASTER_PORT", str(sk.getsockname()[1]))
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            os.environ.setdefault("RANK", "0")
+            os.environ.setdefault("WORLD_SIZE", "1")
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
 
     import nf4_base_lora_b200 as nf
@@ -854,7 +900,7 @@ def run_ours(args, wl):
             with torch.cuda.stream(stream):
                 gw.step(0)  # the backward fills dA, dB
             obj = time_adamw(nf, gw, args, stream, device, world, peaks, l2)
-        if world > 1:
+        if dist.is_initialized():
             dist.barrier()
             dist.destroy_process_group()
         if rank == 0:
@@ -884,7 +930,7 @@ def run_ours(args, wl):
         cb = time_oracle(wl, budget_s=args.cpu_budget)
         cpu_baseline = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
 
-    if world > 1:
+    if dist.is_initialized():
         dist.barrier()
         dist.destroy_process_group()
     if rank != 0:
@@ -918,6 +964,8 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="llama65b_layer_r64_m2048", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--force-exchange", action="store_true",
+                    help="run the data-parallel gradient exchange even on one rank (a process group of one)")
     ap.add_argument("--no-few", action="store_true", help="skip the few-token sub-object")
     ap.add_argument("--no-merge", action="store_true", help="skip the merge + re-encoding phase")
     ap.add_argument("--no-cpu-baseline", action="store_true")

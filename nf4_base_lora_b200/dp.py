@@ -74,6 +74,52 @@ class LoraGradExchange:
             g.reshape(-1).copy_(self.flat[off:off + g.numel()])
 
 
+class OverlappedGradExchange:
+    """The exchange split per module and overlapped with the rest of the
+    backward ("第 04 篇：QLoRA 原理" §10.4: one full quantised base per
+    data-parallel process; only the adapter gradients cross ranks).
+
+    `buckets[i]` lists module i's gradients (its dA and dB).  As soon as the
+    backward of module i has produced them on the current stream,
+    ``launch(i)`` records an event there and, on a side stream that waits for
+    that event, packs them, SUM-all-reduces them and writes them back, while
+    the current stream goes on with the next module.  ``finish()`` makes the
+    current stream wait for every exchange launched so far: call it before
+    anything reads or overwrites the gradients again (the optimizer step, the
+    next step's backward).  On CPU tensors (gloo) there are no streams and
+    ``launch`` exchanges at once.  Each bucket is reduced in fp32 and each
+    bf16 gradient rounded once, as in LoraGradExchange."""
+
+    def __init__(self, buckets: Sequence[Sequence[torch.Tensor]], group: Optional[dist.ProcessGroup] = None,
+                 stream: Optional["torch.cuda.Stream"] = None):
+        if not buckets:
+            raise ValueError("no gradient buckets")
+        self.buckets = [LoraGradExchange(b, group) for b in buckets]
+        dev = self.buckets[0].flat.device
+        if any(b.flat.device != dev for b in self.buckets):
+            raise ValueError("all buckets must be on one device")
+        self.cuda = dev.type == "cuda"
+        self.stream = (stream if stream is not None else torch.cuda.Stream(device=dev)) if self.cuda else None
+        self.launched = 0
+
+    def launch(self, i: int, average: bool = False) -> None:
+        bucket = self.buckets[i]
+        if not self.cuda:
+            bucket(average)
+            return
+        ready = torch.cuda.Event()
+        ready.record(torch.cuda.current_stream(self.stream.device))
+        with torch.cuda.stream(self.stream):
+            self.stream.wait_event(ready)  # module i's gradients are complete
+            bucket(average)
+        self.launched += 1
+
+    def finish(self) -> None:
+        if self.cuda and self.launched:
+            torch.cuda.current_stream(self.stream.device).wait_stream(self.stream)
+            self.launched = 0
+
+
 def max_over_ranks(value: float, device: torch.device, group: Optional[dist.ProcessGroup] = None) -> float:
     """The largest `value` of all ranks (a step time: the slowest rank sets
     the pace of a synchronous data-parallel step)."""

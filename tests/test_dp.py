@@ -115,3 +115,41 @@ def test_exchange_rejects_bad_inputs():
         dp.LoraGradExchange([torch.zeros(4, dtype=torch.float16)])
     with pytest.raises(ValueError):
         dp.LoraGradExchange([torch.zeros(4, 4).t()])
+
+
+def _overlap_worker(rank, world, port):
+    """Per-module buckets exchanged one by one (on CPU the exchange runs at
+    launch): the same sums as one exchange of everything, on every rank."""
+    from nf4_base_lora_b200 import dp
+    _init(rank, world, port)
+    try:
+        c = workloads.linear_case(128, 192, 23, 8, alpha=16.0)
+        b, e = dp.token_shard(23, world, rank)
+        grads = []
+        for i in range(3):                       # three modules, scaled copies of one case
+            dA_s, dB_s = oracle.lora_grads(c.A, c.B, c.X[b:e], c.dY[b:e], c.scaling * (i + 1))
+            grads.append([torch.from_numpy(dA_s).to(torch.bfloat16).contiguous(),
+                          torch.from_numpy(dB_s).to(torch.bfloat16).contiguous()])
+        whole = [t.clone() for g in grads for t in g]
+        dp.LoraGradExchange(whole)()
+        ex = dp.OverlappedGradExchange(grads)
+        assert not ex.cuda and len(ex.buckets) == 3
+        for i in reversed(range(3)):             # the backward visits the modules last to first
+            ex.launch(i)
+        ex.finish()
+        for got, ref in zip([t for g in grads for t in g], whole):
+            assert torch.equal(got, ref)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_overlapped_exchange_matches_single_exchange():
+    mp.spawn(_overlap_worker, args=(WORLD, _free_port()), nprocs=WORLD, join=True)
+
+
+def test_overlapped_exchange_rejects_bad_inputs():
+    from nf4_base_lora_b200 import dp
+    with pytest.raises(ValueError):
+        dp.OverlappedGradExchange([])
+    with pytest.raises(ValueError):
+        dp.OverlappedGradExchange([[torch.zeros(4, dtype=torch.float16)]])
