@@ -164,7 +164,7 @@ int nf4_quantize(const float* W, int64_t d_out, int64_t d_in, const nf4_tensor* 
  * The scratch the encoder needs (the fp32 absmax of every block and the fp64
  * tree partial sums) lives in a fixed array inside the library, sized for
  * at most 4,194,304 blocks of 64 weights (d_out * d_in <= 268,435,456); that
- * array (16 MiB + 128 KiB) stays resident on every GPU that loads the library
+ * array (17 MiB) stays resident on every GPU that loads the library
  * until the process exits.  Larger weights return NF4_ERR_UNSUPPORTED_SHAPE.
  * The call allocates nothing; the caller still passes W and `out`.  An
  * `out` in the fp32-block-scale format (out->absmax != NULL) needs no scratch

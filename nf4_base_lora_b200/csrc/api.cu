@@ -83,7 +83,9 @@ int check_tensor(const nf4_tensor* w) {
 int64_t quant_ws_bytes(int64_t d_out, int64_t d_in) {
     const int64_t nb = d_out * d_in / 64;
     const int64_t tiles = (nb + 255) / 256;
-    return align256(nb * 4) + align256(tiles * 8);
+    const int64_t segs = (tiles + 2047) / 2048;
+    // absmax; 8 fp64 warp sums per tile, the fp64 segment sums and a ticket
+    return align256(nb * 4) + align256(tiles * 8 * 8 + segs * 8 + 8);
 }
 
 int check_layer_common(const nf4_tensor* w, const uint16_t* A, const uint16_t* B, int r, float scaling,

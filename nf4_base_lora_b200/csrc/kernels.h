@@ -8,11 +8,13 @@
 namespace nf4lora {
 
 // Double quantisation: qscale, scale2, scale_mean and both workspaces set.
-// fp32 block scales: qscale, scale2, scale_mean and ws_tile_sums NULL, and
+// ws_warp_sums holds 8 fp64 values per tile of 256 blocks, then one per
+// segment of 2048 tiles and a 4-byte ticket.
+// fp32 block scales: qscale, scale2, scale_mean and ws_warp_sums NULL, and
 // ws_absmax is the tensor's absmax array (the stored scales).
 cudaError_t launch_nf4_quantize(const float* W, int64_t n, uint8_t* codes, int8_t* qscale,
                                 float* scale2, float* scale_mean, float* ws_absmax,
-                                double* ws_tile_sums, int num_sms, cudaStream_t stream);
+                                double* ws_warp_sums, int num_sms, cudaStream_t stream);
 
 // absmax NULL: double-quantised scales; else the fp32 block scales.
 cudaError_t launch_nf4_dequantize(const uint8_t* codes, const int8_t* qscale, const float* scale2,

@@ -2,7 +2,7 @@
 // compiled into the library, for callers that cannot allocate device memory.
 //
 // Scratch of the encoder: the fp32 first-level absmax of every 64-block and
-// one fp64 partial sum per 256 blocks.  Here it lives in g_quant_scratch, a
+// eight fp64 partial sums per 256 blocks.  Here it lives in g_quant_scratch, a
 // file-scope __device__ array sized for kNoallocMaxBlocks blocks, which every
 // GPU that loads the library keeps until the process exits.  Host code must
 // not pass the symbol itself to a kernel (on the host it names a stand-in, not
@@ -24,7 +24,7 @@ namespace {
 constexpr int64_t kNoallocMaxBlocks = int64_t(1) << 22;                 // 268,435,456 weights
 constexpr int64_t kNoallocMaxTiles = kNoallocMaxBlocks / 256;
 constexpr int64_t kAbsmaxBytes = kNoallocMaxBlocks * 4;                  // 16 MiB
-constexpr int64_t kScratchBytes = kAbsmaxBytes + kNoallocMaxTiles * 8;   // + 128 KiB
+constexpr int64_t kScratchBytes = kAbsmaxBytes + kNoallocMaxTiles * 64 + 256;  // + 1 MiB of warp sums, segment sums
 
 static __device__ __align__(256) unsigned char g_quant_scratch[kScratchBytes];
 
