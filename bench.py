@@ -469,6 +469,37 @@ def quantize_bytes(d_out, d_in):
     return 4 * n + n // 2 + nb + 4 * ((nb + 255) // 256) + 4
 
 
+def time_forward(nf, gw, args, stream, device, world):
+    """The forward passes of the step plan on their own, eager: W warm-up
+    passes, then K passes timed together (a short command whose kernels are
+    the step's forwards, to profile)."""
+    fwd = [p for p, (_, _, _, kind) in enumerate(gw.plan) if kind == "fwd"]
+
+    def one_pass():
+        with torch.cuda.stream(stream):
+            for p in fwd:
+                gw.step_pass(0, p)
+
+    for _ in range(args.warmup):
+        one_pass()
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    stop = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(args.steps):
+        one_pass()
+    stop.record(stream)
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(stop)
+    if world > 1:
+        from nf4_base_lora_b200 import dp
+        ms = dp.max_over_ranks(ms, device)
+    flops = sum(pass_flops(mod.d_out, mod.d_in, m, gw.wl.r, "fwd") for _, mod, m, kind in gw.plan if kind == "fwd")
+    ms_pass = ms / args.steps
+    return {"ms_per_pass": ms_pass, "passes": args.steps, "launches_per_pass": len(fwd),
+            "value": world * flops / (ms_pass * 1e-3) / 1e12, "unit": "TFLOP/s"}
+
+
 def time_quantize(nf, gw, args, stream, device, world, peaks):
     """Encoding of every module's fp32 weight through nf4_quantize, timed on
     its own: K passes over all modules after W warm-up passes (the fp32
@@ -894,6 +925,8 @@ def run_ours(args, wl):
         gw = GpuWorkload(nf, wl, device, 1, keep_fp32=args.only == "quantize")
         if args.only == "quantize":
             obj = time_quantize(nf, gw, args, stream, device, world, peaks)
+        elif args.only == "forward":
+            obj = time_forward(nf, gw, args, stream, device, world)
         elif args.only == "merge":
             obj = time_merge(nf, gw, args, stream, device, world)
         else:
@@ -970,8 +1003,9 @@ def main():
     ap.add_argument("--no-merge", action="store_true", help="skip the merge + re-encoding phase")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
-    ap.add_argument("--only", choices=("quantize", "merge", "optimizer"),
-                    help="time one phase of the workload alone (encoding, merge + re-encoding, optimizer step)")
+    ap.add_argument("--only", choices=("quantize", "merge", "optimizer", "forward"),
+                    help="time one phase of the workload alone (encoding, merge + re-encoding, optimizer step, "
+                         "the forward passes)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
