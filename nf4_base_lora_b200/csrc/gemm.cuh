@@ -63,6 +63,7 @@ struct GemmArgs {
     int k_ext;          // extension k-steps (grid.z slice 0 only)
     int ext_wrap_a;     // extension k-step j reads A_ext at (j % ext_wrap_a) when > 0
     int ext_wrap_b;     // ... and B_ext at (j % ext_wrap_b) when > 0
+    int cols_fastest;   // 1: grid.x walks the column tiles and grid.y the row tiles (else the reverse)
     // NF4 operand
     const int8_t* qscale;
     const float* scale2;
@@ -245,8 +246,11 @@ __global__ void __launch_bounds__(GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI, 
     auto b_buf = [&](int it) { return C::kDecB ? dec_slot(it) : load_slot(it) + C::kLoadA; };
     auto codes_buf = [&](int it) { return load_slot(it) + (C::kDecA ? 0 : C::kLoadA); };
 
-    const int r0 = blockIdx.x * C::kRows;
-    const int c0 = blockIdx.y * BN;
+    // consecutive CTAs share their B operand (row tiles fastest) or their A
+    // operand (column tiles fastest): the one they share is read from DRAM
+    // about once, the other once per wave of CTAs
+    const int r0 = (args.cols_fastest ? blockIdx.y : blockIdx.x) * C::kRows;
+    const int c0 = (args.cols_fastest ? blockIdx.x : blockIdx.y) * BN;
     const int z = blockIdx.z;
     int kb_begin, kb_end;
     if constexpr (EPI == EPI_CLUSTER_BF16_T) {

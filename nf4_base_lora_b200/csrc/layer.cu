@@ -255,6 +255,16 @@ static inline int round64(int r) { return (r + 63) / 64 * 64; }
 static inline int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
 static int bn_for(int cols) { return cols <= 64 ? 64 : (cols <= 128 ? 128 : 256); }
 
+// Bytes of an encoded weight (codes, int8 scales, group scales), close enough
+// to choose a tile order.
+static inline int64_t weight_bytes_approx(int64_t d_out, int64_t d_in) { return d_out * d_in * 33 / 64; }
+
+// The grid of a fused GEMM: row tiles x column tiles, the column tiles along
+// grid.x when g.cols_fastest is set.
+static inline dim3 tile_grid(int row_tiles, int col_tiles, const GemmArgs& g) {
+    return g.cols_fastest ? dim3(col_tiles, row_tiles, 1) : dim3(row_tiles, col_tiles, 1);
+}
+
 static constexpr int kSmallM = 16;
 
 // Many-token fused GEMMs: 256-row CTA tiles (two accumulators sharing each
@@ -406,14 +416,18 @@ static int layer_fwd_r8(const LayerCtx& c, const uint16_t* A, const uint16_t* B,
     g.k_per_split = g.k_main;
     g.out = Y;
     g.ldo = c.d_out;
+    // re-read the smaller operand once per wave: X (2 M K bytes) or the codes
+    // (about 0.52 N K bytes)
+    g.cols_fastest = 2 * M * c.d_in > weight_bytes_approx(c.d_out, c.d_in) ? 1 : 0;
     cudaError_t e;
     if (wide_tiles(M, c.d_out, c.num_sms)) {
-        dim3 grid(ceil_div(M, 256), ceil_div(c.d_out, 256), 1);
         e = launch<256, SRC_TMA_K, SRC_DEC_K, 0, 0, EPI_BF16, kWideLoad, kWideDec, kWideTeams, 2>(
-            "nf4_gemm_fwd", m.a, m.b, m.ae, m.be, g, grid, c.stream);
+            "nf4_gemm_fwd", m.a, m.b, m.ae, m.be, g, tile_grid(ceil_div(M, 256), ceil_div(c.d_out, 256), g),
+            c.stream);
     } else {
-        dim3 grid(ceil_div(M, 128), ceil_div(c.d_out, 256), 1);
-        e = launch<256, SRC_TMA_K, SRC_DEC_K, 0, 0, EPI_BF16>("nf4_gemm_fwd", m.a, m.b, m.ae, m.be, g, grid, c.stream);
+        e = launch<256, SRC_TMA_K, SRC_DEC_K, 0, 0, EPI_BF16>("nf4_gemm_fwd", m.a, m.b, m.ae, m.be, g,
+                                                             tile_grid(ceil_div(M, 128), ceil_div(c.d_out, 256), g),
+                                                             c.stream);
     }
     return e == cudaSuccess ? 0 : -2;
 }
@@ -490,15 +504,18 @@ static int layer_bwd_r8(const LayerCtx& c, const uint16_t* A, const uint16_t* B,
             g.k_per_split = g.k_main;
             g.out = dX;
             g.ldo = c.d_in;
+            // re-read the smaller operand once per wave: dY (2 M N bytes) or the
+            // codes (about 0.52 N K bytes)
+            g.cols_fastest = 2 * M * c.d_out > weight_bytes_approx(c.d_out, c.d_in) ? 1 : 0;
             cudaError_t e;
             if (wide_tiles(M, c.d_in, c.num_sms)) {
-                dim3 grid(ceil_div(M, 256), ceil_div(c.d_in, 256), 1);
                 e = launch<256, SRC_TMA_K, SRC_DEC_MN, 0, 1, EPI_BF16, kWideLoad, kWideDec, kWideTeams, 2>(
-                    "nf4_gemm_dx", m.a, m.b, m.ae, m.be, g, grid, c.stream);
+                    "nf4_gemm_dx", m.a, m.b, m.ae, m.be, g, tile_grid(ceil_div(M, 256), ceil_div(c.d_in, 256), g),
+                    c.stream);
             } else {
-                dim3 grid(ceil_div(M, 128), ceil_div(c.d_in, 256), 1);
-                e = launch<256, SRC_TMA_K, SRC_DEC_MN, 0, 1, EPI_BF16>("nf4_gemm_dx", m.a, m.b, m.ae, m.be, g, grid,
-                                                                       c.stream);
+                e = launch<256, SRC_TMA_K, SRC_DEC_MN, 0, 1, EPI_BF16>(
+                    "nf4_gemm_dx", m.a, m.b, m.ae, m.be, g, tile_grid(ceil_div(M, 128), ceil_div(c.d_in, 256), g),
+                    c.stream);
             }
             if (e != cudaSuccess) return -2;
         }
