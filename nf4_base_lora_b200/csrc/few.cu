@@ -54,8 +54,9 @@ __device__ __forceinline__ void store_split(uint16_t* dst_hi, uint16_t* dst_lo, 
 // memory with asynchronous copies issued all at once, after the wait for the
 // preceding kernel (the rows of A were asked into L2 before it), and the
 // dependent launch is released right after that wait.  The CTAs are small (four warps, 37 KB of
-// shared memory) and many (one per SM for r = 64), so that the loads are
-// spread over SMs and the CTAs share SMs with the dependent kernel's.  Warp w
+// shared memory) and many, so that the loads are spread over SMs (the
+// dependent forward's CTAs hold an SM's whole register file, so they start on
+// an SM once these have left it).  Warp w
 // takes every fourth 16-wide chunk; partials are added in a fixed order: the
 // four warps in shared memory, then the cluster ranks by rank 0 reading the
 // others' shared memory.

@@ -15,35 +15,40 @@
 //   halves of whole block quads (4 x 64 weights).  74 clusters of two fill
 //   the 148 SMs of a B200, and octet granularity keeps them within one octet
 //   of even (4096 rows: 7 octets per cluster).
-// * Streaming.  Thread 0 puts the CTA's quads in flight at once through a
-//   ring of stages, each stage one quad (where the ring is shorter than the
-//   CTA's quads, the last warp to finish with a stage refills it): the packed
-//   codes of all O
-//   octets and the quad's 256 activation columns of the 16 token rows (four
-//   boxes of 64 columns), all by TMA with the 128-byte swizzle, completing on
-//   the stage's barrier.  The
-//   block-scale codes and the second-level steps a2 / 127 of the CTA's rows are
-//   staged once in shared memory before the first stage lands.
+// * Streaming.  The CTA's quads go through a ring of stages, each stage one
+//   quad: the packed codes of all O octets and the quad's four 64-column
+//   activation boxes of the token rows, all by TMA with the 128-byte swizzle,
+//   completing on the stage's barrier (rows beyond M and blocks beyond K read
+//   as zeros).  Thread 0 initialises the barriers and issues the first two
+//   stages before the CTA barrier; after it, lane 0 of warp w issues stages
+//   w, w + 16, ... of the rest that fit the ring, so every stage that fits
+//   is in flight from the start; where the ring is shorter than the CTA's
+//   quads, the last warp to finish with a stage refills it.  Lanes 1 .. 31 of
+//   every warp stage the block-scale codes and the second-level steps
+//   a2 / 127 of the CTA's rows once in shared memory (or the fp32 block
+//   scales of the format without double quantisation).
 // * Decode.  Each lane holds the 16 scaled levels of one (row, block) as byte
 //   planes in registers (csrc/decode.cuh) and turns four codes into two
-//   bf16 pairs with eight byte permutes; the pairs are the B operand of the
+//   bf16 pairs with eight byte permutes; the pairs are the A operand of the
 //   warp-level tensor instruction (mma.sync m16n8k16, bf16 in, fp32
-//   accumulate) whose A operand is 16 tokens of activations.  Lane (g, q) of a
-//   warp covers row g of an octet and block q of a quad; the 16-wide
-//   contraction of each MMA takes four consecutive columns of every lane's
-//   block, so one scale serves a lane for a whole block.  Lane q walks its
-//   block starting 2q words in (its code words are loaded rotated), which puts
-//   the 16-byte activation loads of a quarter warp (two tokens, four blocks)
-//   on eight different bank groups of the swizzled boxes; the rotated 8-byte
-//   code loads of a half warp are conflict-free too.
+//   accumulate: 16 weight rows, the rows g and g + 8 of an octet pair, by 16
+//   columns) whose B operand is eight tokens of activations.  Lane (g, q) of
+//   a warp covers rows g and g + 8 of a pair and block q of a quad; the
+//   16-wide contraction of each MMA takes four consecutive columns of every
+//   lane's block, so one scale serves a lane for a whole block.  Lane q walks
+//   its block's words in the order j ^ 2q (its code words are loaded in that
+//   order), which puts the 16-byte activation loads of a quarter warp (two
+//   tokens, four blocks) on eight different bank groups of the swizzled
+//   boxes; the 8-byte code loads of a half warp are conflict-free too.
 // * Reduction.  Warps of one pair group add their partials in shared memory
 //   in a fixed order; the two CTAs of a cluster then each finish half the
 //   octets: the other half's partials go to the peer through distributed
 //   shared memory, and the owner adds the two and writes bf16 rows.  The
 //   rank-r term is computed by the owner for its octets once the kernel
-//   producing T2 has finished (programmatic dependent launch; warp 0 stages
-//   T2 and the owner's rows of B after its first stage).  The summation
-//   order is fixed, so the result is the same on every run.
+//   producing T2 has finished (programmatic dependent launch; lane 0 of the
+//   last warp that issues a first stage also copies the owner's rows of B,
+//   then waits for that kernel and copies T2).  The summation order is
+//   fixed, so the result is the same on every run.
 //
 // Launch overlap: the kernel releases its own dependents as soon as it starts,
 // and reads the activations, the encoded weight and B before its wait: the
