@@ -170,6 +170,14 @@ __global__ void __launch_bounds__(256, 3) k_nf4_encode(const float* __restrict__
         const int it = static_cast<int>(u & 3);
         const int64_t b = b0 + grp;
         const bool valid = b < n_blocks;
+        {
+            // ask L2 for the same unit of this CTA's next tile (four units
+            // ahead): lane l < 16 one 128-byte line of it, so the loads that
+            // follow there find their lines in L2
+            const int64_t pb = b0 + tile_step + (lane >> 1);
+            if (lane < 16 && pb < n_blocks)
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(W + pb * 64 + (lane & 1) * 32));
+        }
         float v[16];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
