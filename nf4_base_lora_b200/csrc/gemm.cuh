@@ -80,8 +80,13 @@ struct GemmArgs {
     int64_t ldp;        // EPI_F32_PART_T: part[z * part_slice + col * ldp + row]
     int64_t part_slice;
     // 1: the kernel runs as a programmatic dependent of the previous kernel on
-    // the stream, which produces the extension operand.
+    // the stream, which produces the extension operand (the producer waits
+    // for it before the extension steps only; the main operands come from
+    // kernels that completed before that one started).
     int pdl;
+    // 1: a programmatic dependent that waits for the previous kernel before
+    // anything else (it reads or overwrites what that kernel may still use).
+    int wait_first;
 };
 
 template <int SRC>
@@ -277,6 +282,12 @@ __global__ void __launch_bounds__(GemmConfig<BN, ASRC, BSRC, AE_MN, BE_MN, EPI, 
     const int n_main = kb_end > kb_begin ? kb_end - kb_begin : 0;
     const int n_ext = (z == 0) ? args.k_ext : 0;
     const int n_iter = n_main + n_ext;
+
+    // the next kernel on the stream may be scheduled once every CTA of this
+    // grid has started (it waits for this grid's completion before it reads
+    // anything this grid writes)
+    if (args.wait_first) grid_dependency_wait();
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < LS; ++i) {

@@ -119,7 +119,7 @@ static cudaError_t launch(const char* name, const CUtensorMap& a, const CUtensor
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
     int n_attr = 0;
-    if (args.pdl) {
+    if (args.pdl || args.wait_first) {
         // may start while the previous kernel on the stream still runs; the
         // kernel waits for it (griddepcontrol.wait) where it needs its output
         attr[n_attr].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -160,10 +160,13 @@ struct ReduceArgs {
     int accumulate;
     float* out32;
     int64_t ldo32;
+    int pdl;  // launched as a programmatic dependent: waits for the previous kernel first
     int out32_cols;
 };
 
 __global__ void k_reduce_splits(const ReduceArgs a) {
+    if (a.pdl) asm volatile("griddepcontrol.wait;" ::: "memory");  // the partials are complete
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int64_t total = static_cast<int64_t>(a.rows) * a.cols;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -199,6 +202,13 @@ static cudaError_t reduce(const ReduceArgs& a, int num_sms, cudaStream_t st) {
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
     cfg.blockDim = dim3(256);
     cfg.stream = st;
+    cudaLaunchAttribute attr{};
+    if (a.pdl) {
+        attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr.val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = &attr;
+        cfg.numAttrs = 1;
+    }
     TraceScope trace("reduce_splits", st);
     return note(cudaLaunchKernelEx(&cfg, k_reduce_splits, a));
 }
@@ -206,6 +216,7 @@ static cudaError_t reduce(const ReduceArgs& a, int num_sms, cudaStream_t st) {
 static ReduceArgs reduce_args(const float* part, int splits, int64_t slice, int rows, int cols, int64_t ldp,
                               float alpha, uint16_t* out, int64_t ldo) {
     ReduceArgs a{};
+    a.pdl = 1;  // it follows the split-K GEMM that wrote the partials
     a.part = part;
     a.splits = splits;
     a.slice = slice;
@@ -342,6 +353,7 @@ static int lora_down(const LayerCtx& c, const uint16_t* A, int r, float s, const
     if (!map_bf16(&m.a, X, c.d_in, M, c.d_in, 128) || !map_bf16(&m.b, A, c.d_in, r, c.d_in, bn)) return -1;
     const Split sp = split_down(M, c.d_in, c.num_sms);
     GemmArgs g{};
+    g.wait_first = 1;  // it overwrites the split-K partials the kernels before it used
     g.rows = static_cast<int>(M);
     g.cols = r64;
     g.k_main = ceil_div(c.d_in, 64);
@@ -411,6 +423,7 @@ static int layer_fwd_r8(const LayerCtx& c, const uint16_t* A, const uint16_t* B,
         !map_bf16(&m.ae, T2, 2 * r64, M, 2 * r64, 128) || !map_bf16(&m.be, B, r, c.d_out, r, 256))
         return -1;
     g.ext_wrap_b = kx;
+    g.pdl = 1;  // T (hi | lo) comes from the reduction just launched
     g.rows = static_cast<int>(M);
     g.cols = static_cast<int>(c.d_out);
     g.k_per_split = g.k_main;
@@ -461,6 +474,7 @@ static int layer_bwd_r8(const LayerCtx& c, const uint16_t* A, const uint16_t* B,
         if (!map_bf16(&m.a, dY, c.d_out, M, c.d_out, 128) || !map_bf16(&m.b, B, r, c.d_out, r, 64)) return -1;
         const Split sp = split_v(M, c.d_out, c.num_sms);
         GemmArgs g{};
+        g.wait_first = 1;
         g.rows = static_cast<int>(M);
         g.cols = r64;
         g.k_main = ceil_div(c.d_out, 64);
@@ -499,6 +513,7 @@ static int layer_bwd_r8(const LayerCtx& c, const uint16_t* A, const uint16_t* B,
                 !map_bf16(&m.ae, V2, 2 * r64, M, 2 * r64, 128) || !map_bf16(&m.be, A, c.d_in, r, c.d_in, 64))
                 return -1;
             g.ext_wrap_b = kx;
+            g.pdl = 1;  // V (hi | lo) comes from the reduction just launched
             g.rows = static_cast<int>(M);
             g.cols = static_cast<int>(c.d_in);
             g.k_per_split = g.k_main;
@@ -543,6 +558,7 @@ static int layer_bwd_r8(const LayerCtx& c, const uint16_t* A, const uint16_t* B,
         if (!map_bf16(&m.a, dY, c.d_out, M, c.d_out, 64) || !map_bf16(&m.b, T2, 2 * r64, M, 2 * r64, 64)) return -1;
         const Split sp = split_tokens(c.d_out, r64, M, c.num_sms);
         GemmArgs g{};
+        g.wait_first = 1;
         g.rows = static_cast<int>(c.d_out);
         g.cols = 2 * r64;
         g.k_main = ceil_div(M, 64);
@@ -564,6 +580,7 @@ static int layer_bwd_r8(const LayerCtx& c, const uint16_t* A, const uint16_t* B,
         if (!map_bf16(&m.a, X, c.d_in, M, c.d_in, 64) || !map_bf16(&m.b, V2, 2 * r64, M, 2 * r64, 64)) return -1;
         const Split sp = split_tokens(c.d_in, r64, M, c.num_sms);
         GemmArgs g{};
+        g.wait_first = 1;
         g.rows = static_cast<int>(c.d_in);
         g.cols = 2 * r64;
         g.k_main = ceil_div(M, 64);
