@@ -16,7 +16,11 @@
 // factor slices of 16 ranks at a time are staged in shared memory as fp64
 // (B transposed), and each thread keeps 8 rows x 4 columns of fp64 sums; the
 // epilogue decodes the tile's codes (one 64-block per row) and writes fp32
-// rows.
+// rows.  The bf16 rows of the next slice travel by 16-byte asynchronous
+// copies into a staging buffer while the current slice is multiplied, so the
+// fp64 pipe does not wait for global loads between slices (B's rows are
+// copied this way when r is a multiple of 8, which makes every row of B start
+// on 16 bytes; otherwise B is read element by element at each slice).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -35,16 +39,26 @@ constexpr int kMergeRows = 128;  // rows n per CTA
 constexpr int kMergeCols = 64;   // columns k per CTA: one 64-block of each row
 constexpr int kMergeRanks = 16;  // ranks j per staged slice
 
-__global__ void __launch_bounds__(256) k_merge_lora(const uint8_t* __restrict__ codes,
-                                                   const int8_t* __restrict__ qscale,
-                                                   const float* __restrict__ scale2,
-                                                   const float* __restrict__ scale_mean,
-                                                   const float* __restrict__ absmax,
-                                                   const uint16_t* __restrict__ A, const uint16_t* __restrict__ B,
-                                                   int r, int64_t N, int64_t K, float s,
-                                                   float* __restrict__ out) {
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// VEC_B: r is a multiple of 8, so the 8-rank pieces of B's rows start on 16 bytes.
+template <bool VEC_B>
+__global__ void __launch_bounds__(256, 2) k_merge_lora(const uint8_t* __restrict__ codes,
+                                                      const int8_t* __restrict__ qscale,
+                                                      const float* __restrict__ scale2,
+                                                      const float* __restrict__ scale_mean,
+                                                      const float* __restrict__ absmax,
+                                                      const uint16_t* __restrict__ A, const uint16_t* __restrict__ B,
+                                                      int r, int64_t N, int64_t K, float s,
+                                                      float* __restrict__ out) {
     __shared__ __align__(16) double sA[kMergeRanks][kMergeCols];  // A[j0 + jj][k0 + c]
     __shared__ __align__(16) double sB[kMergeRanks][kMergeRows];  // B[n0 + rr][j0 + jj], transposed
+    __shared__ __align__(16) uint16_t stA[kMergeRanks][kMergeCols];  // bf16 staging of the next slice of A
+    __shared__ __align__(16) uint16_t stB[kMergeRows][kMergeRanks];  // and of B (VEC_B only), row-major
     __shared__ float s_lvl[16];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid < 16) s_lvl[tid] = nf4_level(tid);
@@ -55,6 +69,21 @@ __global__ void __launch_bounds__(256) k_merge_lora(const uint8_t* __restrict__ 
     // this thread's columns: 2 tx, 2 tx + 1 and 32 + 2 tx, 33 + 2 tx, so that the
     // 16-byte reads of eight consecutive lanes cover 128 contiguous bytes
     const int cb = 2 * tx;
+    // staging roles: threads 0..127 copy one 16-byte piece of A (rank row
+    // tid / 8, columns 8 (tid % 8) ..), every thread one 8-rank piece of B
+    // (row tid % 128, ranks 8 (tid / 128) ..)
+    const int a_jj = tid >> 3, a_c = 8 * (tid & 7);
+    const int b_rr = tid & 127, b_h = tid >> 7;
+
+    // copies of the slice that starts at rank j0 into the staging buffers;
+    // rank rows at or past r, and rows of B at or past N, are not copied (the
+    // conversion below writes zeros for them)
+    auto stage = [&](int j0) {
+        if (tid < 128 && j0 + a_jj < r) cp_async16(&stA[a_jj][a_c], A + static_cast<int64_t>(j0 + a_jj) * K + k0 + a_c);
+        if (VEC_B && n0 + b_rr < N && j0 + 8 * b_h < r)
+            cp_async16(&stB[b_rr][8 * b_h], B + (n0 + b_rr) * r + j0 + 8 * b_h);
+        cp_async_commit();
+    };
 
     double acc[8][4];
 #pragma unroll
@@ -62,20 +91,43 @@ __global__ void __launch_bounds__(256) k_merge_lora(const uint8_t* __restrict__ 
 #pragma unroll
         for (int c = 0; c < 4; ++c) acc[i][c] = 0.0;
 
+    stage(0);
     for (int j0 = 0; j0 < r; j0 += kMergeRanks) {
         const int nj = min(kMergeRanks, r - j0);
-        __syncthreads();  // the previous slice is no longer read
-        for (int i = tid; i < kMergeRanks * kMergeCols; i += 256) {
-            const int jj = i / kMergeCols, c = i % kMergeCols;
-            sA[jj][c] = jj < nj ? static_cast<double>(bf16_bits_to_float(A[static_cast<int64_t>(j0 + jj) * K + k0 + c]))
-                                : 0.0;
+        cp_async_wait_all();
+        __syncthreads();  // the staged slice is visible, and the previous slice is no longer read
+        {
+            // A: 4 consecutive columns of one rank row per thread
+            const int jj = tid >> 4, c = 4 * (tid & 15);
+            const uint2 v = *reinterpret_cast<const uint2*>(&stA[jj][c]);
+            const bool live = jj < nj;
+            const double2 lo = make_double2(live ? static_cast<double>(bf16_bits_to_float(v.x & 0xffffu)) : 0.0,
+                                            live ? static_cast<double>(bf16_bits_to_float(v.x >> 16)) : 0.0);
+            const double2 hi = make_double2(live ? static_cast<double>(bf16_bits_to_float(v.y & 0xffffu)) : 0.0,
+                                            live ? static_cast<double>(bf16_bits_to_float(v.y >> 16)) : 0.0);
+            *reinterpret_cast<double2*>(&sA[jj][c]) = lo;
+            *reinterpret_cast<double2*>(&sA[jj][c + 2]) = hi;
         }
-        for (int i = tid; i < kMergeRanks * kMergeRows; i += 256) {
-            const int jj = i / kMergeRows, rr = i % kMergeRows;  // consecutive lanes: consecutive rows (no conflicts)
-            const int64_t n = n0 + rr;
-            sB[jj][rr] = (jj < nj && n < N) ? static_cast<double>(bf16_bits_to_float(B[n * r + j0 + jj])) : 0.0;
+        if (VEC_B) {
+            // B: the thread's own 8-rank piece, written transposed
+            const uint4 v = *reinterpret_cast<const uint4*>(&stB[b_rr][8 * b_h]);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            const bool row_live = n0 + b_rr < N;
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+                const int jj = 8 * b_h + t;
+                const uint32_t bits = (t & 1) ? (w[t >> 1] >> 16) : (w[t >> 1] & 0xffffu);
+                sB[jj][b_rr] = (row_live && jj < nj) ? static_cast<double>(bf16_bits_to_float(bits)) : 0.0;
+            }
+        } else {
+            for (int i = tid; i < kMergeRanks * kMergeRows; i += 256) {
+                const int jj = i / kMergeRows, rr = i % kMergeRows;  // consecutive lanes: consecutive rows
+                const int64_t n = n0 + rr;
+                sB[jj][rr] = (jj < nj && n < N) ? static_cast<double>(bf16_bits_to_float(B[n * r + j0 + jj])) : 0.0;
+            }
         }
-        __syncthreads();
+        __syncthreads();  // sA / sB hold the slice; the staging buffers are free
+        if (j0 + kMergeRanks < r) stage(j0 + kMergeRanks);  // lands while this slice is multiplied
         for (int jj = 0; jj < nj; ++jj) {
             const double2 a01 = *reinterpret_cast<const double2*>(&sA[jj][cb]);
             const double2 a23 = *reinterpret_cast<const double2*>(&sA[jj][32 + cb]);
@@ -131,7 +183,11 @@ cudaError_t launch_merge_lora(const uint8_t* codes, const int8_t* qscale, const 
     cfg.blockDim = dim3(256);
     cfg.stream = stream;
     TraceScope trace("nf4_merge_lora", stream);
-    return cudaLaunchKernelEx(&cfg, k_merge_lora, codes, qscale, scale2, scale_mean, absmax, A, B, r, N, K, s, out);
+    if (r % 8 == 0)
+        return cudaLaunchKernelEx(&cfg, k_merge_lora<true>, codes, qscale, scale2, scale_mean, absmax, A, B, r, N, K, s,
+                                  out);
+    return cudaLaunchKernelEx(&cfg, k_merge_lora<false>, codes, qscale, scale2, scale_mean, absmax, A, B, r, N, K, s,
+                              out);
 }
 
 }  // namespace nf4lora

@@ -2,8 +2,9 @@
 re-encoding (nf4_merge_requantize) with the oracle: the merged fp32 weight and
 the new encoding must match bit for bit (every step of the merge is a fixed
 sequence of IEEE operations, and the encoding is exact).  Cases cover a
-ragged row tile (d_out not a multiple of 128), a rank that is not a multiple
-of the 16-rank staging slice, the largest rank, products whose fp64 running
+ragged row tile (d_out not a multiple of 128), ranks that are not a multiple
+of the 16-rank staging slice (with and without whole 16-byte pieces of B's
+rows), the largest rank, products whose fp64 running
 sum must round, re-encoding in place and the LLaMA-7B q_proj size."""
 import numpy as np
 import pytest
@@ -38,7 +39,7 @@ def _assert_encoding_equal(dev, ref):
 
 
 @pytest.mark.parametrize("d_out,d_in,r,s", [(512, 512, 8, 2.0), (300, 448, 16, 0.25), (136, 192, 5, 1.0),
-                                            (64, 256, 256, 0.0625)])
+                                            (200, 320, 24, 0.5), (64, 256, 256, 0.0625)])
 def test_merge_bit_exact(nf, d_out, d_in, r, s):
     qt, enc, A, B = _setup(nf, d_out, d_in, r, index=d_out % 5)
     W_hat = oracle.dequantize(qt, (d_out, d_in))
