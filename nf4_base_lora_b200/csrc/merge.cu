@@ -16,7 +16,8 @@
 // factor slices of 16 ranks at a time are staged in shared memory as fp64
 // (B transposed), and each thread keeps 8 rows x 4 columns of fp64 sums; the
 // epilogue decodes the tile's codes (one 64-block per row) and writes fp32
-// rows.  The bf16 rows of the next slice travel by 16-byte asynchronous
+// rows (codes and block scales fetched into shared memory at the start).
+// The bf16 rows of the next slice travel by 16-byte asynchronous
 // copies into a staging buffer while the current slice is multiplied, so the
 // fp64 pipe does not wait for global loads between slices (B's rows are
 // copied this way when r is a multiple of 8, which makes every row of B start
@@ -59,6 +60,8 @@ __global__ void __launch_bounds__(256, 2) k_merge_lora(const uint8_t* __restrict
     __shared__ __align__(16) double sB[kMergeRanks][kMergeRows];  // B[n0 + rr][j0 + jj], transposed
     __shared__ __align__(16) uint16_t stA[kMergeRanks][kMergeCols];  // bf16 staging of the next slice of A
     __shared__ __align__(16) uint16_t stB[kMergeRows][kMergeRanks];  // and of B (VEC_B only), row-major
+    __shared__ __align__(16) uint8_t s_codes[kMergeRows][kMergeCols / 2];  // the tile's codes
+    __shared__ float s_sc[kMergeRows];  // fp32 scale of each row's block
     __shared__ float s_lvl[16];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid < 16) s_lvl[tid] = nf4_level(tid);
@@ -91,6 +94,23 @@ __global__ void __launch_bounds__(256, 2) k_merge_lora(const uint8_t* __restrict
 #pragma unroll
         for (int c = 0; c < 4; ++c) acc[i][c] = 0.0;
 
+    // the epilogue's inputs come in with the first slice: the tile's codes
+    // (32 bytes of each row, in the first slice's copy group) and each row's
+    // block scale
+    const int64_t bpr = K / 64, blk = k0 / 64;
+    {
+        const int rr = tid >> 1, h = tid & 1;
+        if (n0 + rr < N) cp_async16(&s_codes[rr][16 * h], codes + ((n0 + rr) * K + k0) / 2 + 16 * h);
+    }
+    if (tid < kMergeRows) {
+        const int64_t n = n0 + tid;
+        float sc = 0.0f;
+        if (n < N) {
+            const int64_t bi = n * bpr + blk;
+            sc = absmax ? absmax[bi] : nf4_block_scale(qscale[bi], scale2[bi >> 8], *scale_mean);
+        }
+        s_sc[tid] = sc;
+    }
     stage(0);
     for (int j0 = 0; j0 < r; j0 += kMergeRanks) {
         const int nj = min(kMergeRanks, r - j0);
@@ -147,18 +167,15 @@ __global__ void __launch_bounds__(256, 2) k_merge_lora(const uint8_t* __restrict
     }
 
     // epilogue: W_hat of the tile's block in each row, then the merged value
-    const float mu = absmax ? 0.0f : *scale_mean;
-    const int64_t bpr = K / 64, blk = k0 / 64;
     const double sd = static_cast<double>(s);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const int64_t n = n0 + rb + i;
         if (n >= N) break;
-        const int64_t bi = n * bpr + blk;
-        const float sc = absmax ? absmax[bi] : nf4_block_scale(qscale[bi], scale2[bi >> 8], mu);
+        const float sc = s_sc[rb + i];
         // codes of elements k0 + cb, + 1 and k0 + 32 + cb, + 1 of row n: one byte
         // each, the even element in the high nibble
-        const uint8_t* row = codes + (n * K + k0) / 2;
+        const uint8_t* row = s_codes[rb + i];
         const uint32_t b0 = row[cb / 2], b1 = row[16 + cb / 2];
         const uint32_t code[4] = {b0 >> 4, b0 & 15u, b1 >> 4, b1 & 15u};
         float o[4];
