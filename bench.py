@@ -781,16 +781,38 @@ def time_workload(nf, wl, args, stream, device, world, peaks, l2, with_e2e):
     tflops = world * step_flops / (ms_per_step * 1e-3) / 1e12
 
     # per-kernel device times: a separate pass of the same steps with the
-    # library's launch tracing on (event pairs around each launch, eager)
-    k_eager = max(cycle, min(args.steps, 50))
-    nf.trace_start(int(launches_per_step) * k_eager + 64)
-    with torch.cuda.stream(stream):
-        for i in range(k_eager):
-            enqueue(args.warmup + i)
-    torch.cuda.synchronize()
-    records = nf.trace_records()
-    nf.trace_stop()
-    timing_source = "traced eager pass of %d steps right after the timed region" % k_eager
+    # library's launch tracing on (an event pair around each launch).  With
+    # graphs, the traced steps are captured too (the events become
+    # event-record nodes) and replayed, so no host launch latency falls
+    # between a pair; otherwise the traced steps run eagerly.
+    if graphs and exchange is None:
+        nf.trace_start(int(launches_per_step) * cycle + 64)
+        traced = []
+        for g in range(cycle):
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=stream):
+                gw.step(g * len(plan))
+            traced.append(graph)
+        with torch.cuda.stream(stream):
+            for _ in range(2):  # the records hold the second replay's times
+                for graph in traced:
+                    graph.replay()
+        torch.cuda.synchronize()
+        records = nf.trace_records()
+        nf.trace_stop()
+        del traced
+        timing_source = ("traced graph replay of %d steps right after the timed region (an event-record node "
+                         "before and after each launch)" % cycle)
+    else:
+        k_eager = max(cycle, min(args.steps, 50))
+        nf.trace_start(int(launches_per_step) * k_eager + 64)
+        with torch.cuda.stream(stream):
+            for i in range(k_eager):
+                enqueue(args.warmup + i)
+        torch.cuda.synchronize()
+        records = nf.trace_records()
+        nf.trace_stop()
+        timing_source = "traced eager pass of %d steps right after the timed region" % k_eager
     hbm = not tensor_bound(wl)
     names = ("nf4_gemm_fwd_few", "nf4_gemm_dx_few") if hbm else ("nf4_gemm_fwd", "nf4_gemm_dx")
     dom, kstats = dominant_kernel_stats(records, names)

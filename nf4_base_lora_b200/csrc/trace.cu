@@ -35,6 +35,17 @@ void destroy_pool() {
     g_used = 0;
 }
 
+// Inside a stream capture a plain record only marks a point for the capture's
+// own dependency tracking; the external flag makes it an event-record node of
+// the graph, which records the event at every replay.
+void record(cudaEvent_t ev, cudaStream_t stream) {
+    cudaStreamCaptureStatus st = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &st) == cudaSuccess && st == cudaStreamCaptureStatusActive)
+        cudaEventRecordWithFlags(ev, stream, cudaEventRecordExternal);
+    else
+        cudaEventRecord(ev, stream);
+}
+
 }  // namespace
 
 int trace_begin(const char* name, cudaStream_t stream) {
@@ -44,14 +55,14 @@ int trace_begin(const char* name, cudaStream_t stream) {
     if (g_used >= static_cast<int>(g_pool.size())) return -1;
     const int slot = g_used++;
     g_pool[slot].name = name;
-    cudaEventRecord(g_pool[slot].start, stream);
+    record(g_pool[slot].start, stream);
     return slot;
 }
 
 void trace_end(int slot, cudaStream_t stream) {
     if (slot < 0) return;
     std::lock_guard<std::mutex> lk(g_mu);
-    if (slot < static_cast<int>(g_pool.size())) cudaEventRecord(g_pool[slot].stop, stream);
+    if (slot < static_cast<int>(g_pool.size())) record(g_pool[slot].stop, stream);
 }
 
 }  // namespace nf4lora

@@ -1,6 +1,7 @@
 // Launch tracing: while enabled, every kernel the library launches is
 // bracketed by two CUDA events recorded on its stream.  Inside a stream
-// capture the records become graph nodes and are refreshed at each replay.
+// capture the records become event-record nodes of the graph (recorded with
+// the external flag), so each replay records them again.
 #pragma once
 
 #include <cuda_runtime.h>
